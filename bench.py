@@ -1,0 +1,441 @@
+#!/usr/bin/env python
+"""Benchmark of the greedy MoE speculative-verify step on B200.
+
+One step = the whole hot path over one batch: 32 sequences x (K+1 = 4) token
+rows through 12 MoE layers (router top-6 of 64 routed experts + 2 shared,
+SwiGLU experts, residual combine), the 129,280-token LM-head argmax and greedy
+acceptance -- the concurrency-32 decode verify workload (hidden 1280, expert
+intermediate 896, shared 1792).  Inputs are seeded synthetic bf16 tensors
+(weights N(0, 0.02^2), hidden states N(0, 1)); drafts copy the verifier's own
+argmax with probability 0.576, else a uniform token id.
+
+Prints ONE JSON line (rank 0).  `value` = committed tokens (accepted + 1 per
+sequence) per second over all ranks, device-timed with CUDA events, inputs
+resident in HBM.  `e2e` = the same metric through the public API with the
+step's inputs copied from pinned host memory and its results read back inside
+the timed region.  Multi-GPU (torchrun): independent replicas, one batch per
+rank, no collective on the data path (weak scaling); time = max over ranks.
+
+--impl reference times the CPU oracle (test infrastructure, plain C++ loops)
+on the host cores, each step a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from moe_decoder_speculative_b200 import workloads as wl  # noqa: E402
+
+METRIC = "verified tokens/s per MoE verify step at 32x(K+1) rows"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=2, help="workload id (default: concurrency-32 verify)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        try:
+            d = json.load(open(p))
+            return float(d["hbm_gbs"]), "measured"
+        except Exception:
+            pass
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest(files):
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+GEMM_SOURCES = ["moe_decoder_speculative_b200/csrc/gemm_tc.cu", "moe_decoder_speculative_b200/csrc/mv_device.cuh"]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary, if the
+    summary was taken on the current kernel source (else None)."""
+    digest = source_digest(GEMM_SOURCES)
+    pat = re.compile(r"traffic\[(\w+)\]:\s*bytes_per_launch=(\d+)\s+source=(\w+)")
+    for f in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for line in open(f):
+            m = pat.search(line)
+            if m and m.group(1) == kernel and m.group(3) == digest:
+                return int(m.group(2))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+            if self.gpu_id:
+                cmd += ["-i", self.gpu_id]
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_uuid(torch, dev):
+    try:
+        u = torch.cuda.get_device_properties(dev).uuid
+        s = str(u)
+        return s if s.startswith("GPU-") else "GPU-" + s
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (what the method must move per launch)
+# ---------------------------------------------------------------------------
+
+def algorithmic_bytes(w, touched, T):
+    """Per-launch algorithmic bytes of each kernel kind for one verify step.
+    touched[l] = distinct routed experts chosen in layer l."""
+    H, I, Ish, k, V, E = w.H, w.I, w.I_sh, w.k, w.V, w.E
+    n = T * k
+    L = len(touched)
+    avg_t = float(np.mean(touched)) if L else 0.0
+    return {
+        "grouped_swiglu_gemm": avg_t * 2 * I * H * 2 + 2 * Ish * H * 2 + (n + T) * H * 2 + (n * I + T * Ish) * 2,
+        "grouped_down_gemm": avg_t * H * I * 2 + H * Ish * 2 + (n * I + T * Ish) * 2 + (n + T) * H * 4,
+        "lm_head_gemm_argmax": V * H * 2 + T * H * 2 + ((V + 127) // 128 * 4) * T * 8,
+        "router_topk": E * H * 2 + T * H * 2 + T * k * 8,
+        "expert_permute": n * 4 * 3 + n * H * 2 * 2,
+        "combine_unpermute": n * H * 4 + T * H * 4 + T * H * 2 * 2 + n * 12,
+    }
+
+
+def step_algorithmic_bytes(w, touched, T):
+    H, I, Ish, k, V, E = w.H, w.I, w.I_sh, w.k, w.V, w.E
+    per_layer = [t * 3 * I * H * 2 + 3 * Ish * H * 2 + E * H * 2 for t in touched]
+    return sum(per_layer) + V * H * 2 + 2 * T * H * 2
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle runs (baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_step(oracle, w, inp, drafts, S):
+    rows = S * (w.K + 1)
+    st = oracle.verify_step(inp["hidden"][:rows], drafts[:S], S, w.K, inp["layers"], w.k, inp["w_lm"])
+    return int(np.sum(st["accepted"] + 1))
+
+
+def oracle_sample_size(oracle, w, inp, budget_s):
+    """Sequences per oracle step so that one step takes about budget_s seconds."""
+    t0 = time.perf_counter()
+    lay = inp["layers"][0]
+    x = inp["hidden"]
+    idx, tw, _, _ = oracle.router(x, lay["w_router"], w.k)
+    oracle.moe_ffn(x, lay, idx, tw, residual=x)
+    t_layer = time.perf_counter() - t0            # one layer on all T rows
+    t_full = (w.L + 6.0) * t_layer                # + LM head ~ 6 layers of work per row
+    S = w.B if t_full <= budget_s else max(1, int(w.B * budget_s / t_full))
+    return S, t_full
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    w = wl.workload(args.workload)
+    inp = wl.make_inputs(w)
+    # drafts copy the oracle's own argmax (one oracle LM pass on the final h of a short sample)
+    S, t_full = oracle_sample_size(oracle, w, inp, budget_s=max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup))))
+    rows = S * (w.K + 1)
+    st = oracle.verify_step(inp["hidden"][:rows], np.zeros((S, w.K), np.int32), S, w.K, inp["layers"], w.k,
+                            inp["w_lm"])
+    am = np.concatenate([st["argmax"], np.zeros((w.B - S) * (w.K + 1), np.int32)])
+    drafts = wl.make_drafts(w, am)
+    for _ in range(args.warmup):
+        oracle_step(oracle, w, inp, drafts, S)
+    t0 = time.perf_counter()
+    committed = 0
+    for _ in range(args.steps):
+        committed += oracle_step(oracle, w, inp, drafts, S)
+    dt = time.perf_counter() - t0
+    value = committed / dt
+    cores = oracle.num_threads()
+    sample = f"{S} of {w.B} sequences ({rows} rows) x {w.L} layers + LM head + accept per step"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": {"workload": w.name, "B": w.B, "K": w.K, "rows": w.T, "layers": w.L,
+                                         "sampled_sequences": S},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from moe_decoder_speculative_b200 import binding as bd
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = wl.workload(args.workload)
+    assert w.has_verify, "the benchmark times the verify step"
+    inp = wl.make_inputs(w)
+    if rank > 0:   # each replica verifies its own batch of sequences
+        inp["hidden"] = wl.normal_bf16(np.random.SeedSequence([w.id, rank]), (w.T, w.H), w.x_std)
+    shape = bd.shape_of(w)
+    layers = [bd.LayerWeights(l, dev) for l in inp["layers"]]
+    w_lm = bd.bf16_to_device(inp["w_lm"], dev)
+    hidden = bd.bf16_to_device(inp["hidden"], dev)
+    plan = bd.VerifyPlan(shape, layers, w_lm, w.B, w.K, dev)
+    T = w.T
+
+    # drafts: the verifier's own argmax (one untimed pass) copied with p = 0.576
+    zero = torch.zeros((w.B, w.K), dtype=torch.int32, device=dev)
+    _, _, _, am = plan(hidden, zero)
+    drafts_np = wl.make_drafts(w, am.cpu().numpy())
+    drafts = torch.from_numpy(drafts_np).to(dev)
+
+    # touched experts per layer (for the algorithmic byte count), via the public per-step calls
+    touched = []
+    h = hidden
+    for lw in layers:
+        idx, tw = bd.moe_router_topk(h, shape, lw.t["w_router"], lw.t["router_bias"])
+        touched.append(int(torch.unique(idx).numel()))
+        h = bd.moe_ffn_forward(h, shape, lw, idx, tw, residual=h)
+    plan.sync_status()
+
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        plan(hidden, drafts)
+    torch.cuda.synchronize()
+    acc, _, _, _ = plan(hidden, drafts)
+    committed_per_step = int((acc + 1).sum().item())
+
+    with ClockSampler(gpu_uuid(torch, dev)) as clocks:
+        # ---- headline: device-timed K steps, inputs resident ----
+        barrier()
+        torch.cuda.synchronize()
+        n0 = bd.launch_count()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            plan(hidden, drafts)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        launches = bd.launch_count() - n0
+        ms = ev0.elapsed_time(ev1)
+        plan.sync_status()
+
+        # ---- per-kernel durations: the same K steps with an event pair around every launch ----
+        barrier()
+        torch.cuda.synchronize()
+        bd.profile_enable(True)
+        ev2, ev3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev2.record(stream)
+        for _ in range(args.steps):
+            plan(hidden, drafts)
+        ev3.record(stream)
+        torch.cuda.synchronize()
+        bd.profile_enable(False)
+        kern = bd.profile_collect()
+        ms_instr = ev2.elapsed_time(ev3)
+        barrier()
+
+        # ---- end to end through the public API with host buffers ----
+        hid_h = torch.from_numpy(inp["hidden"].view(np.int16)).pin_memory()
+        dr_h = torch.from_numpy(drafts_np).pin_memory()
+        hid_d = torch.empty_like(hid_h, device=dev)
+        dr_d = torch.empty_like(dr_h, device=dev)
+        acc_h = torch.empty(w.B, dtype=torch.int32).pin_memory()
+        nxt_h = torch.empty(w.B, dtype=torch.int32).pin_memory()
+        em_h = torch.empty((w.B, w.K + 1), dtype=torch.int32).pin_memory()
+        barrier()
+        torch.cuda.synchronize()
+        ev4, ev5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev4.record(stream)
+        for _ in range(args.steps):
+            hid_d.copy_(hid_h, non_blocking=True)
+            dr_d.copy_(dr_h, non_blocking=True)
+            a, nx, em, _ = plan(hid_d.view(torch.bfloat16), dr_d)
+            acc_h.copy_(a, non_blocking=True)
+            nxt_h.copy_(nx, non_blocking=True)
+            em_h.copy_(em, non_blocking=True)
+        ev5.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = ev4.elapsed_time(ev5)
+        barrier()
+    clk = clocks.summary()
+
+    if world > 1:
+        t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, ms_e2e = float(t[0]), float(t[1])
+        c = torch.tensor([committed_per_step], dtype=torch.int64, device=dev)
+        dist.all_reduce(c, op=dist.ReduceOp.SUM)
+        committed_all = int(c.item())
+    else:
+        committed_all = committed_per_step
+
+    K = args.steps
+    value = committed_all * K / (ms / 1e3)
+    e2e_value = committed_all * K / (ms_e2e / 1e3)
+    peak, peak_kind = measured_peaks()
+    alg = algorithmic_bytes(w, touched, T)
+    kernels = {}
+    for name, d in kern.items():
+        if d["launches"] == 0:
+            continue
+        avg_s = d["ms"] / d["launches"] / 1e3
+        entry = {"launches": d["launches"], "avg_us": round(avg_s * 1e6, 3),
+                 "share": round(d["ms"] / max(1e-9, sum(x["ms"] for x in kern.values())), 4)}
+        if name in alg:
+            entry["alg_bytes"] = int(alg[name])
+            entry["gbs"] = round(alg[name] / avg_s / 1e9, 1)
+        kernels[name] = entry
+    dom = max(kernels, key=lambda n: kern[n]["ms"])
+    dom_avg_s = kern[dom]["ms"] / kern[dom]["launches"] / 1e3
+    achieved = alg[dom] / dom_avg_s / 1e9
+    traffic = ncu_traffic(dom)
+    step_bytes = step_algorithmic_bytes(w, touched, T)
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded bf16 weights N(0,0.02^2), hidden N(0,1); drafts copy the "
+                                  "verifier argmax w.p. 0.576)",
+        "config": {"workload": w.name, "B": w.B, "K": w.K, "rows": T, "layers": w.L, "H": w.H, "E": w.E,
+                   "top_k": w.k, "I": w.I, "I_shared": w.I_sh, "V": w.V,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "weights (5.8 GB) far larger than L2: no flush needed"},
+        "rows_per_s": world * T * K / (ms / 1e3),
+        "committed_per_step": committed_all,
+        "step_roofline": {"alg_bytes": int(step_bytes), "achieved_gbs": round(step_bytes / (ms / K / 1e3) / 1e9, 1),
+                          "peak_gbs": peak, "frac": round(step_bytes / (ms / K / 1e3) / 1e9 / peak, 4)},
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "peak_source": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "alg_bytes_per_launch": int(alg[dom])},
+        "kernels": kernels,
+        "instrumented_ms_per_step": ms_instr / K,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(hid_h.numel() * 2 + dr_h.numel() * 4),
+                "d2h_bytes_per_step": int(acc_h.numel() * 4 + nxt_h.numel() * 4 + em_h.numel() * 4)},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "touched_experts": touched,
+    }
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        S, _ = oracle_sample_size(oracle, w, inp, budget_s=20.0)
+        t0 = time.perf_counter()
+        committed = oracle_step(oracle, w, inp, drafts_np, S)
+        dt = time.perf_counter() - t0
+        out["cpu_baseline"] = {"value": committed / dt, "unit": UNIT, "cores": oracle.num_threads(),
+                               "kind": "oracle",
+                               "sample": f"{S} of {w.B} sequences ({S * (w.K + 1)} rows) x {w.L} layers + LM head + "
+                                         f"accept, one pass, {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(out))
+    plan = None
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

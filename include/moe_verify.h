@@ -1,0 +1,239 @@
+/*
+ * moe_verify.h - C ABI of the B200 (sm_100a) greedy MoE speculative-verify step.
+ *
+ * The step verifies K draft tokens per sequence for the mixture-of-experts
+ * decoder of jina-ocr-v1.  Shapes and the method come from the jina-ocr-v1
+ * model card (jina.ai/models/jina-ocr-v1):
+ *   - architecture paragraph: 12 decoder layers, hidden 1280, 64 routed
+ *     experts plus 2 shared under top-6 routing, 129,280-token vocabulary;
+ *   - decoding-speed paragraph and introduction: K drafts (K=3) are checked
+ *     greedily, so the output equals plain autoregressive decoding, and up to
+ *     K+1 tokens are committed per verifier pass;
+ *   - usage paragraph: turning speculation off (K = 0) leaves the text as is.
+ * and from the tldrocket write-up "Jina AI Releases jina-ocr-v1 ...",
+ * speculative paragraph: the decoder keeps only the drafts that match its
+ * own choice.
+ *
+ * Conventions for every call below
+ *   Memory      All tensor pointers are DEVICE pointers owned by the caller.
+ *               bf16 tensors are passed as uint16_t bit patterns.  The
+ *               library never allocates device memory on these paths; the
+ *               scratch space it needs is the caller's workspace, sized by the
+ *               matching *_workspace_size() call.
+ *   Layout      Row-major, densely packed, in the shapes given per argument.
+ *               Token rows of a verify step are sequence-major:
+ *               row r = b*(K+1) + j, j = 0 the current token, j = 1..K draft j.
+ *   Alignment   Every pointer must be 16-byte aligned (MV_ERR_MISALIGNED).
+ *               H, I and I_shared must be multiples of 64 and V a multiple
+ *               of 8 (MV_ERR_UNSUPPORTED_SHAPE).  Limits: E <= 256,
+ *               1 <= k <= min(E, 8).
+ *   Streams     Every call is asynchronous on the given stream (NULL = the
+ *               legacy default stream).  Argument checks happen on the host
+ *               before anything is launched; a call that returns an error
+ *               launched nothing.  A launch failure returns MV_ERR_CUDA.
+ *   Device      Waits inside the library's kernels are bounded; a wait that
+ *   errors      runs out records MV_ERR_TIMEOUT in a sticky error word that
+ *               lives in the workspace.  mv_sync_status() reads and clears it.
+ *   Errors      mv_last_error() gives a message for the last non-OK status
+ *               returned on the calling thread.  No C++ exception crosses
+ *               this interface.
+ *   Determinism Every result is a deterministic function of the inputs: no
+ *               floating-point atomics, and the same row gives the same bits
+ *               whatever other rows share its batch.
+ */
+#ifndef MOE_VERIFY_H
+#define MOE_VERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MV_API __attribute__((visibility("default")))
+#else
+#define MV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st* mv_stream_t;
+
+typedef enum {
+  MV_OK = 0,
+  MV_ERR_INVALID_ARG = 1,         /* null pointer, negative size, bad k/E/K */
+  MV_ERR_UNSUPPORTED_SHAPE = 2,   /* H/I/I_shared not multiples of 64, V not of 8, limits */
+  MV_ERR_MISALIGNED = 3,          /* a pointer is not 16-byte aligned */
+  MV_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes below the *_workspace_size() value */
+  MV_ERR_CUDA = 5,                /* a CUDA runtime call or launch failed */
+  MV_ERR_TIMEOUT = 6,             /* a bounded device-side wait ran out */
+  MV_ERR_INTERNAL = 7             /* a device-side consistency check failed */
+} mv_status;
+
+/* Shape of one MoE layer.  I_shared = 0 means no shared expert.  The model
+ * card's "2 shared" experts are passed as one always-on SwiGLU of
+ * I_shared = 2*I whose gate/up rows and down columns are the two concatenated;
+ * that is exactly the sum of the two experts' outputs. */
+typedef struct {
+  int32_t H;        /* hidden size (1280) */
+  int32_t E;        /* routed experts (64) */
+  int32_t I;        /* routed expert intermediate size (896) */
+  int32_t I_shared; /* shared intermediate size (1792), or 0 */
+  int32_t k;        /* experts kept per token (6) */
+} mv_moe_shape;
+
+/* Device pointers to one layer's weights (bf16 bits unless noted). */
+typedef struct {
+  const uint16_t* w_router;  /* [E][H] */
+  const float* router_bias;  /* [E] fp32 added to the router logits, or NULL */
+  const uint16_t* w_gate;    /* [E][I][H] */
+  const uint16_t* w_up;      /* [E][I][H] */
+  const uint16_t* w_down;    /* [E][H][I] */
+  const uint16_t* ws_gate;   /* [I_shared][H]  (NULL when I_shared == 0) */
+  const uint16_t* ws_up;     /* [I_shared][H] */
+  const uint16_t* ws_down;   /* [H][I_shared] */
+} mv_moe_weights;
+
+/* ---------------------------------------------------------------------------
+ * moe_router_topk - router of one MoE layer (model card, architecture
+ * paragraph: "64 routed experts ... under top-6 routing").
+ * For every row r: logits l[e] = x[r] . w_router[e] (+ router_bias[e]) in
+ * fp32; the k largest logits are kept (equal logits: lower expert id first),
+ * slot j holding the j-th largest; topk_w[r][j] = softmax over all E logits
+ * restricted to the kept experts and renormalised to sum 1.
+ *   x          [T][H] bf16           topk_idx  [T][k] int32 (out)
+ *   w_router   [E][H] bf16           topk_w    [T][k] fp32  (out)
+ *   router_bias [E] fp32 or NULL
+ * T = 0 is legal and launches nothing.
+ * ------------------------------------------------------------------------- */
+MV_API mv_status moe_router_topk(const uint16_t* x, int32_t T, const mv_moe_shape* shape,
+                          const uint16_t* w_router, const float* router_bias,
+                          int32_t* topk_idx, float* topk_w, mv_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_expert_permute - group the (row, slot) routing entries by expert.
+ * Entry id i = r*k + j.  counts[e] = number of entries routed to e;
+ * offsets[e] = sum of counts[e'] for e' < e, offsets[E] = T*k; perm lists the
+ * entry ids grouped by expert, ascending within each expert; inv[i] is the
+ * position of entry i in perm.  Integer, exact, deterministic.
+ *   topk_idx [T][k] int32 in [0, E)   counts [E], offsets [E+1],
+ *                                      perm [T*k], inv [T*k]  int32 (out)
+ * ------------------------------------------------------------------------- */
+MV_API mv_status moe_expert_permute(const int32_t* topk_idx, int32_t T, int32_t E, int32_t k,
+                             int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                             mv_stream_t stream);
+
+/* Bytes of workspace moe_ffn_forward needs for T rows. */
+MV_API size_t moe_ffn_workspace_size(int32_t T, const mv_moe_shape* shape);
+
+/* ---------------------------------------------------------------------------
+ * moe_ffn_forward - one MoE FFN layer given its routing.
+ * For every row r: m[r] = sum_j topk_w[r][j] * SwiGLU_{topk_idx[r][j]}(x[r])
+ *                        + SwiGLU_shared(x[r]),
+ * SwiGLU_e(x) = W_down[e] . bf16(silu(W_gate[e] . x) * (W_up[e] . x)),
+ * products in bf16 x bf16 -> fp32, the activation rounded to bf16 once.
+ * out[r] = bf16(residual[r] + m[r]), or bf16(m[r]) when residual is NULL.
+ *   x, residual, out [T][H] bf16 (out may not alias x; it may alias residual)
+ *   topk_idx [T][k] int32, topk_w [T][k] fp32 (e.g. from moe_router_topk)
+ *   ws / ws_bytes: caller-owned device workspace, >= moe_ffn_workspace_size().
+ * Grouping by expert, the grouped tensor-core GEMMs and the combine all run
+ * on the stream; nothing returns to the host.
+ * ------------------------------------------------------------------------- */
+MV_API mv_status moe_ffn_forward(const uint16_t* x, int32_t T, const mv_moe_shape* shape,
+                          const mv_moe_weights* weights, const int32_t* topk_idx,
+                          const float* topk_w, const uint16_t* residual, uint16_t* out,
+                          void* ws, size_t ws_bytes, mv_stream_t stream);
+
+/* Bytes of workspace lm_head_argmax needs for T rows and a V-token vocabulary. */
+MV_API size_t lm_head_workspace_size(int32_t T, int32_t V);
+
+/* ---------------------------------------------------------------------------
+ * lm_head_argmax - the verifier's own greedy choice per row (model card,
+ * architecture paragraph: 129,280-token vocabulary; write-up, speculative
+ * paragraph: drafts are kept only where they match the decoder's choice).
+ * argmax[r] = argmax_v  h[r] . w_lm[v]  (fp32 logits; equal logits: the lower
+ * v wins; -0 and +0 are equal).  The logits are never written to memory.
+ *   h [T][H] bf16, w_lm [V][H] bf16, argmax [T] int32 (out)
+ * ------------------------------------------------------------------------- */
+MV_API mv_status lm_head_argmax(const uint16_t* h, int32_t T, int32_t H, const uint16_t* w_lm,
+                         int32_t V, int32_t* argmax, void* ws, size_t ws_bytes,
+                         mv_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * greedy_accept - greedy acceptance of K drafts per sequence (model card,
+ * introduction and decoding-speed paragraph; write-up, speculative paragraph).
+ * With g = argmax[b*(K+1) .. b*(K+1)+K] and d = drafts[b][0..K-1]:
+ *   accepted[b]   = largest a <= K with d[i] == g[i] for every i < a
+ *   next_token[b] = g[a]
+ *   emitted[b][j] = g[j] for j <= a, -1 for j > a  (emitted may be NULL)
+ * so accepted[b] + 1 tokens are committed.  K = 0 is plain greedy decoding.
+ * Draft ids outside [0, V) are legal and never match.
+ *   argmax [B][K+1], drafts [B][K] (NULL allowed when K = 0), outputs int32.
+ * ------------------------------------------------------------------------- */
+MV_API mv_status greedy_accept(const int32_t* argmax, const int32_t* drafts, int32_t B, int32_t K,
+                        int32_t* accepted, int32_t* next_token, int32_t* emitted,
+                        mv_stream_t stream);
+
+/* Bytes of workspace verify_step needs. */
+MV_API size_t verify_step_workspace_size(int32_t B, int32_t K, const mv_moe_shape* shape, int32_t V);
+
+/* ---------------------------------------------------------------------------
+ * verify_step - the whole greedy speculative-verify step, fused into one
+ * stream of launches with no host synchronisation:
+ *   h_0 = hidden;  for l < n_layers:  route h_l (moe_router_topk with
+ *   layers[l]), h_{l+1} = bf16(h_l + MoE_l(h_l)) (moe_ffn_forward with the
+ *   residual);  g = lm_head_argmax(h_L);  greedy_accept(g, drafts).
+ * The residual add between layers is a reading of the pages (they name no
+ * norms or residuals); n_layers = 12 is the model card's decoder depth.
+ *   hidden  [B*(K+1)][H] bf16, not modified     drafts [B][K] int32
+ *   layers  HOST array of n_layers weight sets (device pointers inside)
+ *   w_lm    [V][H] bf16
+ *   accepted, next_token [B]; emitted [B][K+1] (nullable); argmax [B*(K+1)]
+ *   (nullable: the verifier's choice for every row) - all int32 outputs.
+ * ------------------------------------------------------------------------- */
+MV_API mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, int32_t K,
+                      const mv_moe_shape* shape, const mv_moe_weights* layers,
+                      int32_t n_layers, const uint16_t* w_lm, int32_t V, int32_t* accepted,
+                      int32_t* next_token, int32_t* emitted, int32_t* argmax, void* ws,
+                      size_t ws_bytes, mv_stream_t stream);
+
+/* Clears the workspace's header (its sticky error word) on the stream.  Call
+ * once on a freshly allocated workspace before its first use (a workspace
+ * allocated zero-filled needs no call). */
+MV_API mv_status mv_workspace_init(void* ws, size_t ws_bytes, mv_stream_t stream);
+
+/* Synchronises the stream, then reads and clears the sticky device error
+ * word kept in a workspace used by moe_ffn_forward, lm_head_argmax or
+ * verify_step.  Returns MV_OK, MV_ERR_TIMEOUT, MV_ERR_INTERNAL or MV_ERR_CUDA. */
+MV_API mv_status mv_sync_status(void* ws, mv_stream_t stream);
+
+/* Message for the last non-OK status returned on the calling thread. */
+MV_API const char* mv_last_error(void);
+
+/* Library version string. */
+MV_API const char* mv_version(void);
+
+/* ---------------------------------------------------------------------------
+ * Instrumentation (off the hot path unless enabled).
+ * mv_launch_count: kernels this library has launched in the process.
+ * mv_profile_enable(1) brackets every subsequent kernel launch with CUDA
+ * events on its stream; mv_profile_collect synchronises those events and
+ * writes, per kernel kind (see mv_kernel_name), the number of launches and
+ * the summed device milliseconds, then clears the record.  n_kinds is the
+ * array length; returns the number of kinds written.
+ * ------------------------------------------------------------------------- */
+MV_API uint64_t mv_launch_count(void);
+MV_API void mv_profile_enable(int32_t on);
+MV_API int32_t mv_profile_collect(int64_t* launches, double* total_ms, int32_t n_kinds);
+MV_API const char* mv_kernel_name(int32_t kind);
+
+/* Test hook: the bound, in nanoseconds, on every device-side wait of later
+ * launches (default 2e9).  Values <= 0 restore the default. */
+MV_API void mv_set_wait_timeout_ns(int64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_VERIFY_H */

@@ -6,14 +6,12 @@ thin ctypes layer over it; ``workloads`` draws the seeded synthetic inputs.
 Importing this package does not load the CUDA library; the first call into
 ``binding`` does, and fails loudly if it is missing.
 """
-__all__ = ["binding", "workloads"]
+import importlib
+
+__all__ = ["binding", "workloads", "build"]
 
 
 def __getattr__(name):
-    if name == "binding":
-        from . import binding
-        return binding
-    if name == "workloads":
-        from . import workloads
-        return workloads
+    if name in __all__:
+        return importlib.import_module(f"{__name__}.{name}")
     raise AttributeError(name)

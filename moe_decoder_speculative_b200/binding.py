@@ -1,0 +1,279 @@
+"""ctypes binding over libmoe_verify.so (include/moe_verify.h).
+
+Argument marshalling only: every step of the verify path runs in the
+library's CUDA kernels.  Tensors are torch CUDA tensors used as plain device
+memory (bf16 data may be torch.bfloat16 or any 2-byte dtype holding the bf16
+bits); the stream is torch's current stream unless one is given.  There is no
+CPU fallback: if the library is not built, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libmoe_verify.so")
+
+MV_OK = 0
+STATUS_NAMES = {0: "MV_OK", 1: "MV_ERR_INVALID_ARG", 2: "MV_ERR_UNSUPPORTED_SHAPE", 3: "MV_ERR_MISALIGNED",
+                4: "MV_ERR_WORKSPACE_TOO_SMALL", 5: "MV_ERR_CUDA", 6: "MV_ERR_TIMEOUT", 7: "MV_ERR_INTERNAL"}
+EXPORTED = ["moe_router_topk", "moe_expert_permute", "moe_ffn_workspace_size", "moe_ffn_forward",
+            "lm_head_workspace_size", "lm_head_argmax", "greedy_accept", "verify_step_workspace_size",
+            "verify_step", "mv_workspace_init", "mv_sync_status", "mv_last_error", "mv_version",
+            "mv_launch_count", "mv_profile_enable", "mv_profile_collect", "mv_kernel_name",
+            "mv_set_wait_timeout_ns"]
+
+
+class MVError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class MoeShape(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int32), ("E", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("I_shared", ctypes.c_int32), ("k", ctypes.c_int32)]
+
+
+class MoeWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w_router", "router_bias", "w_gate", "w_up", "w_down",
+                                                "ws_gate", "ws_up", "ws_down")]
+
+
+_lib = None
+
+
+def lib():
+    """Load the shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m moe_decoder_speculative_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        S, W = ctypes.POINTER(MoeShape), ctypes.POINTER(MoeWeights)
+        sig = {
+            "moe_router_topk": (i32, [P, i32, S, P, P, P, P, P]),
+            "moe_expert_permute": (i32, [P, i32, i32, i32, P, P, P, P, P]),
+            "moe_ffn_workspace_size": (sz, [i32, S]),
+            "moe_ffn_forward": (i32, [P, i32, S, W, P, P, P, P, P, sz, P]),
+            "lm_head_workspace_size": (sz, [i32, i32]),
+            "lm_head_argmax": (i32, [P, i32, i32, P, i32, P, P, sz, P]),
+            "greedy_accept": (i32, [P, P, i32, i32, P, P, P, P]),
+            "verify_step_workspace_size": (sz, [i32, i32, S, i32]),
+            "verify_step": (i32, [P, P, i32, i32, S, W, i32, P, i32, P, P, P, P, P, sz, P]),
+            "mv_workspace_init": (i32, [P, sz, P]),
+            "mv_sync_status": (i32, [P, P]),
+            "mv_last_error": (ctypes.c_char_p, []),
+            "mv_version": (ctypes.c_char_p, []),
+            "mv_launch_count": (ctypes.c_uint64, []),
+            "mv_profile_enable": (None, [i32]),
+            "mv_profile_collect": (i32, [P, P, i32]),
+            "mv_kernel_name": (ctypes.c_char_p, [i32]),
+            "mv_set_wait_timeout_ns": (None, [i64]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != MV_OK:
+        raise MVError(status, lib().mv_last_error().decode())
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _shape(H, E, I, I_shared, k):
+    return MoeShape(int(H), int(E), int(I), int(I_shared), int(k))
+
+
+def shape_of(w) -> MoeShape:
+    """MoeShape from an object with H, E, I, I_sh, k attributes (e.g. a Workload)."""
+    return _shape(w.H, w.E, w.I, w.I_sh, w.k)
+
+
+# ---------------------------------------------------------------------------
+# host <-> device helpers (plumbing)
+# ---------------------------------------------------------------------------
+
+def bf16_to_device(a: np.ndarray, device="cuda") -> torch.Tensor:
+    """uint16 bf16 bits (numpy) -> torch.bfloat16 tensor on the device."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint16).view(np.int16))
+    return t.to(device).view(torch.bfloat16)
+
+
+def bf16_from_device(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+class LayerWeights:
+    """Device copies of one MoE layer's weights plus the C struct pointing at them."""
+
+    def __init__(self, layer: dict, device="cuda"):
+        self.t = {}
+        for n in ("w_router", "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down"):
+            v = layer.get(n)
+            self.t[n] = None if v is None else (v if isinstance(v, torch.Tensor) else bf16_to_device(v, device))
+        b = layer.get("router_bias")
+        self.t["router_bias"] = None if b is None else (
+            b if isinstance(b, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(b, np.float32)).to(device))
+        self.c = MoeWeights(*[None if self.t[n] is None else self.t[n].data_ptr()
+                              for n, _ in MoeWeights._fields_])
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A zero-filled device workspace (its error header starts cleared)."""
+    return torch.zeros(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------------------
+# the C-ABI calls
+# ---------------------------------------------------------------------------
+
+def moe_router_topk(x, shape: MoeShape, w_router, router_bias=None, topk_idx=None, topk_w=None, stream=None):
+    T = x.shape[0]
+    dev = x.device
+    if topk_idx is None:
+        topk_idx = torch.empty((T, shape.k), dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty((T, shape.k), dtype=torch.float32, device=dev)
+    _check(lib().moe_router_topk(_p(x), T, ctypes.byref(shape), _p(w_router), _p(router_bias), _p(topk_idx),
+                                 _p(topk_w), _stream(stream)))
+    return topk_idx, topk_w
+
+
+def moe_expert_permute(topk_idx, E: int, stream=None):
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(max(T * k, 4), dtype=torch.int32, device=dev)
+    inv = torch.empty(max(T * k, 4), dtype=torch.int32, device=dev)
+    _check(lib().moe_expert_permute(_p(topk_idx), T, E, k, _p(counts), _p(offsets), _p(perm), _p(inv),
+                                    _stream(stream)))
+    return counts, offsets, perm[:T * k], inv[:T * k]
+
+
+def moe_ffn_workspace_size(T: int, shape: MoeShape) -> int:
+    return int(lib().moe_ffn_workspace_size(T, ctypes.byref(shape)))
+
+
+def moe_ffn_forward(x, shape: MoeShape, weights: LayerWeights, topk_idx, topk_w, residual=None, out=None,
+                    ws=None, stream=None):
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty_like(x)
+    if ws is None:
+        ws = workspace(moe_ffn_workspace_size(T, shape), x.device)
+    _check(lib().moe_ffn_forward(_p(x), T, ctypes.byref(shape), ctypes.byref(weights.c), _p(topk_idx),
+                                 _p(topk_w), _p(residual), _p(out), _p(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def lm_head_workspace_size(T: int, V: int) -> int:
+    return int(lib().lm_head_workspace_size(T, V))
+
+
+def lm_head_argmax(h, w_lm, argmax=None, ws=None, stream=None):
+    T, H = h.shape
+    V = w_lm.shape[0]
+    if argmax is None:
+        argmax = torch.empty(T, dtype=torch.int32, device=h.device)
+    if ws is None:
+        ws = workspace(lm_head_workspace_size(T, V), h.device)
+    _check(lib().lm_head_argmax(_p(h), T, H, _p(w_lm), V, _p(argmax), _p(ws), ws.numel(), _stream(stream)))
+    return argmax
+
+
+def greedy_accept(argmax, drafts, B: int, K: int, emitted=True, stream=None):
+    dev = argmax.device
+    acc = torch.empty(B, dtype=torch.int32, device=dev)
+    nxt = torch.empty(B, dtype=torch.int32, device=dev)
+    em = torch.empty((B, K + 1), dtype=torch.int32, device=dev) if emitted else None
+    _check(lib().greedy_accept(_p(argmax), _p(drafts) if K > 0 else None, B, K, _p(acc), _p(nxt), _p(em),
+                               _stream(stream)))
+    return acc, nxt, em
+
+
+def verify_step_workspace_size(B: int, K: int, shape: MoeShape, V: int) -> int:
+    return int(lib().verify_step_workspace_size(B, K, ctypes.byref(shape), V))
+
+
+class VerifyPlan:
+    """Keeps the C array of layer structs and a workspace for repeated verify steps."""
+
+    def __init__(self, shape: MoeShape, layers: list, w_lm, B: int, K: int, device="cuda"):
+        self.shape, self.layers, self.w_lm, self.B, self.K = shape, layers, w_lm, B, K
+        self.V = w_lm.shape[0]
+        arr = (MoeWeights * max(1, len(layers)))()
+        for i, lw in enumerate(layers):
+            arr[i] = lw.c
+        self.c_layers = arr
+        self.ws = workspace(verify_step_workspace_size(B, K, shape, self.V), device)
+        T = B * (K + 1)
+        self.accepted = torch.empty(B, dtype=torch.int32, device=device)
+        self.next_token = torch.empty(B, dtype=torch.int32, device=device)
+        self.emitted = torch.empty((B, K + 1), dtype=torch.int32, device=device)
+        self.argmax = torch.empty(T, dtype=torch.int32, device=device)
+
+    def __call__(self, hidden, drafts, stream=None):
+        _check(lib().verify_step(_p(hidden), _p(drafts) if self.K > 0 else None, self.B, self.K,
+                                 ctypes.byref(self.shape), self.c_layers, len(self.layers), _p(self.w_lm), self.V,
+                                 _p(self.accepted), _p(self.next_token), _p(self.emitted), _p(self.argmax),
+                                 _p(self.ws), self.ws.numel(), _stream(stream)))
+        return self.accepted, self.next_token, self.emitted, self.argmax
+
+    def sync_status(self, stream=None):
+        sync_status(self.ws, stream)
+
+
+def verify_step(hidden, drafts, B, K, shape, layers, w_lm, stream=None):
+    plan = VerifyPlan(shape, layers, w_lm, B, K, hidden.device)
+    return plan(hidden, drafts, stream)
+
+
+def sync_status(ws, stream=None):
+    _check(lib().mv_sync_status(_p(ws), _stream(stream)))
+
+
+def version() -> str:
+    return lib().mv_version().decode()
+
+
+def launch_count() -> int:
+    return int(lib().mv_launch_count())
+
+
+def set_wait_timeout_ns(ns: int):
+    lib().mv_set_wait_timeout_ns(int(ns))
+
+
+def profile_enable(on: bool):
+    lib().mv_profile_enable(1 if on else 0)
+
+
+def profile_collect() -> dict:
+    n = 16
+    launches = (ctypes.c_int64 * n)()
+    ms = (ctypes.c_double * n)()
+    k = lib().mv_profile_collect(launches, ms, n)
+    out = {}
+    for i in range(k):
+        name = lib().mv_kernel_name(i).decode()
+        out[name] = {"launches": int(launches[i]), "ms": float(ms[i])}
+    return out

@@ -1,0 +1,657 @@
+// C ABI of the verify-step library: host-side argument checks, workspace
+// layout, TMA descriptor creation, kernel launches and launch instrumentation.
+// Declarations and the contract of every entry point: include/moe_verify.h.
+
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <unordered_map>
+#include <vector>
+
+#include "moe_verify.h"
+#include "mv_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<uint64_t> g_launches{0};
+std::atomic<int64_t> g_timeout_ns{2000000000LL};
+constexpr int64_t kDefaultTimeoutNs = 2000000000LL;
+
+mv_status fail(mv_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+mv_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(MV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int num_sms() {
+  static std::mutex mu;
+  static std::unordered_map<int, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(dev);
+  if (it != cache.end()) return it->second;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  cache[dev] = n;
+  return n;
+}
+
+// ---------------------------------------------------------------------------
+// launch instrumentation
+// ---------------------------------------------------------------------------
+enum Kind {
+  KIND_ROUTER = 0,
+  KIND_PERMUTE,
+  KIND_GEMM_SWIGLU,
+  KIND_GEMM_DOWN,
+  KIND_COMBINE,
+  KIND_LM_GEMM,
+  KIND_LM_FINALIZE,
+  KIND_ACCEPT,
+  KIND_COUNT
+};
+const char* kKindNames[KIND_COUNT] = {"router_topk",     "expert_permute",  "grouped_swiglu_gemm",
+                                      "grouped_down_gemm", "combine_unpermute", "lm_head_gemm_argmax",
+                                      "lm_argmax_finalize", "greedy_accept"};
+
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+std::atomic<bool> g_prof_on{false};
+std::vector<ProfRec> g_prof_recs;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+template <class F>
+cudaError_t run_kernel(int kind, cudaStream_t s, F&& launch) {
+  cudaEvent_t a = nullptr, b = nullptr;
+  const bool prof = g_prof_on.load(std::memory_order_relaxed);
+  if (prof) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    a = take_event();
+    b = take_event();
+    cudaEventRecord(a, s);
+  }
+  cudaError_t e = launch();
+  if (prof) {
+    cudaEventRecord(b, s);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_recs.push_back({kind, a, b});
+  }
+  if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors: 2D bf16 [rows][cols] row-major, box = 64 columns x box_rows,
+// 128-byte swizzle, zero fill out of bounds.  Cached by (address, shape, box).
+// ---------------------------------------------------------------------------
+struct TmKey {
+  const void* ptr;
+  uint64_t rows, cols;
+  uint32_t box_rows;
+  bool operator==(const TmKey& o) const {
+    return ptr == o.ptr && rows == o.rows && cols == o.cols && box_rows == o.box_rows;
+  }
+};
+struct TmHash {
+  size_t operator()(const TmKey& k) const {
+    size_t h = reinterpret_cast<size_t>(k.ptr);
+    h ^= (k.rows * 0x9E3779B97F4A7C15ull) + (h << 6) + (h >> 2);
+    h ^= (k.cols * 0xC2B2AE3D27D4EB4Full) + (h << 6) + (h >> 2);
+    h ^= k.box_rows + (h << 6) + (h >> 2);
+    return h;
+  }
+};
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+std::mutex g_tm_mu;
+std::unordered_map<TmKey, CUtensorMap, TmHash> g_tm_cache;
+
+mv_status tmap(CUtensorMap* out, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  TmKey key{ptr, rows, cols, box_rows};
+  {
+    std::lock_guard<std::mutex> lk(g_tm_mu);
+    auto it = g_tm_cache.find(key);
+    if (it != g_tm_cache.end()) {
+      *out = it->second;
+      return MV_OK;
+    }
+  }
+  auto fn = encode_fn();
+  if (!fn) return fail(MV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  CUtensorMap m;
+  std::memset(&m, 0, sizeof(m));
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for [%llu x %llu] box %u", static_cast<int>(r),
+                static_cast<unsigned long long>(rows), static_cast<unsigned long long>(cols), box_rows);
+  std::lock_guard<std::mutex> lk(g_tm_mu);
+  if (g_tm_cache.size() > 8192) g_tm_cache.clear();
+  g_tm_cache[key] = m;
+  *out = m;
+  return MV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// argument checks
+// ---------------------------------------------------------------------------
+#define MV_TRY(expr)                     \
+  do {                                   \
+    mv_status _st = (expr);              \
+    if (_st != MV_OK) return _st;        \
+  } while (0)
+
+mv_status check_ptr(const void* p, const char* name, bool nullable = false) {
+  if (!p) return nullable ? MV_OK : fail(MV_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(MV_ERR_MISALIGNED, "%s is not 16-byte aligned", name);
+  return MV_OK;
+}
+
+mv_status check_shape(const mv_moe_shape* s) {
+  if (!s) return fail(MV_ERR_INVALID_ARG, "shape is NULL");
+  if (s->H <= 0 || s->E <= 0 || s->I <= 0 || s->I_shared < 0 || s->k <= 0)
+    return fail(MV_ERR_INVALID_ARG, "shape has a non-positive size (H=%d E=%d I=%d I_shared=%d k=%d)",
+                s->H, s->E, s->I, s->I_shared, s->k);
+  if (s->k > s->E) return fail(MV_ERR_INVALID_ARG, "k=%d exceeds E=%d", s->k, s->E);
+  if (s->H % 64 || s->I % 64 || s->I_shared % 64)
+    return fail(MV_ERR_UNSUPPORTED_SHAPE, "H, I and I_shared must be multiples of 64 (H=%d I=%d I_shared=%d)",
+                s->H, s->I, s->I_shared);
+  if (s->E > 256 || s->k > 8)
+    return fail(MV_ERR_UNSUPPORTED_SHAPE, "E must be <= 256 and k <= 8 (E=%d k=%d)", s->E, s->k);
+  if (s->H > 16384 || s->I > 65536 || s->I_shared > 65536)
+    return fail(MV_ERR_UNSUPPORTED_SHAPE, "H or I too large");
+  return MV_OK;
+}
+
+mv_status check_rows(int64_t T, const mv_moe_shape* s) {
+  if (T < 0) return fail(MV_ERR_INVALID_ARG, "T=%lld is negative", static_cast<long long>(T));
+  const int64_t wide = std::max<int64_t>(std::max<int64_t>(s->H, s->I), s->I_shared);
+  if (T * s->k * wide >= (int64_t(1) << 31) || T > (int64_t(1) << 24))
+    return fail(MV_ERR_UNSUPPORTED_SHAPE, "T=%lld rows is too large for this shape", static_cast<long long>(T));
+  return MV_OK;
+}
+
+mv_status check_weights(const mv_moe_weights* w, const mv_moe_shape* s) {
+  if (!w) return fail(MV_ERR_INVALID_ARG, "weights is NULL");
+  MV_TRY(check_ptr(w->w_router, "w_router"));
+  MV_TRY(check_ptr(w->router_bias, "router_bias", true));
+  MV_TRY(check_ptr(w->w_gate, "w_gate"));
+  MV_TRY(check_ptr(w->w_up, "w_up"));
+  MV_TRY(check_ptr(w->w_down, "w_down"));
+  if (s->I_shared > 0) {
+    MV_TRY(check_ptr(w->ws_gate, "ws_gate"));
+    MV_TRY(check_ptr(w->ws_up, "ws_up"));
+    MV_TRY(check_ptr(w->ws_down, "ws_down"));
+  }
+  return MV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// workspace layouts (every region 1024-byte aligned relative to the base)
+// ---------------------------------------------------------------------------
+constexpr size_t kHeader = 1024;  // sticky error word + reserved
+
+struct Carve {
+  char* base;
+  size_t off = 0;
+  template <class T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off = align_up(off + count * sizeof(T), 1024);
+    return p;
+  }
+};
+
+struct FfnWs {
+  int32_t *counts, *offsets, *perm, *inv;
+  uint16_t *x_perm, *a_perm, *a_sh;
+  float *y_perm, *y_sh;
+};
+
+FfnWs carve_ffn(Carve& c, int64_t T, const mv_moe_shape& s) {
+  FfnWs w;
+  const size_t n = static_cast<size_t>(T) * s.k;
+  w.counts = c.take<int32_t>(s.E);
+  w.offsets = c.take<int32_t>(s.E + 1);
+  w.perm = c.take<int32_t>(n);
+  w.inv = c.take<int32_t>(n);
+  w.x_perm = c.take<uint16_t>(n * s.H);
+  w.a_perm = c.take<uint16_t>(n * s.I);
+  w.a_sh = c.take<uint16_t>(static_cast<size_t>(T) * s.I_shared);
+  w.y_perm = c.take<float>(n * s.H);
+  w.y_sh = c.take<float>(static_cast<size_t>(T) * s.H);
+  return w;
+}
+
+int lm_parts(int V) { return (V + 127) / 128 * 4; }
+
+uint64_t timeout_ns() {
+  const int64_t t = g_timeout_ns.load();
+  return static_cast<uint64_t>(t > 0 ? t : kDefaultTimeoutNs);
+}
+
+int gemm_grid(int64_t units) {
+  const int sms = num_sms();
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, sms)));
+}
+
+// ---------------------------------------------------------------------------
+// the path
+// ---------------------------------------------------------------------------
+mv_status ffn_forward_impl(const uint16_t* x, int T, const mv_moe_shape& s, const mv_moe_weights& w,
+                           const int32_t* idx, const float* tw, const uint16_t* res, uint16_t* out,
+                           const FfnWs& ws, int* err, cudaStream_t st) {
+  const int H = s.H, E = s.E, I = s.I, Ish = s.I_shared, k = s.k;
+  const int n = T * k;
+  cudaError_t e = run_kernel(KIND_PERMUTE, st, [&] {
+    return mv::launch_permute(idx, T, E, k, ws.counts, ws.offsets, ws.perm, ws.inv, x, H, ws.x_perm, st);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "expert_permute launch");
+
+  constexpr int BN = 128;
+  // gate + up with the SwiGLU epilogue
+  {
+    mv::GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.err = err;
+    p.timeout_ns = timeout_ns();
+    int ns = 0;
+    int64_t units = 0;
+    if (Ish > 0) {
+      mv::GemmSet& S = p.set[ns++];
+      MV_TRY(tmap(&S.a0, w.ws_gate, Ish, H, 128));
+      MV_TRY(tmap(&S.a1, w.ws_up, Ish, H, 128));
+      MV_TRY(tmap(&S.b, x, T, H, 16));
+      S.out = ws.a_sh;
+      S.ld_out = Ish;
+      S.K = H;
+      S.M = Ish;
+      S.groups = 1;
+      S.static_rows = T;
+      units += int64_t((Ish + 127) / 128) * ((T + BN - 1) / BN);
+    }
+    {
+      mv::GemmSet& S = p.set[ns++];
+      MV_TRY(tmap(&S.a0, w.w_gate, static_cast<uint64_t>(E) * I, H, 128));
+      MV_TRY(tmap(&S.a1, w.w_up, static_cast<uint64_t>(E) * I, H, 128));
+      MV_TRY(tmap(&S.b, ws.x_perm, n, H, 16));
+      S.out = ws.a_perm;
+      S.ld_out = I;
+      S.K = H;
+      S.M = I;
+      S.groups = E;
+      S.counts = ws.counts;
+      S.offsets = ws.offsets;
+      S.a_group_stride = I;
+      units += int64_t((I + 127) / 128) * (std::min(E, n) + (n + BN - 1) / BN);
+    }
+    p.nsets = ns;
+    e = run_kernel(KIND_GEMM_SWIGLU, st, [&] { return mv::launch_gemm(mv::EPI_SWIGLU, p, gemm_grid(units), st); });
+    if (e != cudaSuccess) return cuda_fail(e, "grouped_swiglu_gemm launch");
+  }
+  // down projection, fp32 rows
+  {
+    mv::GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.err = err;
+    p.timeout_ns = timeout_ns();
+    int ns = 0;
+    int64_t units = 0;
+    if (Ish > 0) {
+      mv::GemmSet& S = p.set[ns++];
+      MV_TRY(tmap(&S.a0, w.ws_down, H, Ish, 128));
+      MV_TRY(tmap(&S.b, ws.a_sh, T, Ish, 16));
+      S.a1 = S.a0;
+      S.out = ws.y_sh;
+      S.ld_out = H;
+      S.K = Ish;
+      S.M = H;
+      S.groups = 1;
+      S.static_rows = T;
+      units += int64_t((H + 127) / 128) * ((T + BN - 1) / BN);
+    }
+    {
+      mv::GemmSet& S = p.set[ns++];
+      MV_TRY(tmap(&S.a0, w.w_down, static_cast<uint64_t>(E) * H, I, 128));
+      MV_TRY(tmap(&S.b, ws.a_perm, n, I, 16));
+      S.a1 = S.a0;
+      S.out = ws.y_perm;
+      S.ld_out = H;
+      S.K = I;
+      S.M = H;
+      S.groups = E;
+      S.counts = ws.counts;
+      S.offsets = ws.offsets;
+      S.a_group_stride = H;
+      units += int64_t((H + 127) / 128) * (std::min(E, n) + (n + BN - 1) / BN);
+    }
+    p.nsets = ns;
+    e = run_kernel(KIND_GEMM_DOWN, st, [&] { return mv::launch_gemm(mv::EPI_STORE_F32, p, gemm_grid(units), st); });
+    if (e != cudaSuccess) return cuda_fail(e, "grouped_down_gemm launch");
+  }
+  e = run_kernel(KIND_COMBINE, st, [&] {
+    return mv::launch_combine(ws.y_perm, Ish > 0 ? ws.y_sh : nullptr, ws.inv, tw, res, out, T, H, k, err, st);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  return MV_OK;
+}
+
+mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, int V, uint64_t* parts,
+                       int* err, cudaStream_t st) {
+  mv::GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.err = err;
+  p.timeout_ns = timeout_ns();
+  mv::GemmSet& S = p.set[0];
+  MV_TRY(tmap(&S.a0, w_lm, V, H, 128));
+  MV_TRY(tmap(&S.b, h, T, H, 16));
+  S.a1 = S.a0;
+  S.out = parts;
+  S.ld_out = T;
+  S.K = H;
+  S.M = V;
+  S.groups = 1;
+  S.static_rows = T;
+  p.nsets = 1;
+  const int64_t units = int64_t((V + 127) / 128) * ((T + 127) / 128);
+  cudaError_t e = run_kernel(KIND_LM_GEMM, st, [&] { return mv::launch_gemm(mv::EPI_ARGMAX, p, gemm_grid(units), st); });
+  if (e != cudaSuccess) return cuda_fail(e, "lm_head_gemm_argmax launch");
+  return MV_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// exported entry points
+// ===========================================================================
+extern "C" {
+
+const char* mv_last_error(void) { return g_last_error.c_str(); }
+
+const char* mv_version(void) { return "moe_verify 0.1.0 sm_100a"; }
+
+uint64_t mv_launch_count(void) { return g_launches.load(); }
+
+void mv_set_wait_timeout_ns(int64_t ns) { g_timeout_ns.store(ns > 0 ? ns : kDefaultTimeoutNs); }
+
+void mv_profile_enable(int32_t on) { g_prof_on.store(on != 0); }
+
+const char* mv_kernel_name(int32_t kind) {
+  return (kind >= 0 && kind < KIND_COUNT) ? kKindNames[kind] : nullptr;
+}
+
+int32_t mv_profile_collect(int64_t* launches, double* total_ms, int32_t n_kinds) {
+  std::vector<ProfRec> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    recs.swap(g_prof_recs);
+  }
+  const int n = std::min<int>(n_kinds, KIND_COUNT);
+  for (int i = 0; i < n; ++i) {
+    if (launches) launches[i] = 0;
+    if (total_ms) total_ms[i] = 0.0;
+  }
+  for (auto& r : recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess &&
+        r.kind < n) {
+      if (launches) launches[r.kind] += 1;
+      if (total_ms) total_ms[r.kind] += ms;
+    }
+  }
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : recs) {
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  return n;
+}
+
+mv_status moe_router_topk(const uint16_t* x, int32_t T, const mv_moe_shape* shape, const uint16_t* w_router,
+                          const float* router_bias, int32_t* topk_idx, float* topk_w, mv_stream_t stream) {
+  MV_TRY(check_shape(shape));
+  MV_TRY(check_rows(T, shape));
+  MV_TRY(check_ptr(x, "x"));
+  MV_TRY(check_ptr(w_router, "w_router"));
+  MV_TRY(check_ptr(router_bias, "router_bias", true));
+  MV_TRY(check_ptr(topk_idx, "topk_idx"));
+  MV_TRY(check_ptr(topk_w, "topk_w"));
+  if (T == 0) return MV_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = run_kernel(KIND_ROUTER, st, [&] {
+    return mv::launch_router(x, T, shape->H, shape->E, shape->k, w_router, router_bias, topk_idx, topk_w, st);
+  });
+  return e == cudaSuccess ? MV_OK : cuda_fail(e, "router_topk launch");
+}
+
+mv_status moe_expert_permute(const int32_t* topk_idx, int32_t T, int32_t E, int32_t k, int32_t* counts,
+                             int32_t* offsets, int32_t* perm, int32_t* inv, mv_stream_t stream) {
+  if (T < 0 || E <= 0 || E > 256 || k <= 0 || k > 8 || k > E)
+    return fail(MV_ERR_INVALID_ARG, "bad sizes T=%d E=%d k=%d", T, E, k);
+  MV_TRY(check_ptr(topk_idx, "topk_idx", T == 0));
+  MV_TRY(check_ptr(counts, "counts"));
+  MV_TRY(check_ptr(offsets, "offsets"));
+  MV_TRY(check_ptr(perm, "perm", T == 0));
+  MV_TRY(check_ptr(inv, "inv", T == 0));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // H = 0: no rows are gathered
+  cudaError_t e = run_kernel(KIND_PERMUTE, st, [&] {
+    return mv::launch_permute(topk_idx, T, E, k, counts, offsets, perm, inv, nullptr, 0, nullptr, st);
+  });
+  return e == cudaSuccess ? MV_OK : cuda_fail(e, "expert_permute launch");
+}
+
+size_t moe_ffn_workspace_size(int32_t T, const mv_moe_shape* shape) {
+  if (!shape || T < 0) return 0;
+  Carve c{nullptr};
+  carve_ffn(c, T, *shape);
+  return kHeader + c.off + 1024;
+}
+
+mv_status moe_ffn_forward(const uint16_t* x, int32_t T, const mv_moe_shape* shape, const mv_moe_weights* weights,
+                          const int32_t* topk_idx, const float* topk_w, const uint16_t* residual, uint16_t* out,
+                          void* ws, size_t ws_bytes, mv_stream_t stream) {
+  MV_TRY(check_shape(shape));
+  MV_TRY(check_rows(T, shape));
+  MV_TRY(check_weights(weights, shape));
+  MV_TRY(check_ptr(x, "x"));
+  MV_TRY(check_ptr(topk_idx, "topk_idx"));
+  MV_TRY(check_ptr(topk_w, "topk_w"));
+  MV_TRY(check_ptr(residual, "residual", true));
+  MV_TRY(check_ptr(out, "out"));
+  MV_TRY(check_ptr(ws, "workspace"));
+  if (out == x) return fail(MV_ERR_INVALID_ARG, "out may not alias x");
+  const size_t need = moe_ffn_workspace_size(T, shape);
+  if (ws_bytes < need)
+    return fail(MV_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+  if (T == 0) return MV_OK;
+  Carve c{static_cast<char*>(ws) + kHeader};
+  FfnWs fw = carve_ffn(c, T, *shape);
+  return ffn_forward_impl(x, T, *shape, *weights, topk_idx, topk_w, residual, out, fw, static_cast<int*>(ws),
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t lm_head_workspace_size(int32_t T, int32_t V) {
+  if (T < 0 || V <= 0) return 0;
+  return kHeader + align_up(static_cast<size_t>(lm_parts(V)) * T * 8, 1024) + 1024;
+}
+
+mv_status lm_head_argmax(const uint16_t* h, int32_t T, int32_t H, const uint16_t* w_lm, int32_t V, int32_t* argmax,
+                         void* ws, size_t ws_bytes, mv_stream_t stream) {
+  if (T < 0 || H <= 0 || V <= 0) return fail(MV_ERR_INVALID_ARG, "bad sizes T=%d H=%d V=%d", T, H, V);
+  if (H % 64 || V % 8 || H > 16384 || T > (1 << 24))
+    return fail(MV_ERR_UNSUPPORTED_SHAPE, "H must be a multiple of 64 and V of 8 (H=%d V=%d)", H, V);
+  MV_TRY(check_ptr(h, "h"));
+  MV_TRY(check_ptr(w_lm, "w_lm"));
+  MV_TRY(check_ptr(argmax, "argmax"));
+  MV_TRY(check_ptr(ws, "workspace"));
+  const size_t need = lm_head_workspace_size(T, V);
+  if (ws_bytes < need)
+    return fail(MV_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+  if (T == 0) return MV_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint64_t* parts = reinterpret_cast<uint64_t*>(static_cast<char*>(ws) + kHeader);
+  MV_TRY(lm_gemm_impl(h, T, H, w_lm, V, parts, static_cast<int*>(ws), st));
+  cudaError_t e = run_kernel(KIND_LM_FINALIZE, st, [&] { return mv::launch_lm_finalize(parts, lm_parts(V), T, argmax, st); });
+  return e == cudaSuccess ? MV_OK : cuda_fail(e, "lm_argmax_finalize launch");
+}
+
+mv_status greedy_accept(const int32_t* argmax, const int32_t* drafts, int32_t B, int32_t K, int32_t* accepted,
+                        int32_t* next_token, int32_t* emitted, mv_stream_t stream) {
+  if (B < 0 || K < 0 || K > 32) return fail(MV_ERR_INVALID_ARG, "bad sizes B=%d K=%d (K <= 32)", B, K);
+  MV_TRY(check_ptr(argmax, "argmax", B == 0));
+  MV_TRY(check_ptr(drafts, "drafts", K == 0 || B == 0));
+  MV_TRY(check_ptr(accepted, "accepted", B == 0));
+  MV_TRY(check_ptr(next_token, "next_token", B == 0));
+  MV_TRY(check_ptr(emitted, "emitted", true));
+  if (B == 0) return MV_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = run_kernel(KIND_ACCEPT, st, [&] {
+    return mv::launch_accept(argmax, K > 0 ? drafts : nullptr, B, K, accepted, next_token, emitted, st);
+  });
+  return e == cudaSuccess ? MV_OK : cuda_fail(e, "greedy_accept launch");
+}
+
+size_t verify_step_workspace_size(int32_t B, int32_t K, const mv_moe_shape* shape, int32_t V) {
+  if (!shape || B < 0 || K < 0 || V <= 0) return 0;
+  const int64_t T = int64_t(B) * (K + 1);
+  Carve c{nullptr};
+  c.take<uint16_t>(static_cast<size_t>(T) * shape->H);
+  c.take<uint16_t>(static_cast<size_t>(T) * shape->H);
+  c.take<int32_t>(static_cast<size_t>(T) * shape->k);
+  c.take<float>(static_cast<size_t>(T) * shape->k);
+  c.take<uint64_t>(static_cast<size_t>(lm_parts(V)) * T);
+  carve_ffn(c, T, *shape);
+  return kHeader + c.off + 1024;
+}
+
+mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, int32_t K, const mv_moe_shape* shape,
+                      const mv_moe_weights* layers, int32_t n_layers, const uint16_t* w_lm, int32_t V,
+                      int32_t* accepted, int32_t* next_token, int32_t* emitted, int32_t* argmax, void* ws,
+                      size_t ws_bytes, mv_stream_t stream) {
+  MV_TRY(check_shape(shape));
+  if (B < 0 || K < 0 || K > 32 || n_layers < 0 || V <= 0)
+    return fail(MV_ERR_INVALID_ARG, "bad sizes B=%d K=%d (K <= 32) n_layers=%d V=%d", B, K, n_layers, V);
+  if (V % 8) return fail(MV_ERR_UNSUPPORTED_SHAPE, "V=%d must be a multiple of 8", V);
+  const int64_t T = int64_t(B) * (K + 1);
+  MV_TRY(check_rows(T, shape));
+  if (n_layers > 0 && !layers) return fail(MV_ERR_INVALID_ARG, "layers is NULL");
+  for (int l = 0; l < n_layers; ++l) MV_TRY(check_weights(&layers[l], shape));
+  MV_TRY(check_ptr(hidden, "hidden", B == 0));
+  MV_TRY(check_ptr(drafts, "drafts", K == 0 || B == 0));
+  MV_TRY(check_ptr(w_lm, "w_lm"));
+  MV_TRY(check_ptr(accepted, "accepted", B == 0));
+  MV_TRY(check_ptr(next_token, "next_token", B == 0));
+  MV_TRY(check_ptr(emitted, "emitted", true));
+  MV_TRY(check_ptr(argmax, "argmax", true));
+  MV_TRY(check_ptr(ws, "workspace"));
+  const size_t need = verify_step_workspace_size(B, K, shape, V);
+  if (ws_bytes < need)
+    return fail(MV_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+  if (B == 0) return MV_OK;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* err = static_cast<int*>(ws);
+  Carve c{static_cast<char*>(ws) + kHeader};
+  uint16_t* hbuf[2] = {c.take<uint16_t>(static_cast<size_t>(T) * shape->H),
+                       c.take<uint16_t>(static_cast<size_t>(T) * shape->H)};
+  int32_t* idx = c.take<int32_t>(static_cast<size_t>(T) * shape->k);
+  float* tw = c.take<float>(static_cast<size_t>(T) * shape->k);
+  uint64_t* parts = c.take<uint64_t>(static_cast<size_t>(lm_parts(V)) * T);
+  FfnWs fw = carve_ffn(c, T, *shape);
+
+  const uint16_t* h = hidden;
+  for (int l = 0; l < n_layers; ++l) {
+    const mv_moe_weights& w = layers[l];
+    cudaError_t e = run_kernel(KIND_ROUTER, st, [&] {
+      return mv::launch_router(h, static_cast<int>(T), shape->H, shape->E, shape->k, w.w_router, w.router_bias, idx,
+                               tw, st);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "router_topk launch");
+    uint16_t* next = hbuf[l & 1];
+    MV_TRY(ffn_forward_impl(h, static_cast<int>(T), *shape, w, idx, tw, h, next, fw, err, st));
+    h = next;
+  }
+  MV_TRY(lm_gemm_impl(h, static_cast<int>(T), shape->H, w_lm, V, parts, err, st));
+  cudaError_t e = run_kernel(KIND_ACCEPT, st, [&] {
+    return mv::launch_accept_from_keys(parts, lm_parts(V), K > 0 ? drafts : nullptr, B, K, accepted, next_token,
+                                       emitted, argmax, st);
+  });
+  return e == cudaSuccess ? MV_OK : cuda_fail(e, "greedy_accept launch");
+}
+
+mv_status mv_workspace_init(void* ws, size_t ws_bytes, mv_stream_t stream) {
+  MV_TRY(check_ptr(ws, "workspace"));
+  if (ws_bytes < kHeader) return fail(MV_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes is below the header", ws_bytes);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kHeader, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MV_OK : cuda_fail(e, "clearing the workspace header");
+}
+
+mv_status mv_sync_status(void* ws, mv_stream_t stream) {
+  MV_TRY(check_ptr(ws, "workspace"));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int word = 0;
+  e = cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (word != 0) {
+    e = cudaMemset(ws, 0, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+    if (word & mv::kErrTimeout) return fail(MV_ERR_TIMEOUT, "a device-side wait ran out (error word 0x%x)", word);
+    return fail(MV_ERR_INTERNAL, "a device-side check failed (error word 0x%x)", word);
+  }
+  return MV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,437 @@
+// CUDA-core kernels of the verify step: router top-k, grouping by expert,
+// weighted combine, LM-head argmax finalisation and greedy acceptance.
+// Methods follow the jina-ocr-v1 model card (jina.ai/models/jina-ocr-v1):
+// architecture paragraph (64 routed + 2 shared experts, top-6 routing,
+// 129,280-token vocabulary), decoding-speed paragraph and introduction
+// (K drafts verified greedily, lossless).
+
+#include "mv_device.cuh"
+#include "mv_internal.h"
+
+namespace mv {
+
+namespace {
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// (value, index) pair comparison: larger value wins, equal values -> lower index.
+__device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
+  return v > bv || (v == bv && i < bi);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Router: logits = x . W_r^T (+ bias) in fp32, top-k on the logits (ties to
+// the lower expert id, slots in descending order), weights =
+// exp(l_j - l_max) / sum_selected exp(l - l_max), which equals the softmax
+// over all E restricted to the kept experts and renormalised.
+// A CTA of 8 warps owns R rows: the rows sit in shared memory, warp w computes
+// experts w, w+8, ... for all R rows (each router weight row is read once per
+// CTA, 16-byte loads), then warp r < R selects the top-k of row r.
+// ---------------------------------------------------------------------------
+template <int R>
+__global__ void __launch_bounds__(256) router_topk_kernel(const uint16_t* __restrict__ x, int T,
+                                                          int H, int E, int k,
+                                                          const uint16_t* __restrict__ wr,
+                                                          const float* __restrict__ bias,
+                                                          int32_t* __restrict__ idx,
+                                                          float* __restrict__ wout) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  uint16_t* xs = reinterpret_cast<uint16_t*>(sm);                        // [R][H]
+  float* ls = reinterpret_cast<float*>(sm + static_cast<size_t>(R) * H * 2);  // [R][E]
+  const int row0 = blockIdx.x * R;
+  const int nrows = min(R, T - row0);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int hv = H / 8;  // 16-byte vectors per row
+
+  for (int i = tid; i < R * hv; i += blockDim.x) {
+    const int r = i / hv, c = i % hv;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < nrows) v = reinterpret_cast<const uint4*>(x + static_cast<size_t>(row0 + r) * H)[c];
+    reinterpret_cast<uint4*>(xs + static_cast<size_t>(r) * H)[c] = v;
+  }
+  __syncthreads();
+
+  for (int e = warp; e < E; e += 8) {
+    float acc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r] = 0.f;
+    const uint4* we = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e) * H);
+    for (int c = lane; c < hv; c += 32) {
+      float wf[8];
+      bf16x8_to_f32(__ldg(we + c), wf);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        float xf[8];
+        bf16x8_to_f32(reinterpret_cast<const uint4*>(xs + static_cast<size_t>(r) * H)[c], xf);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[r] = fmaf(xf[j], wf[j], acc[r]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float v = acc[r];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) ls[r * E + e] = bias ? v + bias[e] : v;
+    }
+  }
+  __syncthreads();
+
+  if (warp < nrows) {
+    const int r = warp;
+    constexpr int kMaxPer = 8;  // E <= 256
+    float v[kMaxPer];
+    const int per = (E + 31) / 32;
+#pragma unroll
+    for (int q = 0; q < kMaxPer; ++q) {
+      const int e = lane + 32 * q;
+      v[q] = (q < per && e < E) ? ls[r * E + e] : -__int_as_float(0x7f800000);
+    }
+    float selv[8];
+    int sele[8];
+    for (int j = 0; j < k; ++j) {
+      float bv = -__int_as_float(0x7f800000);
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int q = 0; q < kMaxPer; ++q) {
+        const int e = lane + 32 * q;
+        if (q < per && e < E && better(v[q], e, bv, bi)) {
+          bv = v[q];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (better(ov, oi, bv, bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      selv[j] = bv;
+      sele[j] = bi;
+      // the lane holding the winner removes it from further rounds
+#pragma unroll
+      for (int q = 0; q < kMaxPer; ++q)
+        if (lane + 32 * q == bi) v[q] = -__int_as_float(0x7f800000);
+    }
+    const float mx = selv[0];
+    float s = 0.f;
+    for (int j = 0; j < k; ++j) s += expf(selv[j] - mx);
+    if (lane < k) {
+      float my_v = selv[0];
+      int my_e = sele[0];
+      for (int j = 1; j < k; ++j)
+        if (j == lane) {
+          my_v = selv[j];
+          my_e = sele[j];
+        }
+      const size_t o = static_cast<size_t>(row0 + r) * k + lane;
+      idx[o] = my_e;
+      wout[o] = expf(my_v - mx) / s;
+    }
+  }
+}
+
+template <int R>
+static void launch_router_r(const uint16_t* x, int T, int H, int E, int k, const uint16_t* wr,
+                            const float* bias, int32_t* idx, float* w, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(R) * H * 2 + static_cast<size_t>(R) * E * 4;
+  router_topk_kernel<R><<<(T + R - 1) / R, 256, smem, s>>>(x, T, H, E, k, wr, bias, idx, w);
+}
+
+// Rows per CTA: 4 for decode-sized batches (more CTAs share the router weight
+// stream), 8 for large batches; fewer when the rows would not fit in 48 KB of
+// shared memory.
+cudaError_t launch_router(const uint16_t* x, int T, int H, int E, int k, const uint16_t* wr,
+                          const float* bias, int32_t* idx, float* w, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  auto fits = [&](int R) { return static_cast<size_t>(R) * H * 2 + static_cast<size_t>(R) * E * 4 <= 48 * 1024; };
+  int R = (T <= 1024) ? 4 : 8;
+  while (R > 1 && !fits(R)) R >>= 1;
+  switch (R) {
+    case 8: launch_router_r<8>(x, T, H, E, k, wr, bias, idx, w, s); break;
+    case 4: launch_router_r<4>(x, T, H, E, k, wr, bias, idx, w, s); break;
+    case 2: launch_router_r<2>(x, T, H, E, k, wr, bias, idx, w, s); break;
+    default: launch_router_r<1>(x, T, H, E, k, wr, bias, idx, w, s); break;
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Grouping by expert.  One CTA per expert e:
+//   counts[e]  = #entries routed to e, offsets[e] = #entries routed below e,
+//   perm[offsets[e] + p] = the p-th entry (row order) routed to e,
+//   inv[entry] = its position in perm,
+//   x_perm[position] = x[row of entry]  (the gathered GEMM input).
+// Entries are i = r*k + j; a row never selects the same expert twice, so row
+// order within an expert is (row, slot) order.  Exact and deterministic.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) permute_kernel(const int32_t* __restrict__ idx, int T, int E,
+                                                      int k, int32_t* __restrict__ counts,
+                                                      int32_t* __restrict__ offsets,
+                                                      int32_t* __restrict__ perm,
+                                                      int32_t* __restrict__ inv,
+                                                      const uint16_t* __restrict__ x, int H,
+                                                      uint16_t* __restrict__ x_perm) {
+  const int e = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = T * k;
+  __shared__ int red_eq[8], red_lt[8], wsum[8];
+  __shared__ int base_s, running_s;
+
+  int c_eq = 0, c_lt = 0;
+  for (int i = tid; i < n; i += blockDim.x) {
+    const int v = idx[i];
+    c_eq += (v == e);
+    c_lt += (v >= 0 && v < e);
+    if (e == 0 && (v < 0 || v >= E)) inv[i] = -1;  // out-of-range id: routed nowhere
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    c_eq += __shfl_xor_sync(0xffffffffu, c_eq, o);
+    c_lt += __shfl_xor_sync(0xffffffffu, c_lt, o);
+  }
+  if (lane == 0) {
+    red_eq[warp] = c_eq;
+    red_lt[warp] = c_lt;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int a = 0, b = 0;
+    for (int w = 0; w < 8; ++w) {
+      a += red_eq[w];
+      b += red_lt[w];
+    }
+    counts[e] = a;
+    offsets[e] = b;
+    if (e == E - 1) offsets[E] = a + b;
+    base_s = b;
+    running_s = 0;
+  }
+  __syncthreads();
+  const int base = base_s;
+
+  for (int r0 = 0; r0 < T; r0 += blockDim.x) {
+    const int r = r0 + tid;
+    int slot = -1;
+    if (r < T)
+      for (int j = 0; j < k; ++j)
+        if (idx[static_cast<size_t>(r) * k + j] == e) slot = j;
+    const unsigned bal = __ballot_sync(0xffffffffu, slot >= 0);
+    const int before = __popc(bal & ((1u << lane) - 1u));
+    if (lane == 0) wsum[warp] = __popc(bal);
+    __syncthreads();
+    int wpre = 0, tot = 0;
+    for (int w = 0; w < 8; ++w) {
+      if (w < warp) wpre += wsum[w];
+      tot += wsum[w];
+    }
+    if (slot >= 0) {
+      const int pos = base + running_s + wpre + before;
+      const int ent = r * k + slot;
+      perm[pos] = ent;
+      inv[ent] = pos;
+    }
+    __syncthreads();
+    if (tid == 0) running_s += tot;
+    __syncthreads();
+  }
+
+  // gather the routed rows (each warp copies whole rows with 16-byte vectors)
+  const int cnt = running_s;
+  const int hv = H / 8;
+  for (int p = warp; p < cnt; p += 8) {
+    const int ent = perm[base + p];
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(ent / k) * H);
+    uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(base + p) * H);
+    for (int c = lane; c < hv; c += 32) dst[c] = src[c];
+  }
+}
+
+cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
+                           int32_t* offsets, int32_t* perm, int32_t* inv, const uint16_t* x,
+                           int H, uint16_t* x_perm, cudaStream_t s) {
+  permute_kernel<<<E, 256, 0, s>>>(idx, T, E, k, counts, offsets, perm, inv, x, H, x_perm);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Combine: m = sum_j w_j * y_j (slot order) + y_shared, out = bf16(res + m).
+// Each product and sum is rounded separately (no fused multiply-add), in the
+// order written.  One thread owns 8 consecutive hidden features of a row.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y_perm,
+                                                      const float* __restrict__ y_sh,
+                                                      const int32_t* __restrict__ inv,
+                                                      const float* __restrict__ w,
+                                                      const uint16_t* res, uint16_t* out, int T,
+                                                      int H, int k, int n_pos, int* err) {
+  const int hv = H / 8;
+  const long long total = static_cast<long long>(T) * hv;
+  for (long long t = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; t < total;
+       t += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(t / hv);
+    const int c = static_cast<int>(t % hv);
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int p = inv[static_cast<size_t>(r) * k + j];
+      if (p < 0 || p >= n_pos) {  // entry routed to no valid expert
+        if (err && c == 0) atomicOr(err, kErrInternal);
+        continue;
+      }
+      const float wj = w[static_cast<size_t>(r) * k + j];
+      const float4* yp = reinterpret_cast<const float4*>(y_perm + static_cast<size_t>(p) * H) + 2 * c;
+      const float4 a = yp[0], b = yp[1];
+      const float yv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(m[i], __fmul_rn(wj, yv[i]));
+    }
+    if (y_sh) {
+      const float4* ys = reinterpret_cast<const float4*>(y_sh + static_cast<size_t>(r) * H) + 2 * c;
+      const float4 a = ys[0], b = ys[1];
+      const float yv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(m[i], yv[i]);
+    }
+    if (res) {
+      float rf[8];
+      bf16x8_to_f32(reinterpret_cast<const uint4*>(res + static_cast<size_t>(r) * H)[c], rf);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(rf[i], m[i]);
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      o[i] = static_cast<uint32_t>(f32_to_bf16_bits(m[2 * i])) |
+             (static_cast<uint32_t>(f32_to_bf16_bits(m[2 * i + 1])) << 16);
+    reinterpret_cast<uint4*>(out + static_cast<size_t>(r) * H)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t* inv,
+                           const float* w, const uint16_t* res, uint16_t* out, int T, int H,
+                           int k, int* err, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  const long long total = static_cast<long long>(T) * (H / 8);
+  const long long blocks = (total + 255) / 256;
+  const int grid = static_cast<int>(blocks < 148LL * 8 ? blocks : 148LL * 8);
+  combine_kernel<<<grid, 256, 0, s>>>(y_perm, y_sh, inv, w, res, out, T, H, k, T * k, err);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// LM-head argmax finalisation: the GEMM epilogue leaves one packed
+// (order-preserving logit, inverted index) key per (32-row vocabulary block,
+// token); the largest key is the argmax with ties to the lower index.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t max_key_over_parts(const uint64_t* keys, int nparts, int T,
+                                                       int t, int lane) {
+  uint64_t best = 0;
+  for (int p = lane; p < nparts; p += 32) {
+    const uint64_t v = keys[static_cast<size_t>(p) * T + t];
+    best = v > best ? v : best;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t v = __shfl_xor_sync(0xffffffffu, best, o);
+    best = v > best ? v : best;
+  }
+  return best;
+}
+
+__global__ void __launch_bounds__(256) lm_finalize_kernel(const uint64_t* __restrict__ keys,
+                                                          int nparts, int T,
+                                                          int32_t* __restrict__ argmax) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const uint64_t best = max_key_over_parts(keys, nparts, T, t, lane);
+  if (lane == 0) argmax[t] = static_cast<int32_t>(argmax_key_index(best));
+}
+
+cudaError_t launch_lm_finalize(const uint64_t* keys, int nparts, int T, int32_t* argmax,
+                               cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  lm_finalize_kernel<<<(T + 7) / 8, 256, 0, s>>>(keys, nparts, T, argmax);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Greedy acceptance (one thread per sequence).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void accept_one(const int32_t* g, const int32_t* d, int K, int b,
+                                           int32_t* accepted, int32_t* next_token,
+                                           int32_t* emitted) {
+  int a = 0;
+  while (a < K && d[a] == g[a]) ++a;
+  accepted[b] = a;
+  next_token[b] = g[a];
+  if (emitted)
+    for (int j = 0; j <= K; ++j) emitted[static_cast<size_t>(b) * (K + 1) + j] = (j <= a) ? g[j] : -1;
+}
+
+__global__ void accept_kernel(const int32_t* __restrict__ argmax, const int32_t* __restrict__ drafts,
+                              int B, int K, int32_t* accepted, int32_t* next_token,
+                              int32_t* emitted) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  accept_one(argmax + static_cast<size_t>(b) * (K + 1),
+             drafts ? drafts + static_cast<size_t>(b) * K : nullptr, K, b, accepted, next_token,
+             emitted);
+}
+
+cudaError_t launch_accept(const int32_t* argmax, const int32_t* drafts, int B, int K,
+                          int32_t* accepted, int32_t* next_token, int32_t* emitted,
+                          cudaStream_t s) {
+  if (B <= 0) return cudaSuccess;
+  accept_kernel<<<(B + 127) / 128, 128, 0, s>>>(argmax, drafts, B, K, accepted, next_token, emitted);
+  return cudaGetLastError();
+}
+
+// Fused LM finalisation + acceptance: one CTA per sequence, warp j finalises
+// row b*(K+1)+j, then one thread accepts.
+__global__ void __launch_bounds__(256) accept_from_keys_kernel(
+    const uint64_t* __restrict__ keys, int nparts, const int32_t* __restrict__ drafts, int B, int K,
+    int32_t* accepted, int32_t* next_token, int32_t* emitted, int32_t* argmax_out) {
+  __shared__ int32_t g[64];
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = B * (K + 1);
+  for (int j = warp; j <= K; j += blockDim.x >> 5) {
+    const int t = b * (K + 1) + j;
+    const uint64_t best = max_key_over_parts(keys, nparts, T, t, lane);
+    if (lane == 0) {
+      g[j] = static_cast<int32_t>(argmax_key_index(best));
+      if (argmax_out) argmax_out[t] = g[j];
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    accept_one(g, drafts ? drafts + static_cast<size_t>(b) * K : nullptr, K, b, accepted,
+               next_token, emitted);
+}
+
+cudaError_t launch_accept_from_keys(const uint64_t* keys, int nparts, const int32_t* drafts,
+                                    int B, int K, int32_t* accepted, int32_t* next_token,
+                                    int32_t* emitted, int32_t* argmax, cudaStream_t s) {
+  if (B <= 0) return cudaSuccess;
+  const int warps = min(8, K + 1);
+  accept_from_keys_kernel<<<B, warps * 32, 0, s>>>(keys, nparts, drafts, B, K, accepted,
+                                                    next_token, emitted, argmax);
+  return cudaGetLastError();
+}
+
+}  // namespace mv

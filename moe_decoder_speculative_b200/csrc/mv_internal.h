@@ -1,0 +1,64 @@
+// Internal host/device declarations shared by the library's translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace mv {
+
+enum { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_ARGMAX = 2 };
+
+// Sticky device error bits, OR-ed into the workspace's error word.
+constexpr int kErrTimeout = 1;
+constexpr int kErrInternal = 2;
+
+// One operand set of the grouped GEMM: `groups` groups that share tensor maps.
+// Group gi multiplies A rows [gi*a_group_stride, +M) by the B rows
+// [offsets[gi], +counts[gi]) and writes output rows at the same B row index
+// (EPI_SWIGLU: bf16 [rows][ld_out]; EPI_STORE_F32: fp32 [rows][ld_out];
+// EPI_ARGMAX: uint64 keys [(M tile)*4 + lane quarter][ld_out]).
+struct GemmSet {
+  CUtensorMap a0;          // A operand (gate weights for EPI_SWIGLU)
+  CUtensorMap a1;          // second A operand (up weights), EPI_SWIGLU only
+  CUtensorMap b;           // B operand, box of 16 rows x 64 columns
+  void* out;
+  const int32_t* counts;   // device [groups] or nullptr (static_rows)
+  const int32_t* offsets;  // device [groups] or nullptr (0)
+  int32_t ld_out;
+  int32_t K;               // reduction length, multiple of 64
+  int32_t M;               // valid A rows per group
+  int32_t groups;
+  int32_t static_rows;
+  int32_t a_group_stride;
+};
+
+struct GemmParams {
+  GemmSet set[2];
+  int32_t nsets;
+  int* err;
+  uint64_t timeout_ns;
+};
+
+cudaError_t launch_gemm(int epi, const GemmParams& p, int grid, cudaStream_t stream);
+
+// Small CUDA-core kernels (kernels_small.cu).
+cudaError_t launch_router(const uint16_t* x, int T, int H, int E, int k, const uint16_t* wr,
+                          const float* bias, int32_t* idx, float* w, cudaStream_t s);
+cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
+                           int32_t* offsets, int32_t* perm, int32_t* inv, const uint16_t* x,
+                           int H, uint16_t* x_perm, cudaStream_t s);
+cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t* inv,
+                           const float* w, const uint16_t* res, uint16_t* out, int T, int H,
+                           int k, int* err, cudaStream_t s);
+cudaError_t launch_lm_finalize(const uint64_t* keys, int nparts, int T, int32_t* argmax,
+                               cudaStream_t s);
+cudaError_t launch_accept(const int32_t* argmax, const int32_t* drafts, int B, int K,
+                          int32_t* accepted, int32_t* next_token, int32_t* emitted,
+                          cudaStream_t s);
+cudaError_t launch_accept_from_keys(const uint64_t* keys, int nparts, const int32_t* drafts,
+                                    int B, int K, int32_t* accepted, int32_t* next_token,
+                                    int32_t* emitted, int32_t* argmax, cudaStream_t s);
+
+}  // namespace mv

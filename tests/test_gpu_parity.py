@@ -1,0 +1,274 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded inputs.
+
+Exact for indices, accepted lengths and tokens (except rows the flag rules
+excuse, which are counted); MoE outputs within max-abs 2e-2 x RMS of the
+oracle's.  Sizes run from the tiny workload through the full model shape.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_decoder_speculative_b200 import binding as bd
+from moe_decoder_speculative_b200 import workloads as wl
+from parity_helpers import (GATE_GAP, LM_GAP, MOE_TOL, gate_flags, moe_error, reference, row_flags)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from moe_decoder_speculative_b200 import build
+    build.build()
+
+
+def dev_layers(inp):
+    return [bd.LayerWeights(l) for l in inp["layers"]]
+
+
+def to_np(t):
+    return t.cpu().numpy()
+
+
+# ---------------------------------------------------------------------------
+# per kernel
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("wid", [0, 1, 4])
+def test_router_topk(wid):
+    w, inp, st = reference(wid)
+    shape = bd.shape_of(w)
+    x = bd.bf16_to_device(inp["hidden"])
+    lw = bd.LayerWeights(inp["layers"][0])
+    idx, tw = bd.moe_router_topk(x, shape, lw.t["w_router"], lw.t["router_bias"])
+    torch.cuda.synchronize()
+    idx, tw = to_np(idx), to_np(tw)
+    ref = st["layers"][0]
+    ok = ref["gap"] >= GATE_GAP
+    np.testing.assert_array_equal(idx[ok], ref["idx"][ok])
+    same = np.all(idx == ref["idx"], axis=1)
+    np.testing.assert_allclose(tw[same], ref["w"][same], rtol=2e-5, atol=2e-6)
+    assert np.all(np.abs(tw.sum(1) - 1) < 1e-5)
+
+
+@pytest.mark.parametrize("T,E,k", [(16, 8, 2), (128, 64, 6), (37, 64, 6), (1, 8, 8), (1000, 256, 8)])
+def test_expert_permute(T, E, k):
+    rng = np.random.default_rng(T * 7 + E)
+    idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    counts, offsets, perm, inv = bd.moe_expert_permute(torch.from_numpy(idx).cuda(), E)
+    torch.cuda.synchronize()
+    flat = idx.reshape(-1)
+    want_perm = np.argsort(flat, kind="stable")
+    np.testing.assert_array_equal(to_np(counts), np.bincount(flat, minlength=E))
+    np.testing.assert_array_equal(to_np(offsets), np.concatenate([[0], np.cumsum(np.bincount(flat, minlength=E))]))
+    np.testing.assert_array_equal(to_np(perm), want_perm)
+    np.testing.assert_array_equal(to_np(perm)[to_np(inv)], np.arange(T * k))
+
+
+@pytest.mark.parametrize("wid", [0, 1, 4])
+def test_moe_ffn_teacher_forced(wid):
+    """GPU MoE layer fed the oracle's input and routing, against the oracle's MoE output."""
+    w, inp, st = reference(wid)
+    shape = bd.shape_of(w)
+    ref = st["layers"][0]
+    lw = bd.LayerWeights(inp["layers"][0])
+    x = bd.bf16_to_device(ref["h_in"])
+    idx = torch.from_numpy(ref["idx"]).cuda()
+    tw = torch.from_numpy(ref["w"]).cuda()
+    out = bd.moe_ffn_forward(x, shape, lw, idx, tw)           # bf16(m)
+    out_r = bd.moe_ffn_forward(x, shape, lw, idx, tw, residual=x)
+    torch.cuda.synchronize()
+    m_gpu = wl.bf16_bits_to_f32(bd.bf16_from_device(out))
+    assert moe_error(m_gpu, ref["m"]) <= MOE_TOL
+    h_gpu = wl.bf16_bits_to_f32(bd.bf16_from_device(out_r))
+    h_ref = wl.bf16_bits_to_f32(st["h"] if len(st["layers"]) == 1 else st["layers"][1]["h_in"])
+    assert np.max(np.abs(h_gpu - h_ref)) <= MOE_TOL * np.sqrt(np.mean(ref["m"].astype(np.float64) ** 2)) + \
+        np.max(np.abs(h_ref)) * 2.0 ** -8
+
+
+@pytest.mark.parametrize("wid", [0, 1, 4])
+def test_lm_head_argmax(wid):
+    w, inp, st = reference(wid)
+    h = bd.bf16_to_device(st["h"])
+    wlm = bd.bf16_to_device(inp["w_lm"])
+    am = to_np(bd.lm_head_argmax(h, wlm))
+    # the LM check alone: the oracle's own h, so only the LM gap excuses a row
+    ok = st["lm_gap"] >= LM_GAP
+    np.testing.assert_array_equal(am[ok], st["argmax"][ok])
+    if "tie_rows" in inp:     # exact ties resolve to the lower index on both sides
+        exact = st["lm_gap"] == 0
+        np.testing.assert_array_equal(am[exact], st["argmax"][exact])
+
+
+def test_lm_head_ragged_vocab_and_rows():
+    """V not a multiple of the 128-row tile, T spanning a ragged N tile."""
+    rng = np.random.default_rng(5)
+    T, H, V = 150, 192, 1000
+    h = wl.f32_to_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    wlm = wl.f32_to_bf16_bits(rng.standard_normal((V, H)).astype(np.float32) * 0.05)
+    ref, _, gap = oracle.lm_head_argmax(h, wlm)
+    am = to_np(bd.lm_head_argmax(bd.bf16_to_device(h), bd.bf16_to_device(wlm)))
+    ok = gap >= LM_GAP
+    np.testing.assert_array_equal(am[ok], ref[ok])
+
+
+def test_greedy_accept_exhaustive():
+    rng = np.random.default_rng(6)
+    for K in (0, 1, 3, 7):
+        B, V = 4096, 3
+        g = rng.integers(0, V, size=(B, K + 1)).astype(np.int32)
+        d = rng.integers(-1, V + 1, size=(B, K)).astype(np.int32)   # includes out-of-range drafts
+        acc, nxt, em = bd.greedy_accept(torch.from_numpy(g.reshape(-1)).cuda(),
+                                        torch.from_numpy(d).cuda() if K else None, B, K)
+        ra, rn, re = oracle.greedy_accept(g.reshape(-1), d, B, K)
+        np.testing.assert_array_equal(to_np(acc), ra)
+        np.testing.assert_array_equal(to_np(nxt), rn)
+        np.testing.assert_array_equal(to_np(em), re)
+
+
+# ---------------------------------------------------------------------------
+# the whole verify step
+# ---------------------------------------------------------------------------
+
+def run_verify(w, inp, drafts):
+    shape = bd.shape_of(w)
+    layers = dev_layers(inp)
+    plan = bd.VerifyPlan(shape, layers, bd.bf16_to_device(inp["w_lm"]), w.B, w.K)
+    hidden = bd.bf16_to_device(inp["hidden"])
+    d = torch.from_numpy(drafts).cuda()
+    acc, nxt, em, am = plan(hidden, d)
+    plan.sync_status()
+    return plan, hidden, d, to_np(acc), to_np(nxt), to_np(em), to_np(am)
+
+
+def check_verify(w, st, acc, nxt, em, am):
+    flags = row_flags(st)
+    ok = ~flags
+    mism = am != st["argmax"]
+    assert not np.any(mism & ok), f"{int(np.sum(mism & ok))} unflagged rows disagree"
+    seq_ok = ok.reshape(w.B, w.K + 1).all(1)
+    np.testing.assert_array_equal(acc[seq_ok], st["accepted"][seq_ok])
+    np.testing.assert_array_equal(nxt[seq_ok], st["next_token"][seq_ok])
+    np.testing.assert_array_equal(em[seq_ok], st["emitted"][seq_ok])
+    assert np.all((acc >= 0) & (acc <= w.K))
+    return {"flagged_rows": int(flags.sum()), "flagged_mismatch": int(np.sum(mism & flags)),
+            "clean_seqs": int(seq_ok.sum())}
+
+
+@pytest.mark.parametrize("wid", [0, 1, 4])
+def test_verify_step(wid):
+    w, inp, st = reference(wid)
+    _, _, _, acc, nxt, em, am = run_verify(w, inp, st["drafts"])
+    info = check_verify(w, st, acc, nxt, em, am)
+    assert info["clean_seqs"] >= 0.5 * w.B or wid == 0
+
+
+@pytest.mark.slow
+def test_verify_step_conc32_12_layers():
+    """The headline workload: 32 sequences x (K+1=4) rows through 12 layers."""
+    w, inp, st = reference(2)
+    plan, hidden, d, acc, nxt, em, am = run_verify(w, inp, st["drafts"])
+    info = check_verify(w, st, acc, nxt, em, am)
+    assert info["clean_seqs"] >= 16
+    # every layer's MoE output, teacher-forced on the oracle's h_l and routing
+    shape = bd.shape_of(w)
+    for l, ref in enumerate(st["layers"]):
+        out = bd.moe_ffn_forward(bd.bf16_to_device(ref["h_in"]), shape, plan.layers[l],
+                                 torch.from_numpy(ref["idx"]).cuda(), torch.from_numpy(ref["w"]).cuda())
+        m_gpu = wl.bf16_bits_to_f32(bd.bf16_from_device(out))
+        assert moe_error(m_gpu, ref["m"]) <= MOE_TOL, f"layer {l}"
+
+
+def test_verify_step_equals_its_calls():
+    """verify_step is bit-identical to router -> ffn (x L) -> lm_head_argmax -> accept."""
+    w, inp, st = reference(0)
+    plan, hidden, d, acc, nxt, em, am = run_verify(w, inp, st["drafts"])
+    shape = bd.shape_of(w)
+    h = hidden
+    for lw in plan.layers:
+        idx, tw = bd.moe_router_topk(h, shape, lw.t["w_router"], lw.t["router_bias"])
+        h = bd.moe_ffn_forward(h, shape, lw, idx, tw, residual=h)
+    am2 = bd.lm_head_argmax(h, plan.w_lm)
+    a2, n2, e2 = bd.greedy_accept(am2, d, w.B, w.K)
+    np.testing.assert_array_equal(to_np(am2), am)
+    np.testing.assert_array_equal(to_np(a2), acc)
+    np.testing.assert_array_equal(to_np(n2), nxt)
+    np.testing.assert_array_equal(to_np(e2), em)
+
+
+def test_k0_is_plain_greedy():
+    """Speculation off (K=0): one row per sequence, the next token is its argmax."""
+    w0 = wl.workload(0)
+    _, inp, st = reference(0)
+    B = 16
+    hidden = inp["hidden"][:B]
+    shape = bd.shape_of(w0)
+    plan = bd.VerifyPlan(shape, dev_layers(inp), bd.bf16_to_device(inp["w_lm"]), B, 0)
+    acc, nxt, em, am = plan(bd.bf16_to_device(hidden), None)
+    ref = oracle.verify_step(hidden, None, B, 0, inp["layers"], w0.k, inp["w_lm"])
+    ok = ~row_flags(ref)
+    assert np.all(to_np(acc) == 0)
+    np.testing.assert_array_equal(to_np(nxt)[ok], ref["argmax"][ok])
+    np.testing.assert_array_equal(to_np(em)[:, 0], to_np(nxt))
+
+
+def test_batch_invariance_and_determinism():
+    """A sequence's result does not depend on the other sequences in the batch,
+    and repeated runs give identical bits."""
+    w, inp, st = reference(1)
+    wb = wl.workload(1)
+    shape = bd.shape_of(wb)
+    layers = dev_layers(inp)
+    wlm = bd.bf16_to_device(inp["w_lm"])
+    rng = np.random.default_rng(9)
+    other = wl.f32_to_bf16_bits(rng.standard_normal((12, wb.H)).astype(np.float32))
+    big = np.concatenate([other[:4], inp["hidden"], other[4:]])   # our sequence is number 1 of 4
+    d_big = np.concatenate([rng.integers(0, wb.V, (1, 3)), st["drafts"], rng.integers(0, wb.V, (2, 3))]).astype(np.int32)
+    p1 = bd.VerifyPlan(shape, layers, wlm, 1, 3)
+    p4 = bd.VerifyPlan(shape, layers, wlm, 4, 3)
+    r1 = [to_np(t).copy() for t in p1(bd.bf16_to_device(inp["hidden"]), torch.from_numpy(st["drafts"]).cuda())]
+    r1b = [to_np(t).copy() for t in p1(bd.bf16_to_device(inp["hidden"]), torch.from_numpy(st["drafts"]).cuda())]
+    r4 = [to_np(t).copy() for t in p4(bd.bf16_to_device(big), torch.from_numpy(d_big).cuda())]
+    for a, b in zip(r1, r1b):
+        np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(r4[3][4:8], r1[3])       # argmax rows
+    assert r4[0][1] == r1[0][0] and r4[1][1] == r1[1][0]
+
+
+def test_skewed_routing_flag_path():
+    """Four hot experts take about half the slots; about 5% of rows carry
+    near-tied LM logits; everything unflagged is exact."""
+    w, inp, st = reference(4)
+    hot = wl.hot_experts(w)
+    share = np.isin(st["layers"][0]["idx"], hot).mean()
+    assert abs(share - 0.5) <= 0.01
+    assert np.sum(st["lm_gap"] < LM_GAP) >= 0.04 * w.T
+    _, _, _, acc, nxt, em, am = run_verify(w, inp, st["drafts"])
+    check_verify(w, st, acc, nxt, em, am)
+
+
+def test_prefill_layer_sampled_rows():
+    """The 9,248-row prefill layer on the GPU; the oracle checks routing on every
+    row and the MoE output on a sample of rows spread over the batch."""
+    w = wl.workload(3)
+    inp = wl.make_inputs(w)
+    shape = bd.shape_of(w)
+    x = inp["hidden"]
+    lay = inp["layers"][0]
+    idx_ref, w_ref, _, gap = oracle.router(x, lay["w_router"], w.k)
+    lw = bd.LayerWeights(lay)
+    xd = bd.bf16_to_device(x)
+    idx, tw = bd.moe_router_topk(xd, shape, lw.t["w_router"], None)
+    out = bd.moe_ffn_forward(xd, shape, lw, idx, tw)
+    torch.cuda.synchronize()
+    idx = to_np(idx)
+    ok = gap >= GATE_GAP
+    np.testing.assert_array_equal(idx[ok], idx_ref[ok])
+    rows = np.unique(np.concatenate([np.arange(0, w.T, 37), [w.T - 1]]))
+    rows = rows[np.all(idx[rows] == idx_ref[rows], axis=1)]
+    m_ref, _ = oracle.moe_ffn(x[rows], lay, idx_ref[rows], w_ref[rows])
+    m_gpu = wl.bf16_bits_to_f32(bd.bf16_from_device(out))[rows]
+    assert moe_error(m_gpu, m_ref) <= MOE_TOL
