@@ -298,7 +298,8 @@ mv_status ffn_forward_impl(const uint16_t* x, int T, const mv_moe_shape& s, cons
   });
   if (e != cudaSuccess) return cuda_fail(e, "expert_permute launch");
 
-  constexpr int BN = 128;
+  // decode configuration when routed groups average 16 rows or fewer
+  const int BN = (static_cast<int64_t>(n) <= 16LL * E) ? 32 : 128;
   // gate + up with the SwiGLU epilogue
   {
     mv::GemmParams p;
@@ -336,7 +337,7 @@ mv_status ffn_forward_impl(const uint16_t* x, int T, const mv_moe_shape& s, cons
       units += int64_t((I + 127) / 128) * (std::min(E, n) + (n + BN - 1) / BN);
     }
     p.nsets = ns;
-    e = run_kernel(KIND_GEMM_SWIGLU, st, [&] { return mv::launch_gemm(mv::EPI_SWIGLU, p, gemm_grid(units), st); });
+    e = run_kernel(KIND_GEMM_SWIGLU, st, [&] { return mv::launch_gemm(mv::EPI_SWIGLU, BN, p, gemm_grid(units), st); });
     if (e != cudaSuccess) return cuda_fail(e, "grouped_swiglu_gemm launch");
   }
   // down projection, fp32 rows
@@ -376,7 +377,7 @@ mv_status ffn_forward_impl(const uint16_t* x, int T, const mv_moe_shape& s, cons
       units += int64_t((H + 127) / 128) * (std::min(E, n) + (n + BN - 1) / BN);
     }
     p.nsets = ns;
-    e = run_kernel(KIND_GEMM_DOWN, st, [&] { return mv::launch_gemm(mv::EPI_STORE_F32, p, gemm_grid(units), st); });
+    e = run_kernel(KIND_GEMM_DOWN, st, [&] { return mv::launch_gemm(mv::EPI_STORE_F32, BN, p, gemm_grid(units), st); });
     if (e != cudaSuccess) return cuda_fail(e, "grouped_down_gemm launch");
   }
   e = run_kernel(KIND_COMBINE, st, [&] {
@@ -397,14 +398,14 @@ mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, in
   MV_TRY(tmap(&S.b, h, T, H, 16));
   S.a1 = S.a0;
   S.out = parts;
-  S.ld_out = T;
+  S.ld_out = lm_parts(V);
   S.K = H;
   S.M = V;
   S.groups = 1;
   S.static_rows = T;
   p.nsets = 1;
   const int64_t units = int64_t((V + 127) / 128) * ((T + 127) / 128);
-  cudaError_t e = run_kernel(KIND_LM_GEMM, st, [&] { return mv::launch_gemm(mv::EPI_ARGMAX, p, gemm_grid(units), st); });
+  cudaError_t e = run_kernel(KIND_LM_GEMM, st, [&] { return mv::launch_gemm(mv::EPI_ARGMAX, 128, p, gemm_grid(units), st); });
   if (e != cudaSuccess) return cuda_fail(e, "lm_head_gemm_argmax launch");
   return MV_OK;
 }

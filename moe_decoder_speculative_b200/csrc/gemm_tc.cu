@@ -360,8 +360,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           const int n = c0 + lane;
           if (n < ui.nvalid) {
             uint64_t* out = static_cast<uint64_t*>(S.out);
-            const int prow = (ui.m0 / 128) * 4 + wq;  // partial row: (M tile, lane quarter)
-            out[static_cast<size_t>(prow) * S.ld_out + ui.b_row0 + n] =
+            const int part = (ui.m0 / 128) * 4 + wq;  // (M tile, lane quarter); keys are token-major
+            out[static_cast<size_t>(ui.b_row0 + n) * S.ld_out + part] =
                 argmax_key(best, static_cast<uint32_t>(ui.m0 + wq * 32 + bi));
           }
         }
@@ -401,15 +401,16 @@ static cudaError_t launch_gemm_impl(const GemmParams& p, int grid, cudaStream_t 
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(int epi, const GemmParams& p, int grid, cudaStream_t stream) {
-  switch (epi) {
-    case EPI_SWIGLU:
-      return launch_gemm_impl<EPI_SWIGLU, 128, 4>(p, grid, stream);
-    case EPI_STORE_F32:
-      return launch_gemm_impl<EPI_STORE_F32, 128, 6>(p, grid, stream);
-    case EPI_ARGMAX:
-      return launch_gemm_impl<EPI_ARGMAX, 128, 6>(p, grid, stream);
-  }
+// Tile configurations.  bn = 32 is the decode configuration (a few tokens per
+// expert): the B tile shrinks to 4 KB per stage so 6 (gate/up) or 10 (down)
+// stages keep 192 / 160 KB of weights in flight per SM.  bn = 128 serves
+// larger groups and the LM head.
+cudaError_t launch_gemm(int epi, int bn, const GemmParams& p, int grid, cudaStream_t stream) {
+  if (epi == EPI_SWIGLU && bn == 32) return launch_gemm_impl<EPI_SWIGLU, 32, 6>(p, grid, stream);
+  if (epi == EPI_SWIGLU && bn == 128) return launch_gemm_impl<EPI_SWIGLU, 128, 4>(p, grid, stream);
+  if (epi == EPI_STORE_F32 && bn == 32) return launch_gemm_impl<EPI_STORE_F32, 32, 10>(p, grid, stream);
+  if (epi == EPI_STORE_F32 && bn == 128) return launch_gemm_impl<EPI_STORE_F32, 128, 6>(p, grid, stream);
+  if (epi == EPI_ARGMAX && bn == 128) return launch_gemm_impl<EPI_ARGMAX, 128, 6>(p, grid, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -26,6 +26,63 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
+// Top-k of one row's E logits (held in shared memory) by one warp: k rounds
+// of a warp argmax (larger logit wins, equal logits -> lower expert id), then
+// the renormalised softmax weights exp(l_j - l_max) / sum_selected.
+__device__ __forceinline__ void topk_select_row(const float* lrow, int E, int k, int lane,
+                                                int32_t* idx_out, float* w_out) {
+  constexpr int kMaxPer = 8;  // E <= 256
+  float v[kMaxPer];
+  const int per = (E + 31) / 32;
+#pragma unroll
+  for (int q = 0; q < kMaxPer; ++q) {
+    const int e = lane + 32 * q;
+    v[q] = (q < per && e < E) ? lrow[e] : -__int_as_float(0x7f800000);
+  }
+  float selv[8];
+  int sele[8];
+  for (int j = 0; j < k; ++j) {
+    float bv = -__int_as_float(0x7f800000);
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int q = 0; q < kMaxPer; ++q) {
+      const int e = lane + 32 * q;
+      if (q < per && e < E && better(v[q], e, bv, bi)) {
+        bv = v[q];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (better(ov, oi, bv, bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    selv[j] = bv;
+    sele[j] = bi;
+#pragma unroll
+    for (int q = 0; q < kMaxPer; ++q)
+      if (lane + 32 * q == bi) v[q] = -__int_as_float(0x7f800000);
+  }
+  const float mx = selv[0];
+  float s = 0.f;
+  for (int j = 0; j < k; ++j) s += expf(selv[j] - mx);
+  if (lane < k) {
+    float my_v = selv[0];
+    int my_e = sele[0];
+    for (int j = 1; j < k; ++j)
+      if (j == lane) {
+        my_v = selv[j];
+        my_e = sele[j];
+      }
+    idx_out[lane] = my_e;
+    w_out[lane] = expf(my_v - mx) / s;
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -86,60 +143,79 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const uint16_t* __rest
   }
   __syncthreads();
 
-  if (warp < nrows) {
-    const int r = warp;
-    constexpr int kMaxPer = 8;  // E <= 256
-    float v[kMaxPer];
-    const int per = (E + 31) / 32;
-#pragma unroll
-    for (int q = 0; q < kMaxPer; ++q) {
-      const int e = lane + 32 * q;
-      v[q] = (q < per && e < E) ? ls[r * E + e] : -__int_as_float(0x7f800000);
+  if (warp < nrows)
+    topk_select_row(ls + warp * E, E, k, lane, idx + static_cast<size_t>(row0 + warp) * k,
+                    wout + static_cast<size_t>(row0 + warp) * k);
+}
+
+// Router with the whole router weight matrix staged in shared memory
+// (E*H bf16, 160 KB at the model shape) by cp.async 16-byte copies, all issued
+// before any is waited on; each CTA then loops over blocks of R rows.  Same
+// arithmetic and selection as router_topk_kernel.
+template <int R>
+__global__ void __launch_bounds__(256, 1) router_smem_kernel(const uint16_t* __restrict__ x, int T,
+                                                          int H, int E, int k,
+                                                          const uint16_t* __restrict__ wr,
+                                                          const float* __restrict__ bias,
+                                                          int32_t* __restrict__ idx,
+                                                          float* __restrict__ wout) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  uint16_t* wsm = reinterpret_cast<uint16_t*>(sm);                            // [E][H]
+  uint16_t* xs = wsm + static_cast<size_t>(E) * H;                           // [R][H]
+  float* ls = reinterpret_cast<float*>(xs + static_cast<size_t>(R) * H);      // [R][E]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int hv = H / 8;
+  const int nvec = E * hv;
+  for (int i = tid; i < nvec; i += blockDim.x) {
+    const uint32_t dst = smem_u32(wsm + static_cast<size_t>(i) * 8);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(wr + static_cast<size_t>(i) * 8)
+                 : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  const int nblocks = (T + R - 1) / R;
+  bool first = true;
+  for (int rb = blockIdx.x; rb < nblocks; rb += gridDim.x) {
+    const int row0 = rb * R;
+    const int nrows = min(R, T - row0);
+    for (int i = tid; i < R * hv; i += blockDim.x) {
+      const int r = i / hv, c = i % hv;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (r < nrows) v = reinterpret_cast<const uint4*>(x + static_cast<size_t>(row0 + r) * H)[c];
+      reinterpret_cast<uint4*>(xs + static_cast<size_t>(r) * H)[c] = v;
     }
-    float selv[8];
-    int sele[8];
-    for (int j = 0; j < k; ++j) {
-      float bv = -__int_as_float(0x7f800000);
-      int bi = 0x7fffffff;
+    if (first) {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      first = false;
+    }
+    __syncthreads();
+    for (int e = warp; e < E; e += 8) {
+      float acc[R];
 #pragma unroll
-      for (int q = 0; q < kMaxPer; ++q) {
-        const int e = lane + 32 * q;
-        if (q < per && e < E && better(v[q], e, bv, bi)) {
-          bv = v[q];
-          bi = e;
+      for (int r = 0; r < R; ++r) acc[r] = 0.f;
+      const uint4* we = reinterpret_cast<const uint4*>(wsm + static_cast<size_t>(e) * H);
+      for (int c = lane; c < hv; c += 32) {
+        float wf[8];
+        bf16x8_to_f32(we[c], wf);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          float xf[8];
+          bf16x8_to_f32(reinterpret_cast<const uint4*>(xs + static_cast<size_t>(r) * H)[c], xf);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[r] = fmaf(xf[j], wf[j], acc[r]);
         }
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (better(ov, oi, bv, bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      selv[j] = bv;
-      sele[j] = bi;
-      // the lane holding the winner removes it from further rounds
+      for (int r = 0; r < R; ++r) {
+        float v = acc[r];
 #pragma unroll
-      for (int q = 0; q < kMaxPer; ++q)
-        if (lane + 32 * q == bi) v[q] = -__int_as_float(0x7f800000);
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) ls[r * E + e] = bias ? v + bias[e] : v;
+      }
     }
-    const float mx = selv[0];
-    float s = 0.f;
-    for (int j = 0; j < k; ++j) s += expf(selv[j] - mx);
-    if (lane < k) {
-      float my_v = selv[0];
-      int my_e = sele[0];
-      for (int j = 1; j < k; ++j)
-        if (j == lane) {
-          my_v = selv[j];
-          my_e = sele[j];
-        }
-      const size_t o = static_cast<size_t>(row0 + r) * k + lane;
-      idx[o] = my_e;
-      wout[o] = expf(my_v - mx) / s;
-    }
+    __syncthreads();
+    if (warp < nrows) topk_select_row(ls + warp * E, E, k, lane, idx + static_cast<size_t>(row0 + warp) * k,
+                                      wout + static_cast<size_t>(row0 + warp) * k);
+    __syncthreads();
   }
 }
 
@@ -150,16 +226,40 @@ static void launch_router_r(const uint16_t* x, int T, int H, int E, int k, const
   router_topk_kernel<R><<<(T + R - 1) / R, 256, smem, s>>>(x, T, H, E, k, wr, bias, idx, w);
 }
 
-// Rows per CTA: 4 for decode-sized batches (more CTAs share the router weight
-// stream), 8 for large batches; fewer when the rows would not fit in 48 KB of
-// shared memory.
+template <int R>
+static cudaError_t launch_router_smem(const uint16_t* x, int T, int H, int E, int k, const uint16_t* wr,
+                                      const float* bias, int32_t* idx, float* w, cudaStream_t s, size_t smem) {
+  static thread_local int configured_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_dev != dev) {
+    cudaError_t e = cudaFuncSetAttribute(router_smem_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         220 * 1024);
+    if (e != cudaSuccess) return e;
+    configured_dev = dev;
+  }
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int nblocks = (T + R - 1) / R;
+  router_smem_kernel<R><<<min(nblocks, sms), 256, smem, s>>>(x, T, H, E, k, wr, bias, idx, w);
+  return cudaGetLastError();
+}
+
+// Rows per block: 4 for decode-sized batches (more CTAs share the work), 8 for
+// large ones.  The router weights go to shared memory when they fit (E*H*2 up
+// to ~200 KB); otherwise the global-load kernel streams them.
 cudaError_t launch_router(const uint16_t* x, int T, int H, int E, int k, const uint16_t* wr,
                           const float* bias, int32_t* idx, float* w, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  auto fits = [&](int R) { return static_cast<size_t>(R) * H * 2 + static_cast<size_t>(R) * E * 4 <= 48 * 1024; };
-  int R = (T <= 1024) ? 4 : 8;
-  while (R > 1 && !fits(R)) R >>= 1;
-  switch (R) {
+  const int R = (T <= 1024) ? 4 : 8;
+  const size_t smem_v2 = static_cast<size_t>(E) * H * 2 + static_cast<size_t>(R) * H * 2 + static_cast<size_t>(R) * E * 4;
+  if (smem_v2 <= 200 * 1024)
+    return R == 4 ? launch_router_smem<4>(x, T, H, E, k, wr, bias, idx, w, s, smem_v2)
+                  : launch_router_smem<8>(x, T, H, E, k, wr, bias, idx, w, s, smem_v2);
+  auto fits = [&](int r) { return static_cast<size_t>(r) * H * 2 + static_cast<size_t>(r) * E * 4 <= 48 * 1024; };
+  int r = R;
+  while (r > 1 && !fits(r)) r >>= 1;
+  switch (r) {
     case 8: launch_router_r<8>(x, T, H, E, k, wr, bias, idx, w, s); break;
     case 4: launch_router_r<4>(x, T, H, E, k, wr, bias, idx, w, s); break;
     case 2: launch_router_r<2>(x, T, H, E, k, wr, bias, idx, w, s); break;
@@ -333,39 +433,47 @@ cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t
 }
 
 // ---------------------------------------------------------------------------
-// LM-head argmax finalisation: the GEMM epilogue leaves one packed
-// (order-preserving logit, inverted index) key per (32-row vocabulary block,
-// token); the largest key is the argmax with ties to the lower index.
+// LM-head argmax finalisation: the GEMM epilogue leaves, per token, one packed
+// (order-preserving logit, inverted index) key per 32-row vocabulary block,
+// token-major ([T][nparts]); the largest key is the argmax with ties to the
+// lower index.  `nthr` threads (a multiple of 32) reduce one token's keys with
+// coalesced, unrolled loads.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint64_t max_key_over_parts(const uint64_t* keys, int nparts, int T,
-                                                       int t, int lane) {
-  uint64_t best = 0;
-  for (int p = lane; p < nparts; p += 32) {
-    const uint64_t v = keys[static_cast<size_t>(p) * T + t];
-    best = v > best ? v : best;
+__device__ __forceinline__ uint64_t umax64(uint64_t a, uint64_t b) { return a > b ? a : b; }
+
+__device__ __forceinline__ uint64_t row_max_key(const uint64_t* row, int nparts, int t0, int nthr,
+                                                uint64_t* red, int lane, int wid) {
+  uint64_t b0 = 0, b1 = 0, b2 = 0, b3 = 0;
+  int p = t0;
+  for (; p + 3 * nthr < nparts; p += 4 * nthr) {
+    b0 = umax64(b0, row[p]);
+    b1 = umax64(b1, row[p + nthr]);
+    b2 = umax64(b2, row[p + 2 * nthr]);
+    b3 = umax64(b3, row[p + 3 * nthr]);
   }
+  for (; p < nparts; p += nthr) b0 = umax64(b0, row[p]);
+  uint64_t best = umax64(umax64(b0, b1), umax64(b2, b3));
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const uint64_t v = __shfl_xor_sync(0xffffffffu, best, o);
-    best = v > best ? v : best;
-  }
+  for (int o = 16; o > 0; o >>= 1) best = umax64(best, __shfl_xor_sync(0xffffffffu, best, o));
+  if (lane == 0) red[wid] = best;
   return best;
 }
 
-__global__ void __launch_bounds__(256) lm_finalize_kernel(const uint64_t* __restrict__ keys,
-                                                          int nparts, int T,
-                                                          int32_t* __restrict__ argmax) {
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t >= T) return;
-  const uint64_t best = max_key_over_parts(keys, nparts, T, t, lane);
-  if (lane == 0) argmax[t] = static_cast<int32_t>(argmax_key_index(best));
+__global__ void __launch_bounds__(128) lm_finalize_kernel(const uint64_t* __restrict__ keys, int nparts,
+                                                          int T, int32_t* __restrict__ argmax) {
+  __shared__ uint64_t red[4];
+  const int t = blockIdx.x;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  row_max_key(keys + static_cast<size_t>(t) * nparts, nparts, threadIdx.x, 128, red, lane, wid);
+  __syncthreads();
+  if (threadIdx.x == 0)
+    argmax[t] = static_cast<int32_t>(argmax_key_index(umax64(umax64(red[0], red[1]), umax64(red[2], red[3]))));
 }
 
 cudaError_t launch_lm_finalize(const uint64_t* keys, int nparts, int T, int32_t* argmax,
                                cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  lm_finalize_kernel<<<(T + 7) / 8, 256, 0, s>>>(keys, nparts, T, argmax);
+  lm_finalize_kernel<<<T, 128, 0, s>>>(keys, nparts, T, argmax);
   return cudaGetLastError();
 }
 
@@ -401,24 +509,32 @@ cudaError_t launch_accept(const int32_t* argmax, const int32_t* drafts, int B, i
   return cudaGetLastError();
 }
 
-// Fused LM finalisation + acceptance: one CTA per sequence, warp j finalises
-// row b*(K+1)+j, then one thread accepts.
-__global__ void __launch_bounds__(256) accept_from_keys_kernel(
+// Fused LM finalisation + acceptance: one CTA per sequence; 4 warps reduce
+// each of its K+1 rows (up to 8 rows at a time), then one thread accepts.
+__global__ void __launch_bounds__(1024) accept_from_keys_kernel(
     const uint64_t* __restrict__ keys, int nparts, const int32_t* __restrict__ drafts, int B, int K,
     int32_t* accepted, int32_t* next_token, int32_t* emitted, int32_t* argmax_out) {
   __shared__ int32_t g[64];
+  __shared__ uint64_t red[32];
   const int b = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int T = B * (K + 1);
-  for (int j = warp; j <= K; j += blockDim.x >> 5) {
-    const int t = b * (K + 1) + j;
-    const uint64_t best = max_key_over_parts(keys, nparts, T, t, lane);
-    if (lane == 0) {
-      g[j] = static_cast<int32_t>(argmax_key_index(best));
-      if (argmax_out) argmax_out[t] = g[j];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int rows_at_once = blockDim.x / 128;
+  const int sub = threadIdx.x / 128;          // which row of the group this thread serves
+  const int t_in = threadIdx.x % 128;
+  for (int j0 = 0; j0 <= K; j0 += rows_at_once) {
+    const int j = j0 + sub;
+    if (j <= K) {
+      const int t = b * (K + 1) + j;
+      row_max_key(keys + static_cast<size_t>(t) * nparts, nparts, t_in, 128, red, lane, wid);
     }
+    __syncthreads();
+    if (t_in == 0 && j <= K) {
+      const uint64_t* r4 = red + sub * 4;
+      g[j] = static_cast<int32_t>(argmax_key_index(umax64(umax64(r4[0], r4[1]), umax64(r4[2], r4[3]))));
+      if (argmax_out) argmax_out[b * (K + 1) + j] = g[j];
+    }
+    __syncthreads();
   }
-  __syncthreads();
   if (threadIdx.x == 0)
     accept_one(g, drafts ? drafts + static_cast<size_t>(b) * K : nullptr, K, b, accepted,
                next_token, emitted);
@@ -428,9 +544,9 @@ cudaError_t launch_accept_from_keys(const uint64_t* keys, int nparts, const int3
                                     int B, int K, int32_t* accepted, int32_t* next_token,
                                     int32_t* emitted, int32_t* argmax, cudaStream_t s) {
   if (B <= 0) return cudaSuccess;
-  const int warps = min(8, K + 1);
-  accept_from_keys_kernel<<<B, warps * 32, 0, s>>>(keys, nparts, drafts, B, K, accepted,
-                                                    next_token, emitted, argmax);
+  const int rows_at_once = min(8, K + 1);
+  accept_from_keys_kernel<<<B, 128 * rows_at_once, 0, s>>>(keys, nparts, drafts, B, K, accepted,
+                                                           next_token, emitted, argmax);
   return cudaGetLastError();
 }
 

@@ -18,7 +18,7 @@ constexpr int kErrInternal = 2;
 // Group gi multiplies A rows [gi*a_group_stride, +M) by the B rows
 // [offsets[gi], +counts[gi]) and writes output rows at the same B row index
 // (EPI_SWIGLU: bf16 [rows][ld_out]; EPI_STORE_F32: fp32 [rows][ld_out];
-// EPI_ARGMAX: uint64 keys [(M tile)*4 + lane quarter][ld_out]).
+// EPI_ARGMAX: uint64 keys [row][ld_out], one per (M tile, lane quarter)).
 struct GemmSet {
   CUtensorMap a0;          // A operand (gate weights for EPI_SWIGLU)
   CUtensorMap a1;          // second A operand (up weights), EPI_SWIGLU only
@@ -41,7 +41,7 @@ struct GemmParams {
   uint64_t timeout_ns;
 };
 
-cudaError_t launch_gemm(int epi, const GemmParams& p, int grid, cudaStream_t stream);
+cudaError_t launch_gemm(int epi, int bn, const GemmParams& p, int grid, cudaStream_t stream);
 
 // Small CUDA-core kernels (kernels_small.cu).
 cudaError_t launch_router(const uint16_t* x, int T, int H, int E, int k, const uint16_t* wr,

@@ -103,3 +103,33 @@ def moe_error(m_gpu: np.ndarray, m_ref: np.ndarray) -> float:
     """max |gpu - ref| / RMS(ref)."""
     rms = float(np.sqrt(np.mean(m_ref.astype(np.float64) ** 2)))
     return float(np.max(np.abs(m_gpu.astype(np.float64) - m_ref)) / rms)
+
+
+def drift_excused(st, w_lm, router_ws, gpu_h):
+    """Rows excused end to end by input drift.
+
+    Through a stack of layers the GPU's hidden states drift from the oracle's by
+    bf16 rounding flips (any change of fp32 summation order does this; the
+    oracle's own float and double modes drift the same way).  A routing choice
+    at layer l can only differ if the oracle's k-th vs (k+1)-th gap is below
+    2 * max_e |dh_l . W_r[e]| (dh_l = GPU input minus oracle input, exact in
+    float64), plus the fp32 allowance GATE_GAP; the LM choice likewise with the
+    LM-head rows and LM_GAP.  Returns (excused rows, per-layer bound).
+    """
+    T = len(st["h"])
+    ex = np.zeros(T, bool)
+    bounds = []
+    for l, lay in enumerate(st["layers"]):
+        dh = wl.bf16_bits_to_f32(gpu_h[l]).astype(np.float64) - wl.bf16_bits_to_f32(lay["h_in"])
+        wr = wl.bf16_bits_to_f32(router_ws[l]).astype(np.float64)
+        b = np.max(np.abs(dh @ wr.T), axis=1)
+        bounds.append(b)
+        ex |= lay["gap"] < GATE_GAP + 2 * b
+    dh = wl.bf16_bits_to_f32(gpu_h[-1]).astype(np.float64) - wl.bf16_bits_to_f32(st["h"])
+    b_lm = np.zeros(T)
+    wlm = wl.bf16_bits_to_f32(w_lm)
+    for v0 in range(0, wlm.shape[0], 16384):
+        b_lm = np.maximum(b_lm, np.max(np.abs(dh @ wlm[v0:v0 + 16384].astype(np.float64).T), axis=1))
+    bounds.append(b_lm)
+    ex |= st["lm_gap"] < LM_GAP + 2 * b_lm
+    return ex, bounds
