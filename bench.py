@@ -78,7 +78,8 @@ def source_digest(files):
     return h.hexdigest()[:16]
 
 
-GEMM_SOURCES = ["moe_decoder_speculative_b200/csrc/gemm_tc.cu", "moe_decoder_speculative_b200/csrc/mv_device.cuh"]
+GEMM_SOURCES = ["moe_decoder_speculative_b200/csrc/gemm_tc.cu", "moe_decoder_speculative_b200/csrc/mv_device.cuh",
+                "moe_decoder_speculative_b200/csrc/mv_internal.h"]
 
 
 def ncu_traffic(kernel: str):
@@ -160,15 +161,17 @@ def gpu_uuid(torch, dev):
 
 def algorithmic_bytes(w, touched, T):
     """Per-launch algorithmic bytes of each kernel kind for one verify step.
-    touched[l] = distinct routed experts chosen in layer l."""
+    touched[l] = distinct routed experts chosen in layer l.  The grouped MoE
+    GEMM streams the touched experts' gate/up/down weights and the shared
+    expert once, reads the gathered and plain token rows, writes and re-reads
+    the bf16 SwiGLU activations and writes the fp32 expert outputs."""
     H, I, Ish, k, V, E = w.H, w.I, w.I_sh, w.k, w.V, w.E
     n = T * k
-    L = len(touched)
-    avg_t = float(np.mean(touched)) if L else 0.0
+    avg_t = float(np.mean(touched)) if len(touched) else 0.0
+    act = n * I + T * Ish
     return {
-        "grouped_swiglu_gemm": avg_t * 2 * I * H * 2 + 2 * Ish * H * 2 + (n + T) * H * 2 + (n * I + T * Ish) * 2,
-        "grouped_down_gemm": avg_t * H * I * 2 + H * Ish * 2 + (n * I + T * Ish) * 2 + (n + T) * H * 4,
-        "lm_head_gemm_argmax": V * H * 2 + T * H * 2 + ((V + 127) // 128 * 4) * T * 8,
+        "grouped_moe_gemm": avg_t * 3 * I * H * 2 + 3 * Ish * H * 2 + (n + T) * H * 2 + 2 * act * 2 + (n + T) * H * 4,
+        "lm_head_gemm_argmax": V * H * 2 + T * H * 2 + ((V + 255) // 256 * 4) * T * 8,
         "router_topk": E * H * 2 + T * H * 2 + T * k * 8,
         "expert_permute": n * 4 * 3 + n * H * 2 * 2,
         "combine_unpermute": n * H * 4 + T * H * 4 + T * H * 2 * 2 + n * 12,

@@ -61,17 +61,16 @@ int num_sms() {
 enum Kind {
   KIND_ROUTER = 0,
   KIND_PERMUTE,
-  KIND_GEMM_SWIGLU,
-  KIND_GEMM_DOWN,
+  KIND_GEMM_MOE,
   KIND_COMBINE,
   KIND_LM_GEMM,
   KIND_LM_FINALIZE,
   KIND_ACCEPT,
   KIND_COUNT
 };
-const char* kKindNames[KIND_COUNT] = {"router_topk",     "expert_permute",  "grouped_swiglu_gemm",
-                                      "grouped_down_gemm", "combine_unpermute", "lm_head_gemm_argmax",
-                                      "lm_argmax_finalize", "greedy_accept"};
+const char* kKindNames[KIND_COUNT] = {"router_topk",       "expert_permute",      "grouped_moe_gemm",
+                                      "combine_unpermute", "lm_head_gemm_argmax", "lm_argmax_finalize",
+                                      "greedy_accept"};
 
 struct ProfRec {
   int kind;
@@ -240,6 +239,7 @@ mv_status check_weights(const mv_moe_weights* w, const mv_moe_shape* s) {
 // workspace layouts (every region 1024-byte aligned relative to the base)
 // ---------------------------------------------------------------------------
 constexpr size_t kHeader = 1024;  // sticky error word + reserved
+constexpr size_t kSchedBytes = mv::kSchedInts * sizeof(int);  // scheduling state of one GEMM launch
 
 struct Carve {
   char* base;
@@ -273,7 +273,9 @@ FfnWs carve_ffn(Carve& c, int64_t T, const mv_moe_shape& s) {
   return w;
 }
 
-int lm_parts(int V) { return (V + 127) / 128 * 4; }
+constexpr int kMaxLayers = 64;  // decoder layers one verify_step call may run
+
+int lm_parts(int V) { return (V + 255) / 256 * 4; }  // (256-row vocabulary tile, lane quarter)
 
 uint64_t timeout_ns() {
   const int64_t t = g_timeout_ns.load();
@@ -288,112 +290,130 @@ int gemm_grid(int64_t units) {
 // ---------------------------------------------------------------------------
 // the path
 // ---------------------------------------------------------------------------
-mv_status ffn_forward_impl(const uint16_t* x, int T, const mv_moe_shape& s, const mv_moe_weights& w,
-                           const int32_t* idx, const float* tw, const uint16_t* res, uint16_t* out,
-                           const FfnWs& ws, int* err, cudaStream_t st) {
+// The fused grouped GEMM of one MoE layer: gate/up (SwiGLU epilogue) and down
+// projection (fp32 rows) of the shared expert and the routed experts in one
+// persistent launch; a down unit waits for its expert's gate/up units.
+mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const mv_moe_weights& w,
+                        const FfnWs& ws, int* err, int* sched, cudaStream_t st) {
   const int H = s.H, E = s.E, I = s.I, Ish = s.I_shared, k = s.k;
   const int n = T * k;
+  const bool decode = static_cast<int64_t>(n) <= 16LL * E;  // routed groups average <= 16 rows
+  const int BN = decode ? 32 : 128;
+  mv::GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.err = err;
+  p.sched = sched;
+  p.timeout_ns = timeout_ns();
+  int ns = 0;
+  int64_t units = 0;
+  int sh1 = -1, rt1 = -1;
+  auto base = [](mv::GemmSet& S, int mode, int epi) {
+    S.mode = mode;
+    S.epi = epi;
+    S.m_tile = 128;
+    S.dep_set = -1;
+  };
+  if (Ish > 0) {  // shared expert, gate/up
+    mv::GemmSet& S = p.set[ns];
+    base(S, mv::MODE_GATEUP, mv::EPI_SWIGLU);
+    MV_TRY(tmap(&S.a0, w.ws_gate, Ish, H, 128));
+    MV_TRY(tmap(&S.a1, w.ws_up, Ish, H, 128));
+    MV_TRY(tmap(&S.b, x, T, H, 16));
+    S.out = ws.a_sh;
+    S.ld_out = Ish;
+    S.K = H;
+    S.M = Ish;
+    S.groups = 1;
+    S.static_rows = T;
+    S.signal = 1;
+    units += int64_t((Ish + 127) / 128) * ((T + BN - 1) / BN);
+    sh1 = ns++;
+  }
+  {  // routed experts, gate/up
+    mv::GemmSet& S = p.set[ns];
+    base(S, mv::MODE_GATEUP, mv::EPI_SWIGLU);
+    MV_TRY(tmap(&S.a0, w.w_gate, static_cast<uint64_t>(E) * I, H, 128));
+    MV_TRY(tmap(&S.a1, w.w_up, static_cast<uint64_t>(E) * I, H, 128));
+    MV_TRY(tmap(&S.b, ws.x_perm, n, H, 16));
+    S.out = ws.a_perm;
+    S.ld_out = I;
+    S.K = H;
+    S.M = I;
+    S.groups = E;
+    S.counts = ws.counts;
+    S.offsets = ws.offsets;
+    S.a_group_stride = I;
+    S.signal = 1;
+    units += int64_t((I + 127) / 128) * (std::min(E, n) + (n + BN - 1) / BN);
+    rt1 = ns++;
+  }
+  if (Ish > 0) {  // shared expert, down
+    mv::GemmSet& S = p.set[ns++];
+    base(S, mv::MODE_KPAIR, mv::EPI_STORE_F32);
+    MV_TRY(tmap(&S.a0, w.ws_down, H, Ish, 128));
+    MV_TRY(tmap(&S.b, ws.a_sh, T, Ish, 16));
+    S.a1 = S.a0;
+    S.out = ws.y_sh;
+    S.ld_out = H;
+    S.K = Ish;
+    S.M = H;
+    S.groups = 1;
+    S.static_rows = T;
+    S.dep_set = sh1;
+    units += int64_t((H + 127) / 128) * ((T + BN - 1) / BN);
+  }
+  {  // routed experts, down
+    mv::GemmSet& S = p.set[ns++];
+    base(S, mv::MODE_KPAIR, mv::EPI_STORE_F32);
+    MV_TRY(tmap(&S.a0, w.w_down, static_cast<uint64_t>(E) * H, I, 128));
+    MV_TRY(tmap(&S.b, ws.a_perm, n, I, 16));
+    S.a1 = S.a0;
+    S.out = ws.y_perm;
+    S.ld_out = H;
+    S.K = I;
+    S.M = H;
+    S.groups = E;
+    S.counts = ws.counts;
+    S.offsets = ws.offsets;
+    S.a_group_stride = H;
+    S.dep_set = rt1;
+    units += int64_t((H + 127) / 128) * (std::min(E, n) + (n + BN - 1) / BN);
+  }
+  p.nsets = ns;
+  cudaError_t e = run_kernel(KIND_GEMM_MOE, st, [&] {
+    return mv::launch_gemm(decode ? mv::GEMM_MOE_DECODE : mv::GEMM_MOE_PREFILL, p, gemm_grid(units), st);
+  });
+  return e == cudaSuccess ? MV_OK : cuda_fail(e, "grouped_moe_gemm launch");
+}
+
+mv_status ffn_forward_impl(const uint16_t* x, int T, const mv_moe_shape& s, const mv_moe_weights& w,
+                           const int32_t* idx, const float* tw, const uint16_t* res, uint16_t* out,
+                           const FfnWs& ws, int* err, int* sched, cudaStream_t st) {
   cudaError_t e = run_kernel(KIND_PERMUTE, st, [&] {
-    return mv::launch_permute(idx, T, E, k, ws.counts, ws.offsets, ws.perm, ws.inv, x, H, ws.x_perm, st);
+    return mv::launch_permute(idx, T, s.E, s.k, ws.counts, ws.offsets, ws.perm, ws.inv, x, s.H, ws.x_perm, st);
   });
   if (e != cudaSuccess) return cuda_fail(e, "expert_permute launch");
-
-  // decode configuration when routed groups average 16 rows or fewer
-  const int BN = (static_cast<int64_t>(n) <= 16LL * E) ? 32 : 128;
-  // gate + up with the SwiGLU epilogue
-  {
-    mv::GemmParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.err = err;
-    p.timeout_ns = timeout_ns();
-    int ns = 0;
-    int64_t units = 0;
-    if (Ish > 0) {
-      mv::GemmSet& S = p.set[ns++];
-      MV_TRY(tmap(&S.a0, w.ws_gate, Ish, H, 128));
-      MV_TRY(tmap(&S.a1, w.ws_up, Ish, H, 128));
-      MV_TRY(tmap(&S.b, x, T, H, 16));
-      S.out = ws.a_sh;
-      S.ld_out = Ish;
-      S.K = H;
-      S.M = Ish;
-      S.groups = 1;
-      S.static_rows = T;
-      units += int64_t((Ish + 127) / 128) * ((T + BN - 1) / BN);
-    }
-    {
-      mv::GemmSet& S = p.set[ns++];
-      MV_TRY(tmap(&S.a0, w.w_gate, static_cast<uint64_t>(E) * I, H, 128));
-      MV_TRY(tmap(&S.a1, w.w_up, static_cast<uint64_t>(E) * I, H, 128));
-      MV_TRY(tmap(&S.b, ws.x_perm, n, H, 16));
-      S.out = ws.a_perm;
-      S.ld_out = I;
-      S.K = H;
-      S.M = I;
-      S.groups = E;
-      S.counts = ws.counts;
-      S.offsets = ws.offsets;
-      S.a_group_stride = I;
-      units += int64_t((I + 127) / 128) * (std::min(E, n) + (n + BN - 1) / BN);
-    }
-    p.nsets = ns;
-    e = run_kernel(KIND_GEMM_SWIGLU, st, [&] { return mv::launch_gemm(mv::EPI_SWIGLU, BN, p, gemm_grid(units), st); });
-    if (e != cudaSuccess) return cuda_fail(e, "grouped_swiglu_gemm launch");
-  }
-  // down projection, fp32 rows
-  {
-    mv::GemmParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.err = err;
-    p.timeout_ns = timeout_ns();
-    int ns = 0;
-    int64_t units = 0;
-    if (Ish > 0) {
-      mv::GemmSet& S = p.set[ns++];
-      MV_TRY(tmap(&S.a0, w.ws_down, H, Ish, 128));
-      MV_TRY(tmap(&S.b, ws.a_sh, T, Ish, 16));
-      S.a1 = S.a0;
-      S.out = ws.y_sh;
-      S.ld_out = H;
-      S.K = Ish;
-      S.M = H;
-      S.groups = 1;
-      S.static_rows = T;
-      units += int64_t((H + 127) / 128) * ((T + BN - 1) / BN);
-    }
-    {
-      mv::GemmSet& S = p.set[ns++];
-      MV_TRY(tmap(&S.a0, w.w_down, static_cast<uint64_t>(E) * H, I, 128));
-      MV_TRY(tmap(&S.b, ws.a_perm, n, I, 16));
-      S.a1 = S.a0;
-      S.out = ws.y_perm;
-      S.ld_out = H;
-      S.K = I;
-      S.M = H;
-      S.groups = E;
-      S.counts = ws.counts;
-      S.offsets = ws.offsets;
-      S.a_group_stride = H;
-      units += int64_t((H + 127) / 128) * (std::min(E, n) + (n + BN - 1) / BN);
-    }
-    p.nsets = ns;
-    e = run_kernel(KIND_GEMM_DOWN, st, [&] { return mv::launch_gemm(mv::EPI_STORE_F32, BN, p, gemm_grid(units), st); });
-    if (e != cudaSuccess) return cuda_fail(e, "grouped_down_gemm launch");
-  }
+  MV_TRY(moe_gemm_impl(x, T, s, w, ws, err, sched, st));
   e = run_kernel(KIND_COMBINE, st, [&] {
-    return mv::launch_combine(ws.y_perm, Ish > 0 ? ws.y_sh : nullptr, ws.inv, tw, res, out, T, H, k, err, st);
+    return mv::launch_combine(ws.y_perm, s.I_shared > 0 ? ws.y_sh : nullptr, ws.inv, tw, res, out, T, s.H, s.k,
+                              err, st);
   });
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   return MV_OK;
 }
 
 mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, int V, uint64_t* parts,
-                       int* err, cudaStream_t st) {
+                       int* err, int* sched, cudaStream_t st) {
   mv::GemmParams p;
   std::memset(&p, 0, sizeof(p));
   p.err = err;
+  p.sched = sched;
   p.timeout_ns = timeout_ns();
   mv::GemmSet& S = p.set[0];
+  S.mode = mv::MODE_MPAIR;
+  S.epi = mv::EPI_ARGMAX;
+  S.m_tile = 256;
+  S.dep_set = -1;
   MV_TRY(tmap(&S.a0, w_lm, V, H, 128));
   MV_TRY(tmap(&S.b, h, T, H, 16));
   S.a1 = S.a0;
@@ -404,8 +424,8 @@ mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, in
   S.groups = 1;
   S.static_rows = T;
   p.nsets = 1;
-  const int64_t units = int64_t((V + 127) / 128) * ((T + 127) / 128);
-  cudaError_t e = run_kernel(KIND_LM_GEMM, st, [&] { return mv::launch_gemm(mv::EPI_ARGMAX, 128, p, gemm_grid(units), st); });
+  const int64_t units = int64_t((V + 255) / 256) * ((T + 127) / 128);
+  cudaError_t e = run_kernel(KIND_LM_GEMM, st, [&] { return mv::launch_gemm(mv::GEMM_LM, p, gemm_grid(units), st); });
   if (e != cudaSuccess) return cuda_fail(e, "lm_head_gemm_argmax launch");
   return MV_OK;
 }
@@ -470,7 +490,8 @@ mv_status moe_router_topk(const uint16_t* x, int32_t T, const mv_moe_shape* shap
   if (T == 0) return MV_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = run_kernel(KIND_ROUTER, st, [&] {
-    return mv::launch_router(x, T, shape->H, shape->E, shape->k, w_router, router_bias, topk_idx, topk_w, st);
+    return mv::launch_router(x, T, shape->H, shape->E, shape->k, w_router, router_bias, topk_idx, topk_w, nullptr,
+                             timeout_ns(), st);
   });
   return e == cudaSuccess ? MV_OK : cuda_fail(e, "router_topk launch");
 }
@@ -495,6 +516,7 @@ mv_status moe_expert_permute(const int32_t* topk_idx, int32_t T, int32_t E, int3
 size_t moe_ffn_workspace_size(int32_t T, const mv_moe_shape* shape) {
   if (!shape || T < 0) return 0;
   Carve c{nullptr};
+  c.take<char>(kSchedBytes);
   carve_ffn(c, T, *shape);
   return kHeader + c.off + 1024;
 }
@@ -516,15 +538,19 @@ mv_status moe_ffn_forward(const uint16_t* x, int32_t T, const mv_moe_shape* shap
   if (ws_bytes < need)
     return fail(MV_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, %zu needed", ws_bytes, need);
   if (T == 0) return MV_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Carve c{static_cast<char*>(ws) + kHeader};
+  int* sched = c.take<int>(mv::kSchedInts);
   FfnWs fw = carve_ffn(c, T, *shape);
-  return ffn_forward_impl(x, T, *shape, *weights, topk_idx, topk_w, residual, out, fw, static_cast<int*>(ws),
-                          reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = cudaMemsetAsync(sched, 0, kSchedBytes, st);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the scheduling state");
+  return ffn_forward_impl(x, T, *shape, *weights, topk_idx, topk_w, residual, out, fw, static_cast<int*>(ws), sched,
+                          st);
 }
 
 size_t lm_head_workspace_size(int32_t T, int32_t V) {
   if (T < 0 || V <= 0) return 0;
-  return kHeader + align_up(static_cast<size_t>(lm_parts(V)) * T * 8, 1024) + 1024;
+  return kHeader + kSchedBytes + align_up(static_cast<size_t>(lm_parts(V)) * T * 8, 1024) + 1024;
 }
 
 mv_status lm_head_argmax(const uint16_t* h, int32_t T, int32_t H, const uint16_t* w_lm, int32_t V, int32_t* argmax,
@@ -541,8 +567,11 @@ mv_status lm_head_argmax(const uint16_t* h, int32_t T, int32_t H, const uint16_t
     return fail(MV_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, %zu needed", ws_bytes, need);
   if (T == 0) return MV_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  uint64_t* parts = reinterpret_cast<uint64_t*>(static_cast<char*>(ws) + kHeader);
-  MV_TRY(lm_gemm_impl(h, T, H, w_lm, V, parts, static_cast<int*>(ws), st));
+  int* sched = reinterpret_cast<int*>(static_cast<char*>(ws) + kHeader);
+  uint64_t* parts = reinterpret_cast<uint64_t*>(static_cast<char*>(ws) + kHeader + kSchedBytes);
+  cudaError_t e0 = cudaMemsetAsync(sched, 0, kSchedBytes, st);
+  if (e0 != cudaSuccess) return cuda_fail(e0, "clearing the scheduling state");
+  MV_TRY(lm_gemm_impl(h, T, H, w_lm, V, parts, static_cast<int*>(ws), sched, st));
   cudaError_t e = run_kernel(KIND_LM_FINALIZE, st, [&] { return mv::launch_lm_finalize(parts, lm_parts(V), T, argmax, st); });
   return e == cudaSuccess ? MV_OK : cuda_fail(e, "lm_argmax_finalize launch");
 }
@@ -572,6 +601,7 @@ size_t verify_step_workspace_size(int32_t B, int32_t K, const mv_moe_shape* shap
   c.take<int32_t>(static_cast<size_t>(T) * shape->k);
   c.take<float>(static_cast<size_t>(T) * shape->k);
   c.take<uint64_t>(static_cast<size_t>(lm_parts(V)) * T);
+  c.take<char>(kSchedBytes * (kMaxLayers + 1));
   carve_ffn(c, T, *shape);
   return kHeader + c.off + 1024;
 }
@@ -581,8 +611,9 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
                       int32_t* accepted, int32_t* next_token, int32_t* emitted, int32_t* argmax, void* ws,
                       size_t ws_bytes, mv_stream_t stream) {
   MV_TRY(check_shape(shape));
-  if (B < 0 || K < 0 || K > 32 || n_layers < 0 || V <= 0)
-    return fail(MV_ERR_INVALID_ARG, "bad sizes B=%d K=%d (K <= 32) n_layers=%d V=%d", B, K, n_layers, V);
+  if (B < 0 || K < 0 || K > 32 || n_layers < 0 || n_layers > kMaxLayers || V <= 0)
+    return fail(MV_ERR_INVALID_ARG, "bad sizes B=%d K=%d (K <= 32) n_layers=%d (<= %d) V=%d", B, K, n_layers,
+                kMaxLayers, V);
   if (V % 8) return fail(MV_ERR_UNSUPPORTED_SHAPE, "V=%d must be a multiple of 8", V);
   const int64_t T = int64_t(B) * (K + 1);
   MV_TRY(check_rows(T, shape));
@@ -609,21 +640,26 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
   int32_t* idx = c.take<int32_t>(static_cast<size_t>(T) * shape->k);
   float* tw = c.take<float>(static_cast<size_t>(T) * shape->k);
   uint64_t* parts = c.take<uint64_t>(static_cast<size_t>(lm_parts(V)) * T);
+  int* sched = c.take<int>(static_cast<size_t>(mv::kSchedInts) * (kMaxLayers + 1));
   FfnWs fw = carve_ffn(c, T, *shape);
+  cudaError_t e0 = cudaMemsetAsync(sched, 0, kSchedBytes * (n_layers + 1), st);
+  if (e0 != cudaSuccess) return cuda_fail(e0, "clearing the scheduling state");
 
   const uint16_t* h = hidden;
   for (int l = 0; l < n_layers; ++l) {
     const mv_moe_weights& w = layers[l];
     cudaError_t e = run_kernel(KIND_ROUTER, st, [&] {
       return mv::launch_router(h, static_cast<int>(T), shape->H, shape->E, shape->k, w.w_router, w.router_bias, idx,
-                               tw, st);
+                               tw, err, timeout_ns(), st);
     });
     if (e != cudaSuccess) return cuda_fail(e, "router_topk launch");
     uint16_t* next = hbuf[l & 1];
-    MV_TRY(ffn_forward_impl(h, static_cast<int>(T), *shape, w, idx, tw, h, next, fw, err, st));
+    MV_TRY(ffn_forward_impl(h, static_cast<int>(T), *shape, w, idx, tw, h, next, fw, err,
+                            sched + static_cast<size_t>(l) * mv::kSchedInts, st));
     h = next;
   }
-  MV_TRY(lm_gemm_impl(h, static_cast<int>(T), shape->H, w_lm, V, parts, err, st));
+  MV_TRY(lm_gemm_impl(h, static_cast<int>(T), shape->H, w_lm, V, parts, err,
+                      sched + static_cast<size_t>(n_layers) * mv::kSchedInts, st));
   cudaError_t e = run_kernel(KIND_ACCEPT, st, [&] {
     return mv::launch_accept_from_keys(parts, lm_parts(V), K > 0 ? drafts : nullptr, B, K, accepted, next_token,
                                        emitted, argmax, st);

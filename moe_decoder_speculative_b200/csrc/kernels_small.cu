@@ -149,29 +149,41 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const uint16_t* __rest
 }
 
 // Router with the whole router weight matrix staged in shared memory
-// (E*H bf16, 160 KB at the model shape) by cp.async 16-byte copies, all issued
-// before any is waited on; each CTA then loops over blocks of R rows.  Same
-// arithmetic and selection as router_topk_kernel.
+// (E*H bf16, 160 KB at the model shape) by bulk asynchronous copies (16 KB
+// each, one mbarrier), so a CTA pulls it with a handful of large requests;
+// each CTA then loops over blocks of R rows.  Same arithmetic and selection as
+// router_topk_kernel.  The wait for the copies is bounded: if it ever ran out
+// the rows get expert id -1 (which the grouping and combine kernels report)
+// and the sticky error bit is set when an error word is given.
 template <int R>
-__global__ void __launch_bounds__(256, 1) router_smem_kernel(const uint16_t* __restrict__ x, int T,
-                                                          int H, int E, int k,
-                                                          const uint16_t* __restrict__ wr,
-                                                          const float* __restrict__ bias,
-                                                          int32_t* __restrict__ idx,
-                                                          float* __restrict__ wout) {
-  extern __shared__ __align__(16) uint8_t sm[];
+__global__ void __launch_bounds__(256, 1) router_smem_kernel(const uint16_t* __restrict__ x, int T, int H, int E,
+                                                             int k, const uint16_t* __restrict__ wr,
+                                                             const float* __restrict__ bias,
+                                                             int32_t* __restrict__ idx, float* __restrict__ wout,
+                                                             int* err, uint64_t timeout_ns) {
+  extern __shared__ __align__(128) uint8_t sm[];
   uint16_t* wsm = reinterpret_cast<uint16_t*>(sm);                            // [E][H]
   uint16_t* xs = wsm + static_cast<size_t>(E) * H;                           // [R][H]
   float* ls = reinterpret_cast<float*>(xs + static_cast<size_t>(R) * H);      // [R][E]
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int ok_s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int hv = H / 8;
-  const int nvec = E * hv;
-  for (int i = tid; i < nvec; i += blockDim.x) {
-    const uint32_t dst = smem_u32(wsm + static_cast<size_t>(i) * 8);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(wr + static_cast<size_t>(i) * 8)
-                 : "memory");
+  const uint32_t total = static_cast<uint32_t>(E) * H * 2;
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    mbar_arrive_expect_tx(&bar, total);
+    constexpr uint32_t kChunk = 16384;
+    for (uint32_t off = 0; off < total; off += kChunk) {
+      const uint32_t sz = min(kChunk, total - off);
+      asm volatile(
+          "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+              smem_u32(sm + off)),
+          "l"(reinterpret_cast<const uint8_t*>(wr) + off), "r"(sz), "r"(smem_u32(&bar))
+          : "memory");
+    }
   }
-  asm volatile("cp.async.commit_group;" ::: "memory");
   const int nblocks = (T + R - 1) / R;
   bool first = true;
   for (int rb = blockIdx.x; rb < nblocks; rb += gridDim.x) {
@@ -184,10 +196,20 @@ __global__ void __launch_bounds__(256, 1) router_smem_kernel(const uint16_t* __r
       reinterpret_cast<uint4*>(xs + static_cast<size_t>(r) * H)[c] = v;
     }
     if (first) {
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      if (tid == 0) {
+        int dummy = 0;
+        ok_s = mbar_wait(&bar, 0, &dummy, err, globaltimer_ns() + timeout_ns) ? 1 : 0;
+      }
       first = false;
     }
     __syncthreads();
+    if (!ok_s) {  // the weights never arrived: report instead of computing on garbage
+      if (warp < nrows && lane < k) {
+        idx[static_cast<size_t>(row0 + warp) * k + lane] = -1;
+        wout[static_cast<size_t>(row0 + warp) * k + lane] = 0.f;
+      }
+      continue;
+    }
     for (int e = warp; e < E; e += 8) {
       float acc[R];
 #pragma unroll
@@ -228,7 +250,8 @@ static void launch_router_r(const uint16_t* x, int T, int H, int E, int k, const
 
 template <int R>
 static cudaError_t launch_router_smem(const uint16_t* x, int T, int H, int E, int k, const uint16_t* wr,
-                                      const float* bias, int32_t* idx, float* w, cudaStream_t s, size_t smem) {
+                                      const float* bias, int32_t* idx, float* w, int* err, uint64_t timeout_ns,
+                                      cudaStream_t s, size_t smem) {
   static thread_local int configured_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -241,7 +264,7 @@ static cudaError_t launch_router_smem(const uint16_t* x, int T, int H, int E, in
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int nblocks = (T + R - 1) / R;
-  router_smem_kernel<R><<<min(nblocks, sms), 256, smem, s>>>(x, T, H, E, k, wr, bias, idx, w);
+  router_smem_kernel<R><<<min(nblocks, sms), 256, smem, s>>>(x, T, H, E, k, wr, bias, idx, w, err, timeout_ns);
   return cudaGetLastError();
 }
 
@@ -249,13 +272,16 @@ static cudaError_t launch_router_smem(const uint16_t* x, int T, int H, int E, in
 // large ones.  The router weights go to shared memory when they fit (E*H*2 up
 // to ~200 KB); otherwise the global-load kernel streams them.
 cudaError_t launch_router(const uint16_t* x, int T, int H, int E, int k, const uint16_t* wr,
-                          const float* bias, int32_t* idx, float* w, cudaStream_t s) {
+                          const float* bias, int32_t* idx, float* w, int* err, uint64_t timeout_ns,
+                          cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  const int R = (T <= 1024) ? 4 : 8;
+  const int R = (T <= 256) ? 2 : (T <= 1024) ? 4 : 8;
   const size_t smem_v2 = static_cast<size_t>(E) * H * 2 + static_cast<size_t>(R) * H * 2 + static_cast<size_t>(R) * E * 4;
-  if (smem_v2 <= 200 * 1024)
-    return R == 4 ? launch_router_smem<4>(x, T, H, E, k, wr, bias, idx, w, s, smem_v2)
-                  : launch_router_smem<8>(x, T, H, E, k, wr, bias, idx, w, s, smem_v2);
+  if (smem_v2 <= 200 * 1024) {
+    if (R == 2) return launch_router_smem<2>(x, T, H, E, k, wr, bias, idx, w, err, timeout_ns, s, smem_v2);
+    if (R == 4) return launch_router_smem<4>(x, T, H, E, k, wr, bias, idx, w, err, timeout_ns, s, smem_v2);
+    return launch_router_smem<8>(x, T, H, E, k, wr, bias, idx, w, err, timeout_ns, s, smem_v2);
+  }
   auto fits = [&](int r) { return static_cast<size_t>(r) * H * 2 + static_cast<size_t>(r) * E * 4 <= 48 * 1024; };
   int r = R;
   while (r > 1 && !fits(r)) r >>= 1;
