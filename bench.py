@@ -175,6 +175,7 @@ def algorithmic_bytes(w, touched, T):
         "router_topk": E * H * 2 + T * H * 2 + T * k * 8,
         "expert_permute": n * 4 * 3 + n * H * 2 * 2,
         "combine_unpermute": n * H * 4 + T * H * 4 + T * H * 2 * 2 + n * 12,
+        "combine_route": n * H * 4 + T * H * 4 + T * H * 2 * 2 + n * 12 + E * H * 2 + T * k * 8,
     }
 
 

@@ -63,14 +63,15 @@ enum Kind {
   KIND_PERMUTE,
   KIND_GEMM_MOE,
   KIND_COMBINE,
+  KIND_COMBINE_ROUTE,
   KIND_LM_GEMM,
   KIND_LM_FINALIZE,
   KIND_ACCEPT,
   KIND_COUNT
 };
-const char* kKindNames[KIND_COUNT] = {"router_topk",       "expert_permute",      "grouped_moe_gemm",
-                                      "combine_unpermute", "lm_head_gemm_argmax", "lm_argmax_finalize",
-                                      "greedy_accept"};
+const char* kKindNames[KIND_COUNT] = {"router_topk",       "expert_permute",     "grouped_moe_gemm",
+                                      "combine_unpermute", "combine_route",      "lm_head_gemm_argmax",
+                                      "lm_argmax_finalize", "greedy_accept"};
 
 struct ProfRec {
   int kind;
@@ -386,20 +387,48 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
   return e == cudaSuccess ? MV_OK : cuda_fail(e, "grouped_moe_gemm launch");
 }
 
+// Grouping, fused GEMM and (unless do_combine is false: the caller fuses the
+// combine into the next layer's routing) the combine of one MoE layer.
 mv_status ffn_forward_impl(const uint16_t* x, int T, const mv_moe_shape& s, const mv_moe_weights& w,
                            const int32_t* idx, const float* tw, const uint16_t* res, uint16_t* out,
-                           const FfnWs& ws, int* err, int* sched, cudaStream_t st) {
+                           const FfnWs& ws, int* err, int* sched, cudaStream_t st, bool do_combine = true) {
   cudaError_t e = run_kernel(KIND_PERMUTE, st, [&] {
     return mv::launch_permute(idx, T, s.E, s.k, ws.counts, ws.offsets, ws.perm, ws.inv, x, s.H, ws.x_perm, st);
   });
   if (e != cudaSuccess) return cuda_fail(e, "expert_permute launch");
   MV_TRY(moe_gemm_impl(x, T, s, w, ws, err, sched, st));
+  if (!do_combine) return MV_OK;
   e = run_kernel(KIND_COMBINE, st, [&] {
     return mv::launch_combine(ws.y_perm, s.I_shared > 0 ? ws.y_sh : nullptr, ws.inv, tw, res, out, T, s.H, s.k,
                               err, st);
   });
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   return MV_OK;
+}
+
+// Routing of T rows: the streaming combine+route kernel in route-only mode for
+// decode-sized batches, the shared-memory-staged router otherwise (both give
+// bit-identical logits and choices).
+mv_status route_impl(const uint16_t* x, int T, const mv_moe_shape& s, const uint16_t* wr, const float* bias,
+                     int32_t* idx, float* tw, int* err, cudaStream_t st) {
+  cudaError_t e = run_kernel(KIND_ROUTER, st, [&] {
+    if (mv::combine_route_supported(T, s.H, s.E)) {
+      mv::CombineRouteArgs a{};
+      a.x = x;
+      a.T = T;
+      a.H = s.H;
+      a.E = s.E;
+      a.k = s.k;
+      a.wr = wr;
+      a.bias = bias;
+      a.idx = idx;
+      a.w = tw;
+      a.err = err;
+      return mv::launch_combine_route(a, st);
+    }
+    return mv::launch_router(x, T, s.H, s.E, s.k, wr, bias, idx, tw, err, timeout_ns(), st);
+  });
+  return e == cudaSuccess ? MV_OK : cuda_fail(e, "router_topk launch");
 }
 
 mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, int V, uint64_t* parts,
@@ -488,12 +517,8 @@ mv_status moe_router_topk(const uint16_t* x, int32_t T, const mv_moe_shape* shap
   MV_TRY(check_ptr(topk_idx, "topk_idx"));
   MV_TRY(check_ptr(topk_w, "topk_w"));
   if (T == 0) return MV_OK;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = run_kernel(KIND_ROUTER, st, [&] {
-    return mv::launch_router(x, T, shape->H, shape->E, shape->k, w_router, router_bias, topk_idx, topk_w, nullptr,
-                             timeout_ns(), st);
-  });
-  return e == cudaSuccess ? MV_OK : cuda_fail(e, "router_topk launch");
+  return route_impl(x, T, *shape, w_router, router_bias, topk_idx, topk_w, nullptr,
+                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 mv_status moe_expert_permute(const int32_t* topk_idx, int32_t T, int32_t E, int32_t k, int32_t* counts,
@@ -598,8 +623,8 @@ size_t verify_step_workspace_size(int32_t B, int32_t K, const mv_moe_shape* shap
   Carve c{nullptr};
   c.take<uint16_t>(static_cast<size_t>(T) * shape->H);
   c.take<uint16_t>(static_cast<size_t>(T) * shape->H);
-  c.take<int32_t>(static_cast<size_t>(T) * shape->k);
-  c.take<float>(static_cast<size_t>(T) * shape->k);
+  c.take<int32_t>(static_cast<size_t>(T) * shape->k * 2);
+  c.take<float>(static_cast<size_t>(T) * shape->k * 2);
   c.take<uint64_t>(static_cast<size_t>(lm_parts(V)) * T);
   c.take<char>(kSchedBytes * (kMaxLayers + 1));
   carve_ffn(c, T, *shape);
@@ -637,25 +662,60 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
   Carve c{static_cast<char*>(ws) + kHeader};
   uint16_t* hbuf[2] = {c.take<uint16_t>(static_cast<size_t>(T) * shape->H),
                        c.take<uint16_t>(static_cast<size_t>(T) * shape->H)};
-  int32_t* idx = c.take<int32_t>(static_cast<size_t>(T) * shape->k);
-  float* tw = c.take<float>(static_cast<size_t>(T) * shape->k);
+  const size_t tk = static_cast<size_t>(T) * shape->k;
+  int32_t* idx_buf = c.take<int32_t>(tk * 2);
+  float* tw_buf = c.take<float>(tk * 2);
   uint64_t* parts = c.take<uint64_t>(static_cast<size_t>(lm_parts(V)) * T);
   int* sched = c.take<int>(static_cast<size_t>(mv::kSchedInts) * (kMaxLayers + 1));
   FfnWs fw = carve_ffn(c, T, *shape);
   cudaError_t e0 = cudaMemsetAsync(sched, 0, kSchedBytes * (n_layers + 1), st);
   if (e0 != cudaSuccess) return cuda_fail(e0, "clearing the scheduling state");
 
+  // Layer l's combine runs fused with layer l+1's routing (combine_route) when
+  // the batch is decode-sized; otherwise as its own kernel before the router.
+  const bool fused = mv::combine_route_supported(static_cast<int>(T), shape->H, shape->E);
   const uint16_t* h = hidden;
+  if (n_layers > 0)
+    MV_TRY(route_impl(h, static_cast<int>(T), *shape, layers[0].w_router, layers[0].router_bias, idx_buf, tw_buf, err,
+                      st));
   for (int l = 0; l < n_layers; ++l) {
     const mv_moe_weights& w = layers[l];
-    cudaError_t e = run_kernel(KIND_ROUTER, st, [&] {
-      return mv::launch_router(h, static_cast<int>(T), shape->H, shape->E, shape->k, w.w_router, w.router_bias, idx,
-                               tw, err, timeout_ns(), st);
-    });
-    if (e != cudaSuccess) return cuda_fail(e, "router_topk launch");
+    int32_t* idx = idx_buf + (l & 1) * tk;
+    float* tw = tw_buf + (l & 1) * tk;
     uint16_t* next = hbuf[l & 1];
+    const bool last = (l + 1 == n_layers);
     MV_TRY(ffn_forward_impl(h, static_cast<int>(T), *shape, w, idx, tw, h, next, fw, err,
-                            sched + static_cast<size_t>(l) * mv::kSchedInts, st));
+                            sched + static_cast<size_t>(l) * mv::kSchedInts, st, last || !fused));
+    if (!last) {
+      int32_t* idx_n = idx_buf + ((l + 1) & 1) * tk;
+      float* tw_n = tw_buf + ((l + 1) & 1) * tk;
+      const mv_moe_weights& wn = layers[l + 1];
+      if (fused) {
+        cudaError_t e = run_kernel(KIND_COMBINE_ROUTE, st, [&] {
+          mv::CombineRouteArgs a{};
+          a.x = h;
+          a.y_perm = fw.y_perm;
+          a.y_sh = shape->I_shared > 0 ? fw.y_sh : nullptr;
+          a.inv = fw.inv;
+          a.w_prev = tw;
+          a.k_prev = shape->k;
+          a.out = next;
+          a.T = static_cast<int>(T);
+          a.H = shape->H;
+          a.E = shape->E;
+          a.k = shape->k;
+          a.wr = wn.w_router;
+          a.bias = wn.router_bias;
+          a.idx = idx_n;
+          a.w = tw_n;
+          a.err = err;
+          return mv::launch_combine_route(a, st);
+        });
+        if (e != cudaSuccess) return cuda_fail(e, "combine_route launch");
+      } else {
+        MV_TRY(route_impl(next, static_cast<int>(T), *shape, wn.w_router, wn.router_bias, idx_n, tw_n, err, st));
+      }
+    }
     h = next;
   }
   MV_TRY(lm_gemm_impl(h, static_cast<int>(T), shape->H, w_lm, V, parts, err,

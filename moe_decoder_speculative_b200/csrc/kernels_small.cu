@@ -12,6 +12,8 @@ namespace mv {
 
 namespace {
 
+constexpr int kPermuteStage = 8192;  // routing entries the grouping kernel stages in shared memory
+
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -295,6 +297,182 @@ cudaError_t launch_router(const uint16_t* x, int T, int H, int E, int k, const u
 }
 
 // ---------------------------------------------------------------------------
+// Combine + route (decode-sized batches).  One CTA owns R token rows:
+//  (1) with expert outputs given: h[r] = bf16(res[r] + sum_j w_j * y_j + y_sh)
+//      for its rows (the combine of the layer that just ran; products and sums
+//      rounded separately, in slot order, shared last), written to `out` and
+//      kept in shared memory; without them, the rows of `x` are loaded as is;
+//  (2) the router of the next layer on those rows: logits h[r] . W_r[e]
+//      (+ bias) in fp32, warp w owning experts w, w+8, ...; the router rows
+//      stream from L2 four experts at a time, all loads of a batch issued
+//      before any is used (NV 16-byte vectors per lane per expert row);
+//  (3) top-k with renormalised softmax weights, one warp per row.
+// ---------------------------------------------------------------------------
+template <int R, int NV>
+__global__ void __launch_bounds__(256) combine_route_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ y_perm, const float* __restrict__ y_sh,
+    const int32_t* __restrict__ inv, const float* __restrict__ w_prev, int k_prev, int n_pos,
+    uint16_t* __restrict__ out, int T, int H, int E, int k, const uint16_t* __restrict__ wr,
+    const float* __restrict__ bias, int32_t* __restrict__ idx, float* __restrict__ wout, int* err) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  uint16_t* hs = reinterpret_cast<uint16_t*>(sm);                         // [R][H]
+  float* ls = reinterpret_cast<float*>(hs + static_cast<size_t>(R) * H);  // [R][E]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int hv = H / 8;
+  const int row0 = blockIdx.x * R;
+  const int nrows = min(R, T - row0);
+
+  // (1) rows of h into shared memory
+  for (int i = tid; i < R * hv; i += blockDim.x) {
+    const int r = i / hv, c = i % hv;
+    uint4 o = make_uint4(0, 0, 0, 0);
+    if (r < nrows) {
+      const size_t row = static_cast<size_t>(row0 + r);
+      if (y_perm) {
+        int pos[8];
+        float wj[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          pos[j] = (j < k_prev) ? inv[row * k_prev + j] : -1;
+          wj[j] = (j < k_prev) ? w_prev[row * k_prev + j] : 0.f;
+        }
+        float4 ya[8], yb[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (pos[j] >= 0 && pos[j] < n_pos) {
+            const float4* yp = reinterpret_cast<const float4*>(y_perm + static_cast<size_t>(pos[j]) * H) + 2 * c;
+            ya[j] = yp[0];
+            yb[j] = yp[1];
+          } else {
+            ya[j] = yb[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+        float4 sa = make_float4(0.f, 0.f, 0.f, 0.f), sb = sa;
+        if (y_sh) {
+          const float4* ys = reinterpret_cast<const float4*>(y_sh + row * H) + 2 * c;
+          sa = ys[0];
+          sb = ys[1];
+        }
+        const uint4 rv = reinterpret_cast<const uint4*>(x + row * H)[c];
+        float m[8];
+#pragma unroll
+        for (int i2 = 0; i2 < 8; ++i2) m[i2] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j < k_prev) {
+            if (pos[j] < 0 || pos[j] >= n_pos) {
+              if (err && c == 0) atomicOr(err, kErrInternal);
+              continue;
+            }
+            const float yv[8] = {ya[j].x, ya[j].y, ya[j].z, ya[j].w, yb[j].x, yb[j].y, yb[j].z, yb[j].w};
+#pragma unroll
+            for (int i2 = 0; i2 < 8; ++i2) m[i2] = __fadd_rn(m[i2], __fmul_rn(wj[j], yv[i2]));
+          }
+        }
+        if (y_sh) {
+          const float yv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+#pragma unroll
+          for (int i2 = 0; i2 < 8; ++i2) m[i2] = __fadd_rn(m[i2], yv[i2]);
+        }
+        float rf[8];
+        bf16x8_to_f32(rv, rf);
+        uint32_t ow[4];
+#pragma unroll
+        for (int i2 = 0; i2 < 4; ++i2)
+          ow[i2] = static_cast<uint32_t>(f32_to_bf16_bits(__fadd_rn(rf[2 * i2], m[2 * i2]))) |
+                   (static_cast<uint32_t>(f32_to_bf16_bits(__fadd_rn(rf[2 * i2 + 1], m[2 * i2 + 1]))) << 16);
+        o = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+        reinterpret_cast<uint4*>(out + row * H)[c] = o;
+      } else {
+        o = reinterpret_cast<const uint4*>(x + row * H)[c];
+      }
+    }
+    reinterpret_cast<uint4*>(hs + static_cast<size_t>(r) * H)[c] = o;
+  }
+  __syncthreads();
+
+  // (2) router logits, four experts per batch of loads
+  constexpr int EB = 4;
+  for (int e0 = warp; e0 < E; e0 += 8 * EB) {
+    uint4 wv[EB][NV];
+#pragma unroll
+    for (int b = 0; b < EB; ++b) {
+      const int e = e0 + 8 * b;
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        const int c = lane + 32 * v;
+        wv[b][v] = (e < E && c < hv) ? __ldg(reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e) * H) + c)
+                                     : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < EB; ++b) {
+      const int e = e0 + 8 * b;
+      float acc[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) acc[r] = 0.f;
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        const int c = lane + 32 * v;
+        if (c < hv) {
+          float wf[8];
+          bf16x8_to_f32(wv[b][v], wf);
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            float xf[8];
+            bf16x8_to_f32(reinterpret_cast<const uint4*>(hs + static_cast<size_t>(r) * H)[c], xf);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[r] = fmaf(xf[j], wf[j], acc[r]);
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        float v = acc[r];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0 && e < E) ls[r * E + e] = bias ? v + bias[e] : v;
+      }
+    }
+  }
+  __syncthreads();
+
+  // (3) top-k
+  if (warp < nrows)
+    topk_select_row(ls + warp * E, E, k, lane, idx + static_cast<size_t>(row0 + warp) * k,
+                    wout + static_cast<size_t>(row0 + warp) * k);
+}
+
+template <int R, int NV>
+static void launch_combine_route_rv(const CombineRouteArgs& a, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(R) * a.H * 2 + static_cast<size_t>(R) * a.E * 4;
+  combine_route_kernel<R, NV><<<(a.T + R - 1) / R, 256, smem, s>>>(
+      a.x, a.y_perm, a.y_sh, a.inv, a.w_prev, a.k_prev, a.T * a.k_prev, a.out, a.T, a.H, a.E, a.k, a.wr, a.bias,
+      a.idx, a.w, a.err);
+}
+
+bool combine_route_supported(int T, int H, int E) {
+  return T <= 4096 && H <= 2048 && E <= 256 && (2 * H * 2 + 2 * E * 4) <= 48 * 1024;
+}
+
+cudaError_t launch_combine_route(const CombineRouteArgs& a, cudaStream_t s) {
+  if (a.T <= 0) return cudaSuccess;
+  if (!combine_route_supported(a.T, a.H, a.E)) return cudaErrorInvalidValue;
+  const int nv = (a.H / 8 + 31) / 32;
+  switch (nv) {
+    case 1: launch_combine_route_rv<2, 1>(a, s); break;
+    case 2: launch_combine_route_rv<2, 2>(a, s); break;
+    case 3: launch_combine_route_rv<2, 3>(a, s); break;
+    case 4: launch_combine_route_rv<2, 4>(a, s); break;
+    case 5: launch_combine_route_rv<2, 5>(a, s); break;
+    case 6: launch_combine_route_rv<2, 6>(a, s); break;
+    case 7: launch_combine_route_rv<2, 7>(a, s); break;
+    default: launch_combine_route_rv<2, 8>(a, s); break;
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Grouping by expert.  One CTA per expert e:
 //   counts[e]  = #entries routed to e, offsets[e] = #entries routed below e,
 //   perm[offsets[e] + p] = the p-th entry (row order) routed to e,
@@ -310,15 +488,23 @@ __global__ void __launch_bounds__(256) permute_kernel(const int32_t* __restrict_
                                                       int32_t* __restrict__ inv,
                                                       const uint16_t* __restrict__ x, int H,
                                                       uint16_t* __restrict__ x_perm) {
+  extern __shared__ int32_t idx_s[];  // the routing staged once (when it fits), else read from global
   const int e = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = T * k;
+  const bool staged = n <= kPermuteStage;
   __shared__ int red_eq[8], red_lt[8], wsum[8];
   __shared__ int base_s, running_s;
+  __shared__ int plist[kPermuteStage / 4];  // this expert's entries (when staged)
+
+  if (staged)
+    for (int i = tid; i < n; i += blockDim.x) idx_s[i] = idx[i];
+  __syncthreads();
+  const int32_t* src = staged ? idx_s : idx;
 
   int c_eq = 0, c_lt = 0;
   for (int i = tid; i < n; i += blockDim.x) {
-    const int v = idx[i];
+    const int v = src[i];
     c_eq += (v == e);
     c_lt += (v >= 0 && v < e);
     if (e == 0 && (v < 0 || v >= E)) inv[i] = -1;  // out-of-range id: routed nowhere
@@ -347,13 +533,14 @@ __global__ void __launch_bounds__(256) permute_kernel(const int32_t* __restrict_
   }
   __syncthreads();
   const int base = base_s;
+  const bool local_list = staged && (n / 4 >= 1);
 
   for (int r0 = 0; r0 < T; r0 += blockDim.x) {
     const int r = r0 + tid;
     int slot = -1;
     if (r < T)
       for (int j = 0; j < k; ++j)
-        if (idx[static_cast<size_t>(r) * k + j] == e) slot = j;
+        if (src[static_cast<size_t>(r) * k + j] == e) slot = j;
     const unsigned bal = __ballot_sync(0xffffffffu, slot >= 0);
     const int before = __popc(bal & ((1u << lane) - 1u));
     if (lane == 0) wsum[warp] = __popc(bal);
@@ -364,10 +551,11 @@ __global__ void __launch_bounds__(256) permute_kernel(const int32_t* __restrict_
       tot += wsum[w];
     }
     if (slot >= 0) {
-      const int pos = base + running_s + wpre + before;
+      const int p = running_s + wpre + before;
       const int ent = r * k + slot;
-      perm[pos] = ent;
-      inv[ent] = pos;
+      perm[base + p] = ent;
+      inv[ent] = base + p;
+      if (local_list && p < kPermuteStage / 4) plist[p] = ent;
     }
     __syncthreads();
     if (tid == 0) running_s += tot;
@@ -378,17 +566,18 @@ __global__ void __launch_bounds__(256) permute_kernel(const int32_t* __restrict_
   const int cnt = running_s;
   const int hv = H / 8;
   for (int p = warp; p < cnt; p += 8) {
-    const int ent = perm[base + p];
-    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(ent / k) * H);
+    const int ent = (local_list && p < kPermuteStage / 4) ? plist[p] : perm[base + p];
+    const uint4* srcr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(ent / k) * H);
     uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(base + p) * H);
-    for (int c = lane; c < hv; c += 32) dst[c] = src[c];
+    for (int c = lane; c < hv; c += 32) dst[c] = srcr[c];
   }
 }
 
 cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
                            int32_t* offsets, int32_t* perm, int32_t* inv, const uint16_t* x,
                            int H, uint16_t* x_perm, cudaStream_t s) {
-  permute_kernel<<<E, 256, 0, s>>>(idx, T, E, k, counts, offsets, perm, inv, x, H, x_perm);
+  const size_t smem = (static_cast<size_t>(T) * k <= kPermuteStage) ? static_cast<size_t>(T) * k * 4 : 0;
+  permute_kernel<<<E, 256, smem, s>>>(idx, T, E, k, counts, offsets, perm, inv, x, H, x_perm);
   return cudaGetLastError();
 }
 

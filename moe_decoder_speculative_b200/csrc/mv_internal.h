@@ -56,6 +56,23 @@ struct GemmParams {
 cudaError_t launch_gemm(int config, const GemmParams& p, int grid, cudaStream_t stream);
 
 // Small CUDA-core kernels (kernels_small.cu).
+struct CombineRouteArgs {
+  const uint16_t* x;        // residual rows (combine) or the rows to route (route only)
+  const float* y_perm;      // expert outputs by grouped position, or nullptr: route only
+  const float* y_sh;        // shared-expert outputs or nullptr
+  const int32_t* inv;       // position of entry r*k_prev+j in y_perm
+  const float* w_prev;      // routing weights of the layer being combined
+  int k_prev;
+  uint16_t* out;            // combined rows (when y_perm is given)
+  int T, H, E, k;
+  const uint16_t* wr;       // router weights of the layer to route
+  const float* bias;
+  int32_t* idx;
+  float* w;
+  int* err;
+};
+bool combine_route_supported(int T, int H, int E);
+cudaError_t launch_combine_route(const CombineRouteArgs& a, cudaStream_t s);
 cudaError_t launch_router(const uint16_t* x, int T, int H, int E, int k, const uint16_t* wr,
                           const float* bias, int32_t* idx, float* w, int* err, uint64_t timeout_ns,
                           cudaStream_t s);
