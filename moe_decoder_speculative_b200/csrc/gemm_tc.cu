@@ -108,6 +108,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   const int lane = tid & 31;
   const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
 
+  pdl_trigger();
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < p.nsets; ++s) {
+      tma_prefetch_desc(&p.set[s].a0);
+      tma_prefetch_desc(&p.set[s].a1);
+      tma_prefetch_desc(&p.set[s].b);
+    }
+  }
+  pdl_wait();  // the group sizes and the B operands come from the previous kernels
+
   // ---- group table (every CTA builds the same one) -----------------------
   if (tid == 0) {
     int b = 0;
@@ -195,13 +205,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   if (warp == 1) {
     tmem_alloc(&tmem_base_s, tmem_cols);
     tmem_relinquish();
-  }
-  if (warp == 0 && lane == 0) {
-    for (int s = 0; s < p.nsets; ++s) {
-      tma_prefetch_desc(&p.set[s].a0);
-      tma_prefetch_desc(&p.set[s].a1);
-      tma_prefetch_desc(&p.set[s].b);
-    }
   }
   tc_fence_before();
   __syncthreads();
@@ -501,8 +504,7 @@ static cudaError_t launch_gemm_impl(const GemmParams& p, int grid, cudaStream_t 
     if (e != cudaSuccess) return e;
     configured_dev = dev;
   }
-  kern<<<grid, kThreads, SMEM, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), SMEM, stream, p);
 }
 
 // Tile configurations:

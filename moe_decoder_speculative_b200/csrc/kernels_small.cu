@@ -106,6 +106,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const uint16_t* __rest
   extern __shared__ __align__(16) uint8_t sm[];
   uint16_t* xs = reinterpret_cast<uint16_t*>(sm);                        // [R][H]
   float* ls = reinterpret_cast<float*>(sm + static_cast<size_t>(R) * H * 2);  // [R][E]
+  pdl_trigger();
+  pdl_wait();
   const int row0 = blockIdx.x * R;
   const int nrows = min(R, T - row0);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -186,6 +188,8 @@ __global__ void __launch_bounds__(256, 1) router_smem_kernel(const uint16_t* __r
           : "memory");
     }
   }
+  pdl_trigger();
+  pdl_wait();  // the rows to route come from the previous kernel
   const int nblocks = (T + R - 1) / R;
   bool first = true;
   for (int rb = blockIdx.x; rb < nblocks; rb += gridDim.x) {
@@ -247,7 +251,7 @@ template <int R>
 static void launch_router_r(const uint16_t* x, int T, int H, int E, int k, const uint16_t* wr,
                             const float* bias, int32_t* idx, float* w, cudaStream_t s) {
   const size_t smem = static_cast<size_t>(R) * H * 2 + static_cast<size_t>(R) * E * 4;
-  router_topk_kernel<R><<<(T + R - 1) / R, 256, smem, s>>>(x, T, H, E, k, wr, bias, idx, w);
+  launch_pdl(router_topk_kernel<R>, dim3((T + R - 1) / R), dim3(256), smem, s, x, T, H, E, k, wr, bias, idx, w);
 }
 
 template <int R>
@@ -266,8 +270,8 @@ static cudaError_t launch_router_smem(const uint16_t* x, int T, int H, int E, in
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int nblocks = (T + R - 1) / R;
-  router_smem_kernel<R><<<min(nblocks, sms), 256, smem, s>>>(x, T, H, E, k, wr, bias, idx, w, err, timeout_ns);
-  return cudaGetLastError();
+  return launch_pdl(router_smem_kernel<R>, dim3(min(nblocks, sms)), dim3(256), smem, s, x, T, H, E, k, wr, bias, idx, w,
+                    err, timeout_ns);
 }
 
 // Rows per block: 4 for decode-sized batches (more CTAs share the work), 8 for
@@ -321,6 +325,9 @@ __global__ void __launch_bounds__(256) combine_route_kernel(
   const int hv = H / 8;
   const int row0 = blockIdx.x * R;
   const int nrows = min(R, T - row0);
+  pdl_trigger();
+  if (blockIdx.x == 0 && tid == 0) prefetch_l2_bulk(wr, static_cast<uint32_t>(E) * H * 2);  // weights: no dependency
+  pdl_wait();  // expert outputs / rows come from the previous kernel
 
   // (1) rows of h into shared memory
   for (int i = tid; i < R * hv; i += blockDim.x) {
@@ -444,11 +451,10 @@ __global__ void __launch_bounds__(256) combine_route_kernel(
 }
 
 template <int R, int NV>
-static void launch_combine_route_rv(const CombineRouteArgs& a, cudaStream_t s) {
+static cudaError_t launch_combine_route_rv(const CombineRouteArgs& a, cudaStream_t s) {
   const size_t smem = static_cast<size_t>(R) * a.H * 2 + static_cast<size_t>(R) * a.E * 4;
-  combine_route_kernel<R, NV><<<(a.T + R - 1) / R, 256, smem, s>>>(
-      a.x, a.y_perm, a.y_sh, a.inv, a.w_prev, a.k_prev, a.T * a.k_prev, a.out, a.T, a.H, a.E, a.k, a.wr, a.bias,
-      a.idx, a.w, a.err);
+  return launch_pdl(combine_route_kernel<R, NV>, dim3((a.T + R - 1) / R), dim3(256), smem, s, a.x, a.y_perm, a.y_sh, a.inv,
+             a.w_prev, a.k_prev, a.T * a.k_prev, a.out, a.T, a.H, a.E, a.k, a.wr, a.bias, a.idx, a.w, a.err);
 }
 
 bool combine_route_supported(int T, int H, int E) {
@@ -460,16 +466,15 @@ cudaError_t launch_combine_route(const CombineRouteArgs& a, cudaStream_t s) {
   if (!combine_route_supported(a.T, a.H, a.E)) return cudaErrorInvalidValue;
   const int nv = (a.H / 8 + 31) / 32;
   switch (nv) {
-    case 1: launch_combine_route_rv<2, 1>(a, s); break;
-    case 2: launch_combine_route_rv<2, 2>(a, s); break;
-    case 3: launch_combine_route_rv<2, 3>(a, s); break;
-    case 4: launch_combine_route_rv<2, 4>(a, s); break;
-    case 5: launch_combine_route_rv<2, 5>(a, s); break;
-    case 6: launch_combine_route_rv<2, 6>(a, s); break;
-    case 7: launch_combine_route_rv<2, 7>(a, s); break;
-    default: launch_combine_route_rv<2, 8>(a, s); break;
+    case 1: return launch_combine_route_rv<2, 1>(a, s);
+    case 2: return launch_combine_route_rv<2, 2>(a, s);
+    case 3: return launch_combine_route_rv<2, 3>(a, s);
+    case 4: return launch_combine_route_rv<2, 4>(a, s);
+    case 5: return launch_combine_route_rv<2, 5>(a, s);
+    case 6: return launch_combine_route_rv<2, 6>(a, s);
+    case 7: return launch_combine_route_rv<2, 7>(a, s);
+    default: return launch_combine_route_rv<2, 8>(a, s);
   }
-  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
@@ -497,6 +502,8 @@ __global__ void __launch_bounds__(256) permute_kernel(const int32_t* __restrict_
   __shared__ int base_s, running_s;
   __shared__ int plist[kPermuteStage / 4];  // this expert's entries (when staged)
 
+  pdl_trigger();
+  pdl_wait();
   if (staged)
     for (int i = tid; i < n; i += blockDim.x) idx_s[i] = idx[i];
   __syncthreads();
@@ -577,8 +584,7 @@ cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* cou
                            int32_t* offsets, int32_t* perm, int32_t* inv, const uint16_t* x,
                            int H, uint16_t* x_perm, cudaStream_t s) {
   const size_t smem = (static_cast<size_t>(T) * k <= kPermuteStage) ? static_cast<size_t>(T) * k * 4 : 0;
-  permute_kernel<<<E, 256, smem, s>>>(idx, T, E, k, counts, offsets, perm, inv, x, H, x_perm);
-  return cudaGetLastError();
+  return launch_pdl(permute_kernel, dim3(E), dim3(256), smem, s, idx, T, E, k, counts, offsets, perm, inv, x, H, x_perm);
 }
 
 // ---------------------------------------------------------------------------
@@ -592,6 +598,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
                                                       const float* __restrict__ w,
                                                       const uint16_t* res, uint16_t* out, int T,
                                                       int H, int k, int n_pos, int* err) {
+  pdl_trigger();
+  pdl_wait();
   const int hv = H / 8;
   const long long total = static_cast<long long>(T) * hv;
   for (long long t = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; t < total;
@@ -643,8 +651,7 @@ cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t
   const long long total = static_cast<long long>(T) * (H / 8);
   const long long blocks = (total + 255) / 256;
   const int grid = static_cast<int>(blocks < 148LL * 8 ? blocks : 148LL * 8);
-  combine_kernel<<<grid, 256, 0, s>>>(y_perm, y_sh, inv, w, res, out, T, H, k, T * k, err);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, s, y_perm, y_sh, inv, w, res, out, T, H, k, T * k, err);
 }
 
 // ---------------------------------------------------------------------------
@@ -677,6 +684,8 @@ __device__ __forceinline__ uint64_t row_max_key(const uint64_t* row, int nparts,
 __global__ void __launch_bounds__(128) lm_finalize_kernel(const uint64_t* __restrict__ keys, int nparts,
                                                           int T, int32_t* __restrict__ argmax) {
   __shared__ uint64_t red[4];
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   row_max_key(keys + static_cast<size_t>(t) * nparts, nparts, threadIdx.x, 128, red, lane, wid);
@@ -688,8 +697,7 @@ __global__ void __launch_bounds__(128) lm_finalize_kernel(const uint64_t* __rest
 cudaError_t launch_lm_finalize(const uint64_t* keys, int nparts, int T, int32_t* argmax,
                                cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  lm_finalize_kernel<<<T, 128, 0, s>>>(keys, nparts, T, argmax);
-  return cudaGetLastError();
+  return launch_pdl(lm_finalize_kernel, dim3(T), dim3(128), 0, s, keys, nparts, T, argmax);
 }
 
 // ---------------------------------------------------------------------------
@@ -709,6 +717,8 @@ __device__ __forceinline__ void accept_one(const int32_t* g, const int32_t* d, i
 __global__ void accept_kernel(const int32_t* __restrict__ argmax, const int32_t* __restrict__ drafts,
                               int B, int K, int32_t* accepted, int32_t* next_token,
                               int32_t* emitted) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= B) return;
   accept_one(argmax + static_cast<size_t>(b) * (K + 1),
@@ -720,8 +730,8 @@ cudaError_t launch_accept(const int32_t* argmax, const int32_t* drafts, int B, i
                           int32_t* accepted, int32_t* next_token, int32_t* emitted,
                           cudaStream_t s) {
   if (B <= 0) return cudaSuccess;
-  accept_kernel<<<(B + 127) / 128, 128, 0, s>>>(argmax, drafts, B, K, accepted, next_token, emitted);
-  return cudaGetLastError();
+  return launch_pdl(accept_kernel, dim3((B + 127) / 128), dim3(128), 0, s, argmax, drafts, B, K, accepted, next_token,
+                    emitted);
 }
 
 // Fused LM finalisation + acceptance: one CTA per sequence; 4 warps reduce
@@ -731,6 +741,8 @@ __global__ void __launch_bounds__(1024) accept_from_keys_kernel(
     int32_t* accepted, int32_t* next_token, int32_t* emitted, int32_t* argmax_out) {
   __shared__ int32_t g[64];
   __shared__ uint64_t red[32];
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int rows_at_once = blockDim.x / 128;
@@ -760,9 +772,8 @@ cudaError_t launch_accept_from_keys(const uint64_t* keys, int nparts, const int3
                                     int32_t* emitted, int32_t* argmax, cudaStream_t s) {
   if (B <= 0) return cudaSuccess;
   const int rows_at_once = min(8, K + 1);
-  accept_from_keys_kernel<<<B, 128 * rows_at_once, 0, s>>>(keys, nparts, drafts, B, K, accepted,
-                                                           next_token, emitted, argmax);
-  return cudaGetLastError();
+  return launch_pdl(accept_from_keys_kernel, dim3(B), dim3(128 * rows_at_once), 0, s, keys, nparts, drafts, B, K,
+                    accepted, next_token, emitted, argmax);
 }
 
 }  // namespace mv
