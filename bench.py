@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=2, help="workload id (default: concurrency-32 verify)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="run only the first N MoE layers (a smaller case for profiling; not a bench line)")
     return ap.parse_args()
 
 
@@ -79,7 +81,7 @@ def source_digest(files):
 
 
 GEMM_SOURCES = ["moe_decoder_speculative_b200/csrc/gemm_tc.cu", "moe_decoder_speculative_b200/csrc/mv_device.cuh",
-                "moe_decoder_speculative_b200/csrc/mv_internal.h"]
+                "moe_decoder_speculative_b200/csrc/gemm_params.h"]
 
 
 def ncu_traffic(kernel: str):
@@ -271,7 +273,7 @@ def run_ours(args):
 
     w = wl.workload(args.workload)
     assert w.has_verify, "the benchmark times the verify step"
-    inp = wl.make_inputs(w)
+    inp = wl.make_inputs(w, layers=args.layers)
     if rank > 0:   # each replica verifies its own batch of sequences
         inp["hidden"] = wl.normal_bf16(np.random.SeedSequence([w.id, rank]), (w.T, w.H), w.x_std)
     shape = bd.shape_of(w)
@@ -395,7 +397,7 @@ def run_ours(args):
         "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded bf16 weights N(0,0.02^2), hidden N(0,1); drafts copy the "
                                   "verifier argmax w.p. 0.576)",
-        "config": {"workload": w.name, "B": w.B, "K": w.K, "rows": T, "layers": w.L, "H": w.H, "E": w.E,
+        "config": {"workload": w.name, "B": w.B, "K": w.K, "rows": T, "layers": len(layers), "H": w.H, "E": w.E,
                    "top_k": w.k, "I": w.I, "I_shared": w.I_sh, "V": w.V,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "weights (5.8 GB) far larger than L2: no flush needed"},

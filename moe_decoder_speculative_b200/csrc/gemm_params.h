@@ -1,0 +1,54 @@
+// Parameters of the grouped tensor-core GEMM engine (gemm_tc.cu).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+
+namespace mv {
+
+enum { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_ARGMAX = 2 };
+enum { MODE_SINGLE = 0, MODE_GATEUP = 1, MODE_KPAIR = 2, MODE_MPAIR = 3 };
+enum { GEMM_MOE_DECODE = 0, GEMM_MOE_PREFILL = 1, GEMM_LM = 2 };
+
+// Sticky device error bits, OR-ed into the workspace's error word.
+constexpr int kErrTimeout = 1;
+constexpr int kErrInternal = 2;
+
+// Ints of scheduling state one grouped-GEMM launch uses (claim counter plus one
+// completion counter per group); zeroed before the launch.
+constexpr int kSchedInts = 1024;
+
+// One operand set of the grouped GEMM: `groups` groups that share tensor maps.
+// Group gi multiplies A rows [gi*a_group_stride, +M) by the B rows
+// [offsets[gi], +counts[gi]) and writes output rows at the same B row index
+// (EPI_SWIGLU: bf16 [rows][ld_out]; EPI_STORE_F32: fp32 [rows][ld_out];
+// EPI_ARGMAX: uint64 keys [row][ld_out], one per (M tile, lane quarter)).
+struct GemmSet {
+  CUtensorMap a0;          // A operand
+  CUtensorMap a1;          // second A operand (up weights), MODE_GATEUP only
+  CUtensorMap b;           // B operand, box of 16 rows x 64 columns
+  void* out;
+  const int32_t* counts;   // device [groups] or nullptr (static_rows)
+  const int32_t* offsets;  // device [groups] or nullptr (0)
+  int32_t ld_out;
+  int32_t K;               // reduction length, multiple of 64
+  int32_t M;               // valid A rows per group
+  int32_t groups;
+  int32_t static_rows;
+  int32_t a_group_stride;
+  int32_t mode;            // MODE_*
+  int32_t epi;             // EPI_*
+  int32_t m_tile;          // A rows per unit: 128, or 256 for MODE_MPAIR
+  int32_t dep_set;         // -1, or the set whose same-index group must finish first
+  int32_t signal;          // 1: count finished epilogue warps per group (a later set depends on it)
+};
+
+struct GemmParams {
+  GemmSet set[4];
+  int32_t nsets;
+  int* err;
+  int* sched;              // kSchedInts ints, zero at launch
+  uint64_t timeout_ns;
+};
+
+}  // namespace mv
