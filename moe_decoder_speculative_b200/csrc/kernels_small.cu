@@ -313,7 +313,7 @@ cudaError_t launch_router(const uint16_t* x, int T, int H, int E, int k, const u
 //  (3) top-k with renormalised softmax weights, one warp per row.
 // ---------------------------------------------------------------------------
 template <int R, int NV>
-__global__ void __launch_bounds__(256) combine_route_kernel(
+__global__ void __launch_bounds__(512) combine_route_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ y_perm, const float* __restrict__ y_sh,
     const int32_t* __restrict__ inv, const float* __restrict__ w_prev, int k_prev, int n_pos,
     uint16_t* __restrict__ out, int T, int H, int E, int k, const uint16_t* __restrict__ wr,
@@ -398,13 +398,15 @@ __global__ void __launch_bounds__(256) combine_route_kernel(
   }
   __syncthreads();
 
-  // (2) router logits, four experts per batch of loads
+  // (2) router logits: warp w owns experts w, w+16, w+32, w+48 (one batch of
+  //     loads for E <= 64); each x vector is converted once and reused.
   constexpr int EB = 4;
-  for (int e0 = warp; e0 < E; e0 += 8 * EB) {
+  const int nwarps = blockDim.x >> 5;
+  for (int e0 = warp; e0 < E; e0 += nwarps * EB) {
     uint4 wv[EB][NV];
 #pragma unroll
     for (int b = 0; b < EB; ++b) {
-      const int e = e0 + 8 * b;
+      const int e = e0 + nwarps * b;
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
         const int c = lane + 32 * v;
@@ -412,30 +414,35 @@ __global__ void __launch_bounds__(256) combine_route_kernel(
                                      : make_uint4(0, 0, 0, 0);
       }
     }
+    float acc[EB][R];
 #pragma unroll
-    for (int b = 0; b < EB; ++b) {
-      const int e = e0 + 8 * b;
-      float acc[R];
+    for (int b = 0; b < EB; ++b)
 #pragma unroll
-      for (int r = 0; r < R; ++r) acc[r] = 0.f;
+      for (int r = 0; r < R; ++r) acc[b][r] = 0.f;
 #pragma unroll
-      for (int v = 0; v < NV; ++v) {
-        const int c = lane + 32 * v;
-        if (c < hv) {
+    for (int v = 0; v < NV; ++v) {
+      const int c = lane + 32 * v;
+      if (c < hv) {
+        float xf[R][8];
+#pragma unroll
+        for (int r = 0; r < R; ++r) bf16x8_to_f32(reinterpret_cast<const uint4*>(hs + static_cast<size_t>(r) * H)[c], xf[r]);
+#pragma unroll
+        for (int b = 0; b < EB; ++b) {
           float wf[8];
           bf16x8_to_f32(wv[b][v], wf);
 #pragma unroll
-          for (int r = 0; r < R; ++r) {
-            float xf[8];
-            bf16x8_to_f32(reinterpret_cast<const uint4*>(hs + static_cast<size_t>(r) * H)[c], xf);
+          for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[r] = fmaf(xf[j], wf[j], acc[r]);
-          }
+            for (int j = 0; j < 8; ++j) acc[b][r] = fmaf(xf[r][j], wf[j], acc[b][r]);
         }
       }
+    }
+#pragma unroll
+    for (int b = 0; b < EB; ++b) {
+      const int e = e0 + nwarps * b;
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        float v = acc[r];
+        float v = acc[b][r];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         if (lane == 0 && e < E) ls[r * E + e] = bias ? v + bias[e] : v;
@@ -453,28 +460,36 @@ __global__ void __launch_bounds__(256) combine_route_kernel(
 template <int R, int NV>
 static cudaError_t launch_combine_route_rv(const CombineRouteArgs& a, cudaStream_t s) {
   const size_t smem = static_cast<size_t>(R) * a.H * 2 + static_cast<size_t>(R) * a.E * 4;
-  return launch_pdl(combine_route_kernel<R, NV>, dim3((a.T + R - 1) / R), dim3(256), smem, s, a.x, a.y_perm, a.y_sh, a.inv,
+  return launch_pdl(combine_route_kernel<R, NV>, dim3((a.T + R - 1) / R), dim3(512), smem, s, a.x, a.y_perm, a.y_sh, a.inv,
              a.w_prev, a.k_prev, a.T * a.k_prev, a.out, a.T, a.H, a.E, a.k, a.wr, a.bias, a.idx, a.w, a.err);
 }
 
+// Larger batches route with the shared-memory-staged router instead (each of
+// its persistent CTAs reads the router weights once).
 bool combine_route_supported(int T, int H, int E) {
-  return T <= 4096 && H <= 2048 && E <= 256 && (2 * H * 2 + 2 * E * 4) <= 48 * 1024;
+  return T <= 1024 && H <= 2048 && E <= 256 && (2 * H * 2 + 2 * E * 4) <= 48 * 1024;
 }
 
 cudaError_t launch_combine_route(const CombineRouteArgs& a, cudaStream_t s) {
   if (a.T <= 0) return cudaSuccess;
   if (!combine_route_supported(a.T, a.H, a.E)) return cudaErrorInvalidValue;
   const int nv = (a.H / 8 + 31) / 32;
-  switch (nv) {
-    case 1: return launch_combine_route_rv<2, 1>(a, s);
-    case 2: return launch_combine_route_rv<2, 2>(a, s);
-    case 3: return launch_combine_route_rv<2, 3>(a, s);
-    case 4: return launch_combine_route_rv<2, 4>(a, s);
-    case 5: return launch_combine_route_rv<2, 5>(a, s);
-    case 6: return launch_combine_route_rv<2, 6>(a, s);
-    case 7: return launch_combine_route_rv<2, 7>(a, s);
-    default: return launch_combine_route_rv<2, 8>(a, s);
+  // one row per CTA while that keeps the router-row traffic from L2 modest
+  const int R = a.T <= 512 ? 1 : 2;
+#define MV_CR(RR)                                              \
+  switch (nv) {                                                \
+    case 1: return launch_combine_route_rv<RR, 1>(a, s);       \
+    case 2: return launch_combine_route_rv<RR, 2>(a, s);       \
+    case 3: return launch_combine_route_rv<RR, 3>(a, s);       \
+    case 4: return launch_combine_route_rv<RR, 4>(a, s);       \
+    case 5: return launch_combine_route_rv<RR, 5>(a, s);       \
+    case 6: return launch_combine_route_rv<RR, 6>(a, s);       \
+    case 7: return launch_combine_route_rv<RR, 7>(a, s);       \
+    default: return launch_combine_route_rv<RR, 8>(a, s);      \
   }
+  if (R == 1) { MV_CR(1) }
+  MV_CR(2)
+#undef MV_CR
 }
 
 // ---------------------------------------------------------------------------
@@ -576,7 +591,19 @@ __global__ void __launch_bounds__(256) permute_kernel(const int32_t* __restrict_
     const int ent = (local_list && p < kPermuteStage / 4) ? plist[p] : perm[base + p];
     const uint4* srcr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(ent / k) * H);
     uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(base + p) * H);
-    for (int c = lane; c < hv; c += 32) dst[c] = srcr[c];
+    for (int c0 = 0; c0 < hv; c0 += 32 * 8) {  // all loads of up to 8 vectors per lane before the stores
+      uint4 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = c0 + lane + 32 * i;
+        if (c < hv) v[i] = srcr[c];
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = c0 + lane + 32 * i;
+        if (c < hv) dst[c] = v[i];
+      }
+    }
   }
 }
 
@@ -606,21 +633,37 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
        t += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int r = static_cast<int>(t / hv);
     const int c = static_cast<int>(t % hv);
+    int pos[8];
+    float wj[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      pos[j] = (j < k) ? inv[static_cast<size_t>(r) * k + j] : -1;
+      wj[j] = (j < k) ? w[static_cast<size_t>(r) * k + j] : 0.f;
+    }
+    float4 ya[8], yb[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (pos[j] >= 0 && pos[j] < n_pos) {
+        const float4* yp = reinterpret_cast<const float4*>(y_perm + static_cast<size_t>(pos[j]) * H) + 2 * c;
+        ya[j] = yp[0];
+        yb[j] = yp[1];
+      } else {
+        ya[j] = yb[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
     float m[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) m[i] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int p = inv[static_cast<size_t>(r) * k + j];
-      if (p < 0 || p >= n_pos) {  // entry routed to no valid expert
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j >= k) continue;
+      if (pos[j] < 0 || pos[j] >= n_pos) {  // entry routed to no valid expert
         if (err && c == 0) atomicOr(err, kErrInternal);
         continue;
       }
-      const float wj = w[static_cast<size_t>(r) * k + j];
-      const float4* yp = reinterpret_cast<const float4*>(y_perm + static_cast<size_t>(p) * H) + 2 * c;
-      const float4 a = yp[0], b = yp[1];
-      const float yv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      const float yv[8] = {ya[j].x, ya[j].y, ya[j].z, ya[j].w, yb[j].x, yb[j].y, yb[j].z, yb[j].w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(m[i], __fmul_rn(wj, yv[i]));
+      for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(m[i], __fmul_rn(wj[j], yv[i]));
     }
     if (y_sh) {
       const float4* ys = reinterpret_cast<const float4*>(y_sh + static_cast<size_t>(r) * H) + 2 * c;
@@ -665,16 +708,17 @@ __device__ __forceinline__ uint64_t umax64(uint64_t a, uint64_t b) { return a > 
 
 __device__ __forceinline__ uint64_t row_max_key(const uint64_t* row, int nparts, int t0, int nthr,
                                                 uint64_t* red, int lane, int wid) {
-  uint64_t b0 = 0, b1 = 0, b2 = 0, b3 = 0;
-  int p = t0;
-  for (; p + 3 * nthr < nparts; p += 4 * nthr) {
-    b0 = umax64(b0, row[p]);
-    b1 = umax64(b1, row[p + nthr]);
-    b2 = umax64(b2, row[p + 2 * nthr]);
-    b3 = umax64(b3, row[p + 3 * nthr]);
+  uint64_t b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) b[i] = 0;
+  for (int p0 = t0; p0 < nparts; p0 += 8 * nthr) {  // eight independent loads in flight per thread
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int p = p0 + i * nthr;
+      if (p < nparts) b[i] = umax64(b[i], row[p]);
+    }
   }
-  for (; p < nparts; p += nthr) b0 = umax64(b0, row[p]);
-  uint64_t best = umax64(umax64(b0, b1), umax64(b2, b3));
+  uint64_t best = umax64(umax64(umax64(b[0], b[1]), umax64(b[2], b[3])), umax64(umax64(b[4], b[5]), umax64(b[6], b[7])));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) best = umax64(best, __shfl_xor_sync(0xffffffffu, best, o));
   if (lane == 0) red[wid] = best;
@@ -739,25 +783,28 @@ cudaError_t launch_accept(const int32_t* argmax, const int32_t* drafts, int B, i
 __global__ void __launch_bounds__(1024) accept_from_keys_kernel(
     const uint64_t* __restrict__ keys, int nparts, const int32_t* __restrict__ drafts, int B, int K,
     int32_t* accepted, int32_t* next_token, int32_t* emitted, int32_t* argmax_out) {
+  constexpr int kRowThreads = 256;
   __shared__ int32_t g[64];
   __shared__ uint64_t red[32];
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int rows_at_once = blockDim.x / 128;
-  const int sub = threadIdx.x / 128;          // which row of the group this thread serves
-  const int t_in = threadIdx.x % 128;
+  const int rows_at_once = blockDim.x / kRowThreads;
+  const int sub = threadIdx.x / kRowThreads;  // which row of the group this thread serves
+  const int t_in = threadIdx.x % kRowThreads;
+  constexpr int kWarpsPerRow = kRowThreads / 32;
   for (int j0 = 0; j0 <= K; j0 += rows_at_once) {
     const int j = j0 + sub;
     if (j <= K) {
       const int t = b * (K + 1) + j;
-      row_max_key(keys + static_cast<size_t>(t) * nparts, nparts, t_in, 128, red, lane, wid);
+      row_max_key(keys + static_cast<size_t>(t) * nparts, nparts, t_in, kRowThreads, red, lane, wid);
     }
     __syncthreads();
     if (t_in == 0 && j <= K) {
-      const uint64_t* r4 = red + sub * 4;
-      g[j] = static_cast<int32_t>(argmax_key_index(umax64(umax64(r4[0], r4[1]), umax64(r4[2], r4[3]))));
+      uint64_t best = 0;
+      for (int i = 0; i < kWarpsPerRow; ++i) best = umax64(best, red[sub * kWarpsPerRow + i]);
+      g[j] = static_cast<int32_t>(argmax_key_index(best));
       if (argmax_out) argmax_out[b * (K + 1) + j] = g[j];
     }
     __syncthreads();
@@ -771,8 +818,8 @@ cudaError_t launch_accept_from_keys(const uint64_t* keys, int nparts, const int3
                                     int B, int K, int32_t* accepted, int32_t* next_token,
                                     int32_t* emitted, int32_t* argmax, cudaStream_t s) {
   if (B <= 0) return cudaSuccess;
-  const int rows_at_once = min(8, K + 1);
-  return launch_pdl(accept_from_keys_kernel, dim3(B), dim3(128 * rows_at_once), 0, s, keys, nparts, drafts, B, K,
+  const int rows_at_once = min(4, K + 1);
+  return launch_pdl(accept_from_keys_kernel, dim3(B), dim3(256 * rows_at_once), 0, s, keys, nparts, drafts, B, K,
                     accepted, next_token, emitted, argmax);
 }
 
