@@ -291,6 +291,42 @@ int gemm_grid(int64_t units) {
 // ---------------------------------------------------------------------------
 // the path
 // ---------------------------------------------------------------------------
+// The weights the grouped MoE GEMM of a layer streams first, in claim order
+// (shared gate/up, then the routed gate/up of experts 0, 1, ...), up to
+// `budget` bytes: what a kernel running before it can pull into L2 while HBM
+// is otherwise idle.
+mv::L2Prefetch moe_first_wave(const mv_moe_shape& s, const mv_moe_weights& w, uint64_t budget) {
+  mv::L2Prefetch pf{};
+  const uint64_t sh = static_cast<uint64_t>(s.I_shared) * s.H * 2;
+  if (s.I_shared > 0 && budget >= 2 * sh) {
+    pf.ptr[pf.n] = w.ws_gate;
+    pf.bytes[pf.n++] = sh;
+    pf.ptr[pf.n] = w.ws_up;
+    pf.bytes[pf.n++] = sh;
+    budget -= 2 * sh;
+  }
+  const uint64_t per_expert = static_cast<uint64_t>(s.I) * s.H * 2;
+  const uint64_t ne = std::min<uint64_t>(s.E, budget / (2 * per_expert));
+  if (ne > 0) {
+    pf.ptr[pf.n] = w.w_gate;
+    pf.bytes[pf.n++] = ne * per_expert;
+    pf.ptr[pf.n] = w.w_up;
+    pf.bytes[pf.n++] = ne * per_expert;
+  }
+  return pf;
+}
+
+// The first vocabulary rows of the LM head, up to `budget` bytes.
+mv::L2Prefetch lm_first_wave(const uint16_t* w_lm, int V, int H, uint64_t budget) {
+  mv::L2Prefetch pf{};
+  pf.ptr[0] = w_lm;
+  pf.bytes[0] = std::min<uint64_t>(static_cast<uint64_t>(V) * H * 2, budget) & ~uint64_t(15);
+  pf.n = 1;
+  return pf;
+}
+
+constexpr uint64_t kPrefetchBudget = 64ull << 20;  // about half of the 126 MB L2
+
 // The fused grouped GEMM of one MoE layer: gate/up (SwiGLU epilogue) and down
 // projection (fp32 rows) of the shared expert and the routed experts in one
 // persistent launch; a down unit waits for its expert's gate/up units.
@@ -391,7 +427,8 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
 // combine into the next layer's routing) the combine of one MoE layer.
 mv_status ffn_forward_impl(const uint16_t* x, int T, const mv_moe_shape& s, const mv_moe_weights& w,
                            const int32_t* idx, const float* tw, const uint16_t* res, uint16_t* out,
-                           const FfnWs& ws, int* err, int* sched, cudaStream_t st, bool do_combine = true) {
+                           const FfnWs& ws, int* err, int* sched, cudaStream_t st, bool do_combine = true,
+                           const mv::L2Prefetch& combine_pf = mv::L2Prefetch{}) {
   cudaError_t e = run_kernel(KIND_PERMUTE, st, [&] {
     return mv::launch_permute(idx, T, s.E, s.k, ws.counts, ws.offsets, ws.perm, ws.inv, x, s.H, ws.x_perm, st);
   });
@@ -400,7 +437,7 @@ mv_status ffn_forward_impl(const uint16_t* x, int T, const mv_moe_shape& s, cons
   if (!do_combine) return MV_OK;
   e = run_kernel(KIND_COMBINE, st, [&] {
     return mv::launch_combine(ws.y_perm, s.I_shared > 0 ? ws.y_sh : nullptr, ws.inv, tw, res, out, T, s.H, s.k,
-                              err, st);
+                              err, combine_pf, st);
   });
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   return MV_OK;
@@ -410,7 +447,8 @@ mv_status ffn_forward_impl(const uint16_t* x, int T, const mv_moe_shape& s, cons
 // decode-sized batches, the shared-memory-staged router otherwise (both give
 // bit-identical logits and choices).
 mv_status route_impl(const uint16_t* x, int T, const mv_moe_shape& s, const uint16_t* wr, const float* bias,
-                     int32_t* idx, float* tw, int* err, cudaStream_t st) {
+                     int32_t* idx, float* tw, int* err, cudaStream_t st,
+                     const mv::L2Prefetch& pf = mv::L2Prefetch{}) {
   cudaError_t e = run_kernel(KIND_ROUTER, st, [&] {
     if (mv::combine_route_supported(T, s.H, s.E)) {
       mv::CombineRouteArgs a{};
@@ -424,6 +462,7 @@ mv_status route_impl(const uint16_t* x, int T, const mv_moe_shape& s, const uint
       a.idx = idx;
       a.w = tw;
       a.err = err;
+      a.pf = pf;
       return mv::launch_combine_route(a, st);
     }
     return mv::launch_router(x, T, s.H, s.E, s.k, wr, bias, idx, tw, err, timeout_ns(), st);
@@ -677,7 +716,7 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
   const uint16_t* h = hidden;
   if (n_layers > 0)
     MV_TRY(route_impl(h, static_cast<int>(T), *shape, layers[0].w_router, layers[0].router_bias, idx_buf, tw_buf, err,
-                      st));
+                      st, moe_first_wave(*shape, layers[0], kPrefetchBudget)));
   for (int l = 0; l < n_layers; ++l) {
     const mv_moe_weights& w = layers[l];
     int32_t* idx = idx_buf + (l & 1) * tk;
@@ -685,7 +724,8 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
     uint16_t* next = hbuf[l & 1];
     const bool last = (l + 1 == n_layers);
     MV_TRY(ffn_forward_impl(h, static_cast<int>(T), *shape, w, idx, tw, h, next, fw, err,
-                            sched + static_cast<size_t>(l) * mv::kSchedInts, st, last || !fused));
+                            sched + static_cast<size_t>(l) * mv::kSchedInts, st, last || !fused,
+                            last ? lm_first_wave(w_lm, V, shape->H, kPrefetchBudget) : mv::L2Prefetch{}));
     if (!last) {
       int32_t* idx_n = idx_buf + ((l + 1) & 1) * tk;
       float* tw_n = tw_buf + ((l + 1) & 1) * tk;
@@ -709,6 +749,7 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
           a.idx = idx_n;
           a.w = tw_n;
           a.err = err;
+          a.pf = moe_first_wave(*shape, wn, kPrefetchBudget);
           return mv::launch_combine_route(a, st);
         });
         if (e != cudaSuccess) return cuda_fail(e, "combine_route launch");

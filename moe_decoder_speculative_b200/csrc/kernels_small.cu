@@ -23,6 +23,32 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
   }
 }
 
+// This CTA's share of the L2 prefetch ranges: the concatenated ranges are cut
+// into gridDim.x equal slices (16-byte multiples), issued as 64 KB bulk
+// prefetches by one thread.  Fire and forget: nothing waits for them.
+__device__ __forceinline__ void prefetch_share(const L2Prefetch& pf) {
+  if (threadIdx.x != 0 || pf.n <= 0) return;
+  uint64_t total = 0;
+  for (int i = 0; i < pf.n; ++i) total += pf.bytes[i];
+  const uint64_t per = ((total + gridDim.x - 1) / gridDim.x + 15) & ~uint64_t(15);
+  uint64_t lo = per * blockIdx.x, hi = lo + per;
+  if (hi > total) hi = total;
+  uint64_t base = 0;
+  for (int i = 0; i < pf.n && lo < hi; ++i) {
+    const uint64_t r0 = base, r1 = base + pf.bytes[i];
+    base = r1;
+    if (hi <= r0 || lo >= r1) continue;
+    uint64_t a = (lo > r0 ? lo : r0) - r0, b = (hi < r1 ? hi : r1) - r0;
+    const uint8_t* p = static_cast<const uint8_t*>(pf.ptr[i]);
+    while (a < b) {
+      const uint32_t sz = static_cast<uint32_t>(((b - a) < 65536 ? (b - a) : 65536) & ~uint64_t(15));
+      if (sz == 0) break;
+      prefetch_l2_bulk(p + a, sz);
+      a += sz;
+    }
+  }
+}
+
 // (value, index) pair comparison: larger value wins, equal values -> lower index.
 __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
@@ -317,7 +343,8 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ y_perm, const float* __restrict__ y_sh,
     const int32_t* __restrict__ inv, const float* __restrict__ w_prev, int k_prev, int n_pos,
     uint16_t* __restrict__ out, int T, int H, int E, int k, const uint16_t* __restrict__ wr,
-    const float* __restrict__ bias, int32_t* __restrict__ idx, float* __restrict__ wout, int* err) {
+    const float* __restrict__ bias, int32_t* __restrict__ idx, float* __restrict__ wout, int* err,
+    const L2Prefetch pf) {
   extern __shared__ __align__(16) uint8_t sm[];
   uint16_t* hs = reinterpret_cast<uint16_t*>(sm);                         // [R][H]
   float* ls = reinterpret_cast<float*>(hs + static_cast<size_t>(R) * H);  // [R][E]
@@ -327,6 +354,7 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
   const int nrows = min(R, T - row0);
   pdl_trigger();
   if (blockIdx.x == 0 && tid == 0) prefetch_l2_bulk(wr, static_cast<uint32_t>(E) * H * 2);  // weights: no dependency
+  prefetch_share(pf);  // the next GEMM's first weights, while HBM is otherwise idle
   pdl_wait();  // expert outputs / rows come from the previous kernel
 
   // (1) rows of h into shared memory
@@ -461,7 +489,7 @@ template <int R, int NV>
 static cudaError_t launch_combine_route_rv(const CombineRouteArgs& a, cudaStream_t s) {
   const size_t smem = static_cast<size_t>(R) * a.H * 2 + static_cast<size_t>(R) * a.E * 4;
   return launch_pdl(combine_route_kernel<R, NV>, dim3((a.T + R - 1) / R), dim3(512), smem, s, a.x, a.y_perm, a.y_sh, a.inv,
-             a.w_prev, a.k_prev, a.T * a.k_prev, a.out, a.T, a.H, a.E, a.k, a.wr, a.bias, a.idx, a.w, a.err);
+             a.w_prev, a.k_prev, a.T * a.k_prev, a.out, a.T, a.H, a.E, a.k, a.wr, a.bias, a.idx, a.w, a.err, a.pf);
 }
 
 // Larger batches route with the shared-memory-staged router instead (each of
@@ -624,8 +652,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
                                                       const int32_t* __restrict__ inv,
                                                       const float* __restrict__ w,
                                                       const uint16_t* res, uint16_t* out, int T,
-                                                      int H, int k, int n_pos, int* err) {
+                                                      int H, int k, int n_pos, int* err, const L2Prefetch pf) {
   pdl_trigger();
+  prefetch_share(pf);
   pdl_wait();
   const int hv = H / 8;
   const long long total = static_cast<long long>(T) * hv;
@@ -689,12 +718,13 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t* inv,
                            const float* w, const uint16_t* res, uint16_t* out, int T, int H,
-                           int k, int* err, cudaStream_t s) {
+                           int k, int* err, const L2Prefetch& pf, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   const long long total = static_cast<long long>(T) * (H / 8);
   const long long blocks = (total + 255) / 256;
   const int grid = static_cast<int>(blocks < 148LL * 8 ? blocks : 148LL * 8);
-  return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, s, y_perm, y_sh, inv, w, res, out, T, H, k, T * k, err);
+  return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, s, y_perm, y_sh, inv, w, res, out, T, H, k, T * k, err,
+                    pf);
 }
 
 // ---------------------------------------------------------------------------

@@ -31,6 +31,15 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 
 cudaError_t launch_gemm(int config, const GemmParams& p, int grid, cudaStream_t stream);
 
+// Up to four device ranges a kernel prefetches into L2 before it waits for its
+// predecessor (the first weights the next GEMM will stream), split evenly over
+// the kernel's CTAs.
+struct L2Prefetch {
+  const void* ptr[4];
+  uint64_t bytes[4];
+  int n;
+};
+
 // Small CUDA-core kernels (kernels_small.cu).
 struct CombineRouteArgs {
   const uint16_t* x;        // residual rows (combine) or the rows to route (route only)
@@ -46,6 +55,7 @@ struct CombineRouteArgs {
   int32_t* idx;
   float* w;
   int* err;
+  L2Prefetch pf;
 };
 bool combine_route_supported(int T, int H, int E);
 cudaError_t launch_combine_route(const CombineRouteArgs& a, cudaStream_t s);
@@ -57,7 +67,7 @@ cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* cou
                            int H, uint16_t* x_perm, cudaStream_t s);
 cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t* inv,
                            const float* w, const uint16_t* res, uint16_t* out, int T, int H,
-                           int k, int* err, cudaStream_t s);
+                           int k, int* err, const L2Prefetch& pf, cudaStream_t s);
 cudaError_t launch_lm_finalize(const uint64_t* keys, int nparts, int T, int32_t* argmax,
                                cudaStream_t s);
 cudaError_t launch_accept(const int32_t* argmax, const int32_t* drafts, int B, int K,
