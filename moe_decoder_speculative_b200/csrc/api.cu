@@ -325,7 +325,10 @@ mv::L2Prefetch lm_first_wave(const uint16_t* w_lm, int V, int H, uint64_t budget
   return pf;
 }
 
-constexpr uint64_t kPrefetchBudget = 64ull << 20;  // about half of the 126 MB L2
+#ifndef MV_PREFETCH_BUDGET_MB
+#define MV_PREFETCH_BUDGET_MB 32  // measured best of 0 / 32 / 64 / 96 MB on the concurrency-32 step
+#endif
+constexpr uint64_t kPrefetchBudget = static_cast<uint64_t>(MV_PREFETCH_BUDGET_MB) << 20;
 
 // The fused grouped GEMM of one MoE layer: gate/up (SwiGLU epilogue) and down
 // projection (fp32 rows) of the shared expert and the routed experts in one
