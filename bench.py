@@ -251,6 +251,20 @@ def run_reference(args):
 # our arm
 # ---------------------------------------------------------------------------
 
+def reduce_over_ranks(ms, ms_e2e, committed, device):
+    """Replicas report the slowest rank's device time (MAX) and the committed
+    tokens of all ranks (SUM); a single process returns its own numbers."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms, ms_e2e, committed
+    t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    c = torch.tensor([committed], dtype=torch.int64, device=device)
+    dist.all_reduce(c, op=dist.ReduceOp.SUM)
+    return float(t[0]), float(t[1]), int(c.item())
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -361,15 +375,7 @@ def run_ours(args):
         barrier()
     clk = clocks.summary()
 
-    if world > 1:
-        t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, ms_e2e = float(t[0]), float(t[1])
-        c = torch.tensor([committed_per_step], dtype=torch.int64, device=dev)
-        dist.all_reduce(c, op=dist.ReduceOp.SUM)
-        committed_all = int(c.item())
-    else:
-        committed_all = committed_per_step
+    ms, ms_e2e, committed_all = reduce_over_ranks(ms, ms_e2e, committed_per_step, dev)
 
     K = args.steps
     value = committed_all * K / (ms / 1e3)
