@@ -175,6 +175,29 @@ MV_API mv_status greedy_accept(const int32_t* argmax, const int32_t* drafts, int
                         int32_t* accepted, int32_t* next_token, int32_t* emitted,
                         mv_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * lm_head_argmax_noalloc - lm_head_argmax for callers that must not allocate
+ * device memory (the pages have no counterpart; this is an interface
+ * convenience).  Some callers cannot call cudaMalloc: code embedded in a host
+ * framework that owns every device allocation, or latency-critical threads
+ * that may not take the allocator's locks and implicit synchronisation.  They
+ * pass inputs and outputs only; the scratch (partial argmax keys, a work
+ * counter and an error word) is a 4 MiB array built into the library, which
+ * every GPU that loads the library holds until the process exits.
+ *   Same arguments and result as lm_head_argmax, without ws / ws_bytes.
+ *   Limit: ceil(V/256)*4*T*8 + 4352 bytes must fit in 4 MiB (T <= 259 rows
+ *   at V = 129,280); larger sizes return MV_ERR_UNSUPPORTED_SHAPE and launch
+ *   nothing.
+ *   The first call on a device looks up the array's device address (this
+ *   may load the library's device code); make that first call before any
+ *   stream capture.  Every call on a device shares the one array and clears
+ *   its counter and error word on the stream, so calls that overlap on the
+ *   GPU (other streams, other threads) race: serialise them.  If a bounded
+ *   device-side wait ever runs out, every argmax of that call is -1.
+ * ------------------------------------------------------------------------- */
+MV_API mv_status lm_head_argmax_noalloc(const uint16_t* h, int32_t T, int32_t H, const uint16_t* w_lm,
+                                        int32_t V, int32_t* argmax, mv_stream_t stream);
+
 /* Bytes of workspace verify_step needs. */
 MV_API size_t verify_step_workspace_size(int32_t B, int32_t K, const mv_moe_shape* shape, int32_t V);
 

@@ -24,7 +24,7 @@ EXPORTED = ["moe_router_topk", "moe_expert_permute", "moe_ffn_workspace_size", "
             "lm_head_workspace_size", "lm_head_argmax", "greedy_accept", "verify_step_workspace_size",
             "verify_step", "mv_workspace_init", "mv_sync_status", "mv_last_error", "mv_version",
             "mv_launch_count", "mv_profile_enable", "mv_profile_collect", "mv_kernel_name",
-            "mv_set_wait_timeout_ns"]
+            "mv_set_wait_timeout_ns", "lm_head_argmax_noalloc"]
 
 
 class MVError(RuntimeError):
@@ -63,6 +63,7 @@ def lib():
             "moe_ffn_forward": (i32, [P, i32, S, W, P, P, P, P, P, sz, P]),
             "lm_head_workspace_size": (sz, [i32, i32]),
             "lm_head_argmax": (i32, [P, i32, i32, P, i32, P, P, sz, P]),
+            "lm_head_argmax_noalloc": (i32, [P, i32, i32, P, i32, P, P]),
             "greedy_accept": (i32, [P, P, i32, i32, P, P, P, P]),
             "verify_step_workspace_size": (sz, [i32, i32, S, i32]),
             "verify_step": (i32, [P, P, i32, i32, S, W, i32, P, i32, P, P, P, P, P, sz, P]),
@@ -197,6 +198,16 @@ def lm_head_argmax(h, w_lm, argmax=None, ws=None, stream=None):
     if ws is None:
         ws = workspace(lm_head_workspace_size(T, V), h.device)
     _check(lib().lm_head_argmax(_p(h), T, H, _p(w_lm), V, _p(argmax), _p(ws), ws.numel(), _stream(stream)))
+    return argmax
+
+
+def lm_head_argmax_noalloc(h, w_lm, argmax=None, stream=None):
+    """lm_head_argmax without a workspace: the library's built-in scratch is used."""
+    T, H = h.shape
+    V = w_lm.shape[0]
+    if argmax is None:
+        argmax = torch.empty(T, dtype=torch.int32, device=h.device)
+    _check(lib().lm_head_argmax_noalloc(_p(h), T, H, _p(w_lm), V, _p(argmax), _stream(stream)))
     return argmax
 
 

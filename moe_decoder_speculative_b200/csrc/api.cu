@@ -14,6 +14,7 @@
 #include <vector>
 
 #include "moe_verify.h"
+#include "mv_device.cuh"
 #include "mv_internal.h"
 
 namespace {
@@ -796,3 +797,103 @@ mv_status mv_sync_status(void* ws, mv_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// lm_head_argmax_noalloc: the LM-head greedy choice for callers that must not
+// allocate device memory.  Its scratch (error word, work-claim counter and the
+// per-token partial argmax keys) is one file-scope device array instead of a
+// caller workspace.
+// ===========================================================================
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB, held by every GPU that loads the library
+constexpr size_t kNoAllocErrBytes = 256;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  The array's name
+// is only a host-side stand-in, so the address is looked up once per device
+// (with that device current) and cached.
+mv_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(MV_ERR_UNSUPPORTED_SHAPE, "device %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress of the no-alloc scratch");
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return MV_OK;
+}
+
+// Reduces each token's partial keys to its argmax; writes -1 for every token
+// if a bounded device-side wait of the GEMM ran out (the callers of this path
+// have no workspace through which to read the error word).
+__global__ void __launch_bounds__(128) noalloc_finalize_kernel(const uint64_t* __restrict__ keys, int nparts,
+                                                               int T, int32_t* __restrict__ argmax,
+                                                               const int* __restrict__ err) {
+  __shared__ uint64_t red[4];
+  mv::pdl_trigger();
+  mv::pdl_wait();
+  const int t = blockIdx.x;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const uint64_t* row = keys + static_cast<size_t>(t) * nparts;
+  uint64_t best = 0;
+  for (int p = threadIdx.x; p < nparts; p += 128) {
+    const uint64_t v = row[p];
+    best = v > best ? v : best;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t v = __shfl_xor_sync(0xffffffffu, best, o);
+    best = v > best ? v : best;
+  }
+  if (lane == 0) red[wid] = best;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint64_t b = red[0];
+    for (int i = 1; i < 4; ++i) b = red[i] > b ? red[i] : b;
+    argmax[t] = (*err != 0) ? -1 : static_cast<int32_t>(mv::argmax_key_index(b));
+  }
+}
+
+}  // namespace
+
+extern "C" MV_API mv_status lm_head_argmax_noalloc(const uint16_t* h, int32_t T, int32_t H, const uint16_t* w_lm,
+                                                   int32_t V, int32_t* argmax, mv_stream_t stream) {
+  if (T < 0 || H <= 0 || V <= 0) return fail(MV_ERR_INVALID_ARG, "bad sizes T=%d H=%d V=%d", T, H, V);
+  if (H % 64 || V % 8 || H > 16384)
+    return fail(MV_ERR_UNSUPPORTED_SHAPE, "H must be a multiple of 64 and V of 8 (H=%d V=%d)", H, V);
+  MV_TRY(check_ptr(h, "h"));
+  MV_TRY(check_ptr(w_lm, "w_lm"));
+  MV_TRY(check_ptr(argmax, "argmax"));
+  const size_t keys_bytes = static_cast<size_t>(lm_parts(V)) * static_cast<size_t>(T) * 8;
+  const size_t need = kNoAllocErrBytes + kSchedBytes + keys_bytes;
+  if (need > kNoAllocScratchBytes)
+    return fail(MV_ERR_UNSUPPORTED_SHAPE,
+                "T=%d rows x V=%d needs %zu bytes of scratch; the built-in no-alloc scratch holds %zu "
+                "(use lm_head_argmax with a workspace)",
+                T, V, need, kNoAllocScratchBytes);
+  if (T == 0) return MV_OK;
+  void* base = nullptr;
+  MV_TRY(noalloc_scratch(&base));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* err = static_cast<int*>(base);
+  int* sched = reinterpret_cast<int*>(static_cast<char*>(base) + kNoAllocErrBytes);
+  uint64_t* parts = reinterpret_cast<uint64_t*>(static_cast<char*>(base) + kNoAllocErrBytes + kSchedBytes);
+  cudaError_t e = cudaMemsetAsync(base, 0, kNoAllocErrBytes + kSchedBytes, st);  // error word and claim counter
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the no-alloc scratch");
+  MV_TRY(lm_gemm_impl(h, T, H, w_lm, V, parts, err, sched, st));
+  e = run_kernel(KIND_LM_FINALIZE, st, [&] {
+    return mv::launch_pdl(noalloc_finalize_kernel, dim3(T), dim3(128), 0, st, static_cast<const uint64_t*>(parts),
+                          lm_parts(V), static_cast<int>(T), argmax, static_cast<const int*>(err));
+  });
+  return e == cudaSuccess ? MV_OK : cuda_fail(e, "no-alloc argmax finalize launch");
+}
