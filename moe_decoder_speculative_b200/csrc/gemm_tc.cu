@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
       }
       // Drain: every issued copy must have landed before the CTA may exit.
-      const uint64_t drain_deadline = globaltimer_ns() + p.timeout_ns;
+      const uint64_t drain_deadline = globaltimer_ns() + kDrainNs;
       for (int i = 0; i < STAGES; ++i)
         if (fills[i] > 0) {
           int dummy = 0;
@@ -370,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       // Every MMA issued must be complete before TMEM is released.
       tc_commit(&mma_done_bar);
       int dummy = 0;
-      mbar_wait(&mma_done_bar, 0, &dummy, p.err, globaltimer_ns() + p.timeout_ns);
+      mbar_wait(&mma_done_bar, 0, &dummy, p.err, globaltimer_ns() + kDrainNs);
     }
   } else {
     // ======================= epilogue (warps 2..5) =========================

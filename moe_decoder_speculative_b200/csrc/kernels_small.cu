@@ -231,6 +231,8 @@ __global__ void __launch_bounds__(256, 1) router_smem_kernel(const uint16_t* __r
       if (tid == 0) {
         int dummy = 0;
         ok_s = mbar_wait(&bar, 0, &dummy, err, globaltimer_ns() + timeout_ns) ? 1 : 0;
+        // Whatever the outcome, the copies must land before this CTA may exit.
+        if (!ok_s) mbar_wait(&bar, 0, &dummy, nullptr, globaltimer_ns() + kDrainNs);
       }
       first = false;
     }

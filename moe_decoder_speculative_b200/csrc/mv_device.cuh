@@ -45,6 +45,12 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) 
                : "memory");
 }
 
+// Bound on a drain: waiting for copies or MMAs this CTA already issued, which
+// always complete.  Fixed and generous, independent of the configurable wait
+// bound, so that a CTA giving up early never exits with a copy still landing
+// in its shared memory or an MMA still using its TMEM.
+constexpr uint64_t kDrainNs = 2000000000ull;
+
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------
