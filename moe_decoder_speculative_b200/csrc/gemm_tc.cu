@@ -236,10 +236,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           const int gd = set_base[S.dep_set] + ui.gi;
           const int target = 4 * group_units(gd);
           const int* flag = p.sched + 1 + gd;
-          uint32_t spins = 0;
           while (ld_acquire_gpu(flag) < target) {
             __nanosleep(64);
-            if ((++spins & 15u) == 0 && (*static_cast<volatile int*>(&abort_s) || globaltimer_ns() > deadline)) {
+            if (*static_cast<volatile int*>(&abort_s) || globaltimer_ns() > deadline) {
               if (!abort_s) {
                 abort_s = 1;
                 atomicOr(p.err, kErrTimeout);

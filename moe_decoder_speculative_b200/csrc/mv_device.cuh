@@ -91,23 +91,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait for the phase with the given parity to complete.  Gives up
 // when `deadline_ns` (globaltimer) passes or when another role of the CTA has
 // already given up (*abort != 0); on giving up it raises the abort flag and
-// the sticky timeout bit and returns false.
+// the sticky timeout bit and returns false.  try_wait itself suspends for a
+// hardware-chosen window, so both conditions are checked after every failed
+// try.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           volatile int* abort, int* err,
                                           uint64_t deadline_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  uint32_t spins = 0;
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((++spins & 63u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() > deadline_ns) {
-        *abort = 1;
-        if (err) atomicOr(err, kErrTimeout);
-        return false;
-      }
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (globaltimer_ns() > deadline_ns) {
+      *abort = 1;
+      if (err) atomicOr(err, kErrTimeout);
+      return false;
     }
   }
+  return true;
 }
 
 // ---------------------------------------------------------------------------
