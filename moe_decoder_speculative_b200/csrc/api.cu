@@ -255,7 +255,7 @@ struct Carve {
 };
 
 struct FfnWs {
-  int32_t *counts, *offsets, *perm, *inv;
+  int32_t *counts, *offsets, *perm, *inv, *sort;
   uint16_t *x_perm, *a_perm, *a_sh;
   float *y_perm, *y_sh;
 };
@@ -267,6 +267,7 @@ FfnWs carve_ffn(Carve& c, int64_t T, const mv_moe_shape& s) {
   w.offsets = c.take<int32_t>(s.E + 1);
   w.perm = c.take<int32_t>(n);
   w.inv = c.take<int32_t>(n);
+  w.sort = c.take<int32_t>(mv::permute_uses_sort(static_cast<int>(T), s.k) ? mv::sort_scratch_ints(static_cast<int>(T), s.E, s.k) : 1);
   w.x_perm = c.take<uint16_t>(n * s.H);
   w.a_perm = c.take<uint16_t>(n * s.I);
   w.a_sh = c.take<uint16_t>(static_cast<size_t>(T) * s.I_shared);
@@ -434,6 +435,9 @@ mv_status ffn_forward_impl(const uint16_t* x, int T, const mv_moe_shape& s, cons
                            const FfnWs& ws, int* err, int* sched, cudaStream_t st, bool do_combine = true,
                            const mv::L2Prefetch& combine_pf = mv::L2Prefetch{}) {
   cudaError_t e = run_kernel(KIND_PERMUTE, st, [&] {
+    if (mv::permute_uses_sort(T, s.k))
+      return mv::launch_permute_sorted(idx, T, s.E, s.k, ws.counts, ws.offsets, ws.perm, ws.inv, x, s.H, ws.x_perm,
+                                       ws.sort, st);
     return mv::launch_permute(idx, T, s.E, s.k, ws.counts, ws.offsets, ws.perm, ws.inv, x, s.H, ws.x_perm, st);
   });
   if (e != cudaSuccess) return cuda_fail(e, "expert_permute launch");

@@ -645,6 +645,153 @@ cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* cou
 }
 
 // ---------------------------------------------------------------------------
+// Grouping by expert for large batches: a stable counting sort of the T*k
+// routing entries by expert, in three kernels.
+//  rank:  one CTA per chunk of kSortChunkRows rows walks its entries in id
+//         order, 256 at a time: ranks within a warp from __match_any_sync,
+//         across warps and waves from per-expert running counts; writes each
+//         entry's rank within (chunk, expert) and the chunk's per-expert counts.
+//  scan:  per expert, exclusive prefix over chunks; counts, offsets.
+//  place: position = offsets[e] + chunk base + rank; writes perm / inv and
+//         copies the row into the grouped input (one warp per entry, all SMs).
+// The result is the same permutation as permute_kernel's.
+// ---------------------------------------------------------------------------
+constexpr int kSortChunkRows = 256;
+
+__global__ void __launch_bounds__(256) sort_rank_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
+                                                        int32_t* __restrict__ rank, int32_t* __restrict__ chunk_counts) {
+  extern __shared__ int32_t sh[];
+  int32_t* cnt = sh;           // [E] running counts of this chunk
+  int32_t* wcnt = sh + E;      // [8][E] per-warp counts of the current wave
+  pdl_trigger();
+  pdl_wait();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x;
+  const int ent0 = c * kSortChunkRows * k;
+  const int ent1 = min(T, (c + 1) * kSortChunkRows) * k;
+  for (int i = tid; i < E; i += 256) cnt[i] = 0;
+  for (int e0 = ent0; e0 < ent1; e0 += 256) {
+    for (int i = tid; i < 8 * E; i += 256) wcnt[i] = 0;
+    __syncthreads();
+    const int ent = e0 + tid;
+    int e = (ent < ent1) ? idx[ent] : -1;
+    if (e >= E) e = -1;
+    const unsigned mask = __match_any_sync(0xffffffffu, e);
+    const int rw = __popc(mask & ((1u << lane) - 1u));
+    if (e >= 0 && rw == 0) wcnt[warp * E + e] = __popc(mask);
+    __syncthreads();
+    for (int ex = tid; ex < E; ex += 256) {  // prefix over warps, carried across waves
+      int run = cnt[ex];
+      for (int w = 0; w < 8; ++w) {
+        const int t = wcnt[w * E + ex];
+        wcnt[w * E + ex] = run;
+        run += t;
+      }
+      cnt[ex] = run;
+    }
+    __syncthreads();
+    if (e >= 0) rank[ent] = wcnt[warp * E + e] + rw;
+    __syncthreads();
+  }
+  for (int i = tid; i < E; i += 256) chunk_counts[static_cast<size_t>(c) * E + i] = cnt[i];
+}
+
+__global__ void __launch_bounds__(256) sort_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
+                                                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  __shared__ int32_t tot[256];
+  pdl_trigger();
+  pdl_wait();
+  const int e = threadIdx.x;
+  int run = 0;
+  if (e < E) {
+    for (int c = 0; c < nchunks; ++c) {  // in place: chunk counts become chunk bases
+      const int v = chunk_counts[static_cast<size_t>(c) * E + e];
+      chunk_counts[static_cast<size_t>(c) * E + e] = run;
+      run += v;
+    }
+    counts[e] = run;
+  }
+  tot[e] = (e < E) ? run : 0;
+  __syncthreads();
+  if (e == 0) {
+    int acc = 0;
+    for (int i = 0; i < E; ++i) {
+      offsets[i] = acc;
+      acc += tot[i];
+    }
+    offsets[E] = acc;
+  }
+}
+
+__global__ void __launch_bounds__(256) sort_place_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
+                                                         const int32_t* __restrict__ rank,
+                                                         const int32_t* __restrict__ chunk_base,
+                                                         const int32_t* __restrict__ offsets,
+                                                         int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                         const uint16_t* __restrict__ x, int H,
+                                                         uint16_t* __restrict__ x_perm) {
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * (blockDim.x >> 5);
+  const int hv = H / 8;
+  for (int ent = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); ent < T * k; ent += nwarps) {
+    const int e = idx[ent];
+    if (e < 0 || e >= E) {
+      if (lane == 0) inv[ent] = -1;  // out-of-range id: routed nowhere
+      continue;
+    }
+    const int row = ent / k;
+    const int pos = offsets[e] + chunk_base[static_cast<size_t>(row / kSortChunkRows) * E + e] + rank[ent];
+    if (lane == 0) {
+      perm[pos] = ent;
+      inv[ent] = pos;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(row) * H);
+    uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(pos) * H);
+    for (int c0 = 0; c0 < hv; c0 += 32 * 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = c0 + lane + 32 * i;
+        if (c < hv) v[i] = src[c];
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = c0 + lane + 32 * i;
+        if (c < hv) dst[c] = v[i];
+      }
+    }
+  }
+}
+
+size_t sort_scratch_ints(int T, int E, int k) {
+  const int nchunks = (T + kSortChunkRows - 1) / kSortChunkRows;
+  return static_cast<size_t>(T) * k + static_cast<size_t>(nchunks) * E;
+}
+
+bool permute_uses_sort(int T, int k) { return static_cast<int64_t>(T) * k > kPermuteStage; }
+
+cudaError_t launch_permute_sorted(const int32_t* idx, int T, int E, int k, int32_t* counts, int32_t* offsets,
+                                  int32_t* perm, int32_t* inv, const uint16_t* x, int H, uint16_t* x_perm,
+                                  int32_t* scratch, cudaStream_t s) {
+  const int nchunks = (T + kSortChunkRows - 1) / kSortChunkRows;
+  int32_t* rank = scratch;
+  int32_t* chunk = scratch + static_cast<size_t>(T) * k;
+  cudaError_t e = launch_pdl(sort_rank_kernel, dim3(nchunks), dim3(256), static_cast<size_t>(9 * E) * 4, s, idx, T, E,
+                             k, rank, chunk);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(sort_scan_kernel, dim3(1), dim3(256), 0, s, chunk, nchunks, E, counts, offsets);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return launch_pdl(sort_place_kernel, dim3(sms * 4), dim3(256), 0, s, idx, T, E, k,
+                    static_cast<const int32_t*>(rank), static_cast<const int32_t*>(chunk),
+                    static_cast<const int32_t*>(offsets), perm, inv, x, H, x_perm);
+}
+
+// ---------------------------------------------------------------------------
 // Combine: m = sum_j w_j * y_j (slot order) + y_shared, out = bf16(res + m).
 // Each product and sum is rounded separately (no fused multiply-add), in the
 // order written.  One thread owns 8 consecutive hidden features of a row.

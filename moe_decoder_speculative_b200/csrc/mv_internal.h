@@ -65,6 +65,11 @@ cudaError_t launch_router(const uint16_t* x, int T, int H, int E, int k, const u
 cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
                            int32_t* offsets, int32_t* perm, int32_t* inv, const uint16_t* x,
                            int H, uint16_t* x_perm, cudaStream_t s);
+bool permute_uses_sort(int T, int k);
+size_t sort_scratch_ints(int T, int E, int k);
+cudaError_t launch_permute_sorted(const int32_t* idx, int T, int E, int k, int32_t* counts, int32_t* offsets,
+                                  int32_t* perm, int32_t* inv, const uint16_t* x, int H, uint16_t* x_perm,
+                                  int32_t* scratch, cudaStream_t s);
 cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t* inv,
                            const float* w, const uint16_t* res, uint16_t* out, int T, int H,
                            int k, int* err, const L2Prefetch& pf, cudaStream_t s);
