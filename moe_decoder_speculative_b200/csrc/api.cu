@@ -389,9 +389,15 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
     units += int64_t((I + 127) / 128) * (std::min(E, n) + (n + BN - 1) / BN);
     rt1 = ns++;
   }
+  // Down projection: decode tiles pair two k-blocks per stage (MODE_KPAIR);
+  // prefill tiles pair two 128-row halves of W_down over one token k-block
+  // (MODE_MPAIR, 256-row units), so every stage still carries 32 KB of weights.
+  const int down_mode = decode ? mv::MODE_KPAIR : mv::MODE_MPAIR;
+  const int down_tile = decode ? 128 : 256;
   if (Ish > 0) {  // shared expert, down
     mv::GemmSet& S = p.set[ns++];
-    base(S, mv::MODE_KPAIR, mv::EPI_STORE_F32);
+    base(S, down_mode, mv::EPI_STORE_F32);
+    S.m_tile = down_tile;
     MV_TRY(tmap(&S.a0, w.ws_down, H, Ish, 128));
     MV_TRY(tmap(&S.b, ws.a_sh, T, Ish, 16));
     S.a1 = S.a0;
@@ -406,7 +412,8 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
   }
   {  // routed experts, down
     mv::GemmSet& S = p.set[ns++];
-    base(S, mv::MODE_KPAIR, mv::EPI_STORE_F32);
+    base(S, down_mode, mv::EPI_STORE_F32);
+    S.m_tile = down_tile;
     MV_TRY(tmap(&S.a0, w.w_down, static_cast<uint64_t>(E) * H, I, 128));
     MV_TRY(tmap(&S.b, ws.a_perm, n, I, 16));
     S.a1 = S.a0;

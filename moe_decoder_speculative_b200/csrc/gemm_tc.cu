@@ -508,12 +508,12 @@ static cudaError_t launch_gemm_impl(const GemmParams& p, int grid, cudaStream_t 
 
 // Tile configurations:
 //   GEMM_MOE_DECODE   BN = 32, two B k-block slots, 5 stages of 40 KB
-//   GEMM_MOE_PREFILL  BN = 128, two B slots, 3 stages of 64 KB
+//   GEMM_MOE_PREFILL  BN = 128, one B slot, 4 stages of 48 KB (down in MODE_MPAIR)
 //   GEMM_LM           BN = 128, one B slot, 4 stages of 48 KB (MODE_MPAIR)
 cudaError_t launch_gemm(int config, const GemmParams& p, int grid, cudaStream_t stream) {
   switch (config) {
     case GEMM_MOE_DECODE: return launch_gemm_impl<32, 5, 2, false>(p, grid, stream);
-    case GEMM_MOE_PREFILL: return launch_gemm_impl<128, 3, 2, false>(p, grid, stream);
+    case GEMM_MOE_PREFILL: return launch_gemm_impl<128, 4, 1, false>(p, grid, stream);
     case GEMM_LM: return launch_gemm_impl<128, 4, 1, true>(p, grid, stream);
   }
   return cudaErrorInvalidValue;
