@@ -279,6 +279,7 @@ FfnWs carve_ffn(Carve& c, int64_t T, const mv_moe_shape& s) {
 constexpr int kMaxLayers = 64;  // decoder layers one verify_step call may run
 
 int lm_parts(int V) { return (V + 255) / 256 * 4; }  // (256-row vocabulary tile, lane quarter)
+int lm_parts_alloc(int V) { return (V + 127) / 128 * 4; }  // any split into 256- and 128-row tiles
 
 uint64_t timeout_ns() {
   const int64_t t = g_timeout_ns.load();
@@ -485,29 +486,67 @@ mv_status route_impl(const uint16_t* x, int T, const mv_moe_shape& s, const uint
   return e == cudaSuccess ? MV_OK : cuda_fail(e, "router_topk launch");
 }
 
-mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, int V, uint64_t* parts,
-                       int* err, int* sched, cudaStream_t st) {
+// LM head + fused argmax.  Units are 256-row vocabulary tiles (two 128-row
+// halves sharing each token k-block).  With `balance`, whole waves of the
+// persistent grid take 256-row units and the rows left over are cut into
+// 128-row units, so the last wave is half as long; keys then need up to
+// lm_parts_alloc(V) slots per token.  Returns the key slots used per token
+// (the row stride of `parts` is `ld`).
+mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, int V, uint64_t* parts, int ld,
+                       int* err, int* sched, cudaStream_t st, bool balance, int* nparts_used) {
   mv::GemmParams p;
   std::memset(&p, 0, sizeof(p));
   p.err = err;
   p.sched = sched;
   p.timeout_ns = timeout_ns();
-  mv::GemmSet& S = p.set[0];
-  S.mode = mv::MODE_MPAIR;
-  S.epi = mv::EPI_ARGMAX;
-  S.m_tile = 256;
-  S.dep_set = -1;
-  MV_TRY(tmap(&S.a0, w_lm, V, H, 128));
-  MV_TRY(tmap(&S.b, h, T, H, 16));
-  S.a1 = S.a0;
-  S.out = parts;
-  S.ld_out = lm_parts(V);
-  S.K = H;
-  S.M = V;
-  S.groups = 1;
-  S.static_rows = T;
-  p.nsets = 1;
-  const int64_t units = int64_t((V + 255) / 256) * ((T + 127) / 128);
+  const int nt = (T + 127) / 128;
+  const int n256 = (V + 255) / 256;
+  const int sms = num_sms();
+  int V0 = V;  // rows served by 256-row units
+  if (balance && n256 * nt > sms && (n256 * nt) % sms != 0) {
+    const int full_units = ((n256 * nt) / sms) * sms;
+    V0 = std::min(V, (full_units / nt) * 256);
+  }
+  auto set_up = [&](mv::GemmSet& S, const uint16_t* a_base, int rows, int row_base, int part_base, bool pair) {
+    S.mode = pair ? mv::MODE_MPAIR : mv::MODE_SINGLE;
+    S.epi = mv::EPI_ARGMAX;
+    S.m_tile = pair ? 256 : 128;
+    S.dep_set = -1;
+    S.key_row_base = row_base;
+    S.key_part_base = part_base;
+    S.out = parts;
+    S.ld_out = ld;
+    S.K = H;
+    S.M = rows;
+    S.groups = 1;
+    S.static_rows = T;
+    return MV_OK;
+  };
+  int ns = 0;
+  int used = 0;
+  int64_t units = 0;
+  if (V0 > 0) {
+    mv::GemmSet& S = p.set[ns++];
+    MV_TRY(tmap(&S.a0, w_lm, V0, H, 128));
+    MV_TRY(tmap(&S.b, h, T, H, 16));
+    S.a1 = S.a0;
+    set_up(S, w_lm, V0, 0, 0, true);
+    used = (V0 + 255) / 256 * 4;
+    units += int64_t((V0 + 255) / 256) * nt;
+  }
+  if (V0 < V) {
+    mv::GemmSet& S = p.set[ns++];
+    const uint16_t* tail = w_lm + static_cast<size_t>(V0) * H;
+    MV_TRY(tmap(&S.a0, tail, V - V0, H, 128));
+    MV_TRY(tmap(&S.b, h, T, H, 16));
+    S.a1 = S.a0;
+    set_up(S, tail, V - V0, V0, used, false);
+    used += (V - V0 + 127) / 128 * 4;
+    units += int64_t((V - V0 + 127) / 128) * nt;
+  }
+  p.nsets = ns;
+  if (used > ld) return fail(MV_ERR_INTERNAL, "LM key slots %d exceed the row stride %d", used, ld);
+  *nparts_used = used;
   cudaError_t e = run_kernel(KIND_LM_GEMM, st, [&] { return mv::launch_gemm(mv::GEMM_LM, p, gemm_grid(units), st); });
   if (e != cudaSuccess) return cuda_fail(e, "lm_head_gemm_argmax launch");
   return MV_OK;
@@ -629,7 +668,7 @@ mv_status moe_ffn_forward(const uint16_t* x, int32_t T, const mv_moe_shape* shap
 
 size_t lm_head_workspace_size(int32_t T, int32_t V) {
   if (T < 0 || V <= 0) return 0;
-  return kHeader + kSchedBytes + align_up(static_cast<size_t>(lm_parts(V)) * T * 8, 1024) + 1024;
+  return kHeader + kSchedBytes + align_up(static_cast<size_t>(lm_parts_alloc(V)) * T * 8, 1024) + 1024;
 }
 
 mv_status lm_head_argmax(const uint16_t* h, int32_t T, int32_t H, const uint16_t* w_lm, int32_t V, int32_t* argmax,
@@ -650,8 +689,11 @@ mv_status lm_head_argmax(const uint16_t* h, int32_t T, int32_t H, const uint16_t
   uint64_t* parts = reinterpret_cast<uint64_t*>(static_cast<char*>(ws) + kHeader + kSchedBytes);
   cudaError_t e0 = cudaMemsetAsync(sched, 0, kSchedBytes, st);
   if (e0 != cudaSuccess) return cuda_fail(e0, "clearing the scheduling state");
-  MV_TRY(lm_gemm_impl(h, T, H, w_lm, V, parts, static_cast<int*>(ws), sched, st));
-  cudaError_t e = run_kernel(KIND_LM_FINALIZE, st, [&] { return mv::launch_lm_finalize(parts, lm_parts(V), T, argmax, st); });
+  int used = 0;
+  MV_TRY(lm_gemm_impl(h, T, H, w_lm, V, parts, lm_parts_alloc(V), static_cast<int*>(ws), sched, st, true, &used));
+  cudaError_t e = run_kernel(KIND_LM_FINALIZE, st, [&] {
+    return mv::launch_lm_finalize(parts, used, lm_parts_alloc(V), T, argmax, st);
+  });
   return e == cudaSuccess ? MV_OK : cuda_fail(e, "lm_argmax_finalize launch");
 }
 
@@ -679,7 +721,7 @@ size_t verify_step_workspace_size(int32_t B, int32_t K, const mv_moe_shape* shap
   c.take<uint16_t>(static_cast<size_t>(T) * shape->H);
   c.take<int32_t>(static_cast<size_t>(T) * shape->k * 2);
   c.take<float>(static_cast<size_t>(T) * shape->k * 2);
-  c.take<uint64_t>(static_cast<size_t>(lm_parts(V)) * T);
+  c.take<uint64_t>(static_cast<size_t>(lm_parts_alloc(V)) * T);
   c.take<char>(kSchedBytes * (kMaxLayers + 1));
   carve_ffn(c, T, *shape);
   return kHeader + c.off + 1024;
@@ -719,7 +761,7 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
   const size_t tk = static_cast<size_t>(T) * shape->k;
   int32_t* idx_buf = c.take<int32_t>(tk * 2);
   float* tw_buf = c.take<float>(tk * 2);
-  uint64_t* parts = c.take<uint64_t>(static_cast<size_t>(lm_parts(V)) * T);
+  uint64_t* parts = c.take<uint64_t>(static_cast<size_t>(lm_parts_alloc(V)) * T);
   int* sched = c.take<int>(static_cast<size_t>(mv::kSchedInts) * (kMaxLayers + 1));
   FfnWs fw = carve_ffn(c, T, *shape);
   cudaError_t e0 = cudaMemsetAsync(sched, 0, kSchedBytes * (n_layers + 1), st);
@@ -774,11 +816,12 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
     }
     h = next;
   }
-  MV_TRY(lm_gemm_impl(h, static_cast<int>(T), shape->H, w_lm, V, parts, err,
-                      sched + static_cast<size_t>(n_layers) * mv::kSchedInts, st));
+  int used = 0;
+  MV_TRY(lm_gemm_impl(h, static_cast<int>(T), shape->H, w_lm, V, parts, lm_parts_alloc(V), err,
+                      sched + static_cast<size_t>(n_layers) * mv::kSchedInts, st, true, &used));
   cudaError_t e = run_kernel(KIND_ACCEPT, st, [&] {
-    return mv::launch_accept_from_keys(parts, lm_parts(V), K > 0 ? drafts : nullptr, B, K, accepted, next_token,
-                                       emitted, argmax, st);
+    return mv::launch_accept_from_keys(parts, used, lm_parts_alloc(V), K > 0 ? drafts : nullptr, B, K, accepted,
+                                       next_token, emitted, argmax, st);
   });
   return e == cudaSuccess ? MV_OK : cuda_fail(e, "greedy_accept launch");
 }
@@ -901,7 +944,8 @@ extern "C" MV_API mv_status lm_head_argmax_noalloc(const uint16_t* h, int32_t T,
   uint64_t* parts = reinterpret_cast<uint64_t*>(static_cast<char*>(base) + kNoAllocErrBytes + kSchedBytes);
   cudaError_t e = cudaMemsetAsync(base, 0, kNoAllocErrBytes + kSchedBytes, st);  // error word and claim counter
   if (e != cudaSuccess) return cuda_fail(e, "clearing the no-alloc scratch");
-  MV_TRY(lm_gemm_impl(h, T, H, w_lm, V, parts, err, sched, st));
+  int used = 0;
+  MV_TRY(lm_gemm_impl(h, T, H, w_lm, V, parts, lm_parts(V), err, sched, st, false, &used));
   e = run_kernel(KIND_LM_FINALIZE, st, [&] {
     return mv::launch_pdl(noalloc_finalize_kernel, dim3(T), dim3(128), 0, st, static_cast<const uint64_t*>(parts),
                           lm_parts(V), static_cast<int>(T), argmax, static_cast<const int*>(err));

@@ -41,6 +41,8 @@ struct GemmSet {
   int32_t m_tile;          // A rows per unit: 128, or 256 for MODE_MPAIR
   int32_t dep_set;         // -1, or the set whose same-index group must finish first
   int32_t signal;          // 1: count finished epilogue warps per group (a later set depends on it)
+  int32_t key_row_base;    // EPI_ARGMAX: vocabulary index of this set's A row 0
+  int32_t key_part_base;   // EPI_ARGMAX: first key slot of this set within a token's row
 };
 
 struct GemmParams {

@@ -455,12 +455,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
               }
             }
             __syncwarp();
-            const uint64_t key = argmax_key(best, static_cast<uint32_t>(ui.m0 + h * 128 + wq * 32 + bi));
+            const uint64_t key =
+                argmax_key(best, static_cast<uint32_t>(S.key_row_base + ui.m0 + h * 128 + wq * 32 + bi));
             best_key = key > best_key ? key : best_key;
           }
           const int n = c0 + lane;
           if (n < ui.nvalid) {
-            const int part = (ui.m0 / S.m_tile) * 4 + wq;  // (M tile, lane quarter); keys are token-major
+            const int part = S.key_part_base + (ui.m0 / S.m_tile) * 4 + wq;  // (M tile, lane quarter), token-major
             out[static_cast<size_t>(ui.b_row0 + n) * S.ld_out + part] = best_key;
           }
         }

@@ -905,22 +905,22 @@ __device__ __forceinline__ uint64_t row_max_key(const uint64_t* row, int nparts,
 }
 
 __global__ void __launch_bounds__(128) lm_finalize_kernel(const uint64_t* __restrict__ keys, int nparts,
-                                                          int T, int32_t* __restrict__ argmax) {
+                                                          int ld, int T, int32_t* __restrict__ argmax) {
   __shared__ uint64_t red[4];
   pdl_trigger();
   pdl_wait();
   const int t = blockIdx.x;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  row_max_key(keys + static_cast<size_t>(t) * nparts, nparts, threadIdx.x, 128, red, lane, wid);
+  row_max_key(keys + static_cast<size_t>(t) * ld, nparts, threadIdx.x, 128, red, lane, wid);
   __syncthreads();
   if (threadIdx.x == 0)
     argmax[t] = static_cast<int32_t>(argmax_key_index(umax64(umax64(red[0], red[1]), umax64(red[2], red[3]))));
 }
 
-cudaError_t launch_lm_finalize(const uint64_t* keys, int nparts, int T, int32_t* argmax,
+cudaError_t launch_lm_finalize(const uint64_t* keys, int nparts, int ld, int T, int32_t* argmax,
                                cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  return launch_pdl(lm_finalize_kernel, dim3(T), dim3(128), 0, s, keys, nparts, T, argmax);
+  return launch_pdl(lm_finalize_kernel, dim3(T), dim3(128), 0, s, keys, nparts, ld, T, argmax);
 }
 
 // ---------------------------------------------------------------------------
@@ -960,7 +960,7 @@ cudaError_t launch_accept(const int32_t* argmax, const int32_t* drafts, int B, i
 // Fused LM finalisation + acceptance: one CTA per sequence; 4 warps reduce
 // each of its K+1 rows (up to 8 rows at a time), then one thread accepts.
 __global__ void __launch_bounds__(1024) accept_from_keys_kernel(
-    const uint64_t* __restrict__ keys, int nparts, const int32_t* __restrict__ drafts, int B, int K,
+    const uint64_t* __restrict__ keys, int nparts, int ld, const int32_t* __restrict__ drafts, int B, int K,
     int32_t* accepted, int32_t* next_token, int32_t* emitted, int32_t* argmax_out) {
   constexpr int kRowThreads = 256;
   __shared__ int32_t g[64];
@@ -977,7 +977,7 @@ __global__ void __launch_bounds__(1024) accept_from_keys_kernel(
     const int j = j0 + sub;
     if (j <= K) {
       const int t = b * (K + 1) + j;
-      row_max_key(keys + static_cast<size_t>(t) * nparts, nparts, t_in, kRowThreads, red, lane, wid);
+      row_max_key(keys + static_cast<size_t>(t) * ld, nparts, t_in, kRowThreads, red, lane, wid);
     }
     __syncthreads();
     if (t_in == 0 && j <= K) {
@@ -993,13 +993,13 @@ __global__ void __launch_bounds__(1024) accept_from_keys_kernel(
                next_token, emitted);
 }
 
-cudaError_t launch_accept_from_keys(const uint64_t* keys, int nparts, const int32_t* drafts,
+cudaError_t launch_accept_from_keys(const uint64_t* keys, int nparts, int ld, const int32_t* drafts,
                                     int B, int K, int32_t* accepted, int32_t* next_token,
                                     int32_t* emitted, int32_t* argmax, cudaStream_t s) {
   if (B <= 0) return cudaSuccess;
   const int rows_at_once = min(4, K + 1);
-  return launch_pdl(accept_from_keys_kernel, dim3(B), dim3(256 * rows_at_once), 0, s, keys, nparts, drafts, B, K,
-                    accepted, next_token, emitted, argmax);
+  return launch_pdl(accept_from_keys_kernel, dim3(B), dim3(256 * rows_at_once), 0, s, keys, nparts, ld, drafts, B,
+                    K, accepted, next_token, emitted, argmax);
 }
 
 }  // namespace mv

@@ -73,12 +73,12 @@ cudaError_t launch_permute_sorted(const int32_t* idx, int T, int E, int k, int32
 cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t* inv,
                            const float* w, const uint16_t* res, uint16_t* out, int T, int H,
                            int k, int* err, const L2Prefetch& pf, cudaStream_t s);
-cudaError_t launch_lm_finalize(const uint64_t* keys, int nparts, int T, int32_t* argmax,
+cudaError_t launch_lm_finalize(const uint64_t* keys, int nparts, int ld, int T, int32_t* argmax,
                                cudaStream_t s);
 cudaError_t launch_accept(const int32_t* argmax, const int32_t* drafts, int B, int K,
                           int32_t* accepted, int32_t* next_token, int32_t* emitted,
                           cudaStream_t s);
-cudaError_t launch_accept_from_keys(const uint64_t* keys, int nparts, const int32_t* drafts,
+cudaError_t launch_accept_from_keys(const uint64_t* keys, int nparts, int ld, const int32_t* drafts,
                                     int B, int K, int32_t* accepted, int32_t* next_token,
                                     int32_t* emitted, int32_t* argmax, cudaStream_t s);
 
