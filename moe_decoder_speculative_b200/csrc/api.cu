@@ -356,9 +356,10 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
     S.m_tile = 128;
     S.dep_set = -1;
   };
+  const bool tokm = !decode;
   if (Ish > 0) {  // shared expert, gate/up
     mv::GemmSet& S = p.set[ns];
-    base(S, mv::MODE_GATEUP, mv::EPI_SWIGLU);
+    base(S, tokm ? mv::MODE_TGATEUP : mv::MODE_GATEUP, tokm ? mv::EPI_SWIGLU_ROWS : mv::EPI_SWIGLU);
     MV_TRY(tmap(&S.a0, w.ws_gate, Ish, H, 128));
     MV_TRY(tmap(&S.a1, w.ws_up, Ish, H, 128));
     MV_TRY(tmap(&S.b, x, T, H, 16));
@@ -374,7 +375,7 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
   }
   {  // routed experts, gate/up
     mv::GemmSet& S = p.set[ns];
-    base(S, mv::MODE_GATEUP, mv::EPI_SWIGLU);
+    base(S, tokm ? mv::MODE_TGATEUP : mv::MODE_GATEUP, tokm ? mv::EPI_SWIGLU_ROWS : mv::EPI_SWIGLU);
     MV_TRY(tmap(&S.a0, w.w_gate, static_cast<uint64_t>(E) * I, H, 128));
     MV_TRY(tmap(&S.a1, w.w_up, static_cast<uint64_t>(E) * I, H, 128));
     MV_TRY(tmap(&S.b, ws.x_perm, n, H, 16));
@@ -390,14 +391,16 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
     units += int64_t((I + 127) / 128) * (std::min(E, n) + (n + BN - 1) / BN);
     rt1 = ns++;
   }
-  // Down projection: decode tiles pair two k-blocks per stage (MODE_KPAIR);
-  // prefill tiles pair two 128-row halves of W_down over one token k-block
-  // (MODE_MPAIR, 256-row units), so every stage still carries 32 KB of weights.
-  const int down_mode = decode ? mv::MODE_KPAIR : mv::MODE_MPAIR;
+  // Decode tiles put the weights on the MMA's M side; the down projection
+  // pairs two k-blocks per stage (MODE_KPAIR).  Prefill tiles put 128 tokens
+  // on M and 256 weight rows on N (gate|up, or two halves of W_down).  Either
+  // way every stage carries 32 KB of weights.
+  const int down_mode = decode ? mv::MODE_KPAIR : mv::MODE_TPAIR;
+  const int down_epi = decode ? mv::EPI_STORE_F32 : mv::EPI_STORE_ROWS;
   const int down_tile = decode ? 128 : 256;
   if (Ish > 0) {  // shared expert, down
     mv::GemmSet& S = p.set[ns++];
-    base(S, down_mode, mv::EPI_STORE_F32);
+    base(S, down_mode, down_epi);
     S.m_tile = down_tile;
     MV_TRY(tmap(&S.a0, w.ws_down, H, Ish, 128));
     MV_TRY(tmap(&S.b, ws.a_sh, T, Ish, 16));
@@ -413,7 +416,7 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
   }
   {  // routed experts, down
     mv::GemmSet& S = p.set[ns++];
-    base(S, down_mode, mv::EPI_STORE_F32);
+    base(S, down_mode, down_epi);
     S.m_tile = down_tile;
     MV_TRY(tmap(&S.a0, w.w_down, static_cast<uint64_t>(E) * H, I, 128));
     MV_TRY(tmap(&S.b, ws.a_perm, n, I, 16));

@@ -6,8 +6,11 @@
 
 namespace mv {
 
-enum { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_ARGMAX = 2 };
-enum { MODE_SINGLE = 0, MODE_GATEUP = 1, MODE_KPAIR = 2, MODE_MPAIR = 3 };
+enum { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_ARGMAX = 2, EPI_SWIGLU_ROWS = 3, EPI_STORE_ROWS = 4 };
+// Operand modes.  The first four put weights on the MMA's M side (swap-AB);
+// the tokens-on-M modes load the same tiles but multiply 128 token rows by 256
+// weight rows (gate|up tiles, or two halves of W_down) into one accumulator.
+enum { MODE_SINGLE = 0, MODE_GATEUP = 1, MODE_KPAIR = 2, MODE_MPAIR = 3, MODE_TGATEUP = 4, MODE_TPAIR = 5 };
 enum { GEMM_MOE_DECODE = 0, GEMM_MOE_PREFILL = 1, GEMM_LM = 2 };
 
 // Sticky device error bits, OR-ed into the workspace's error word.

@@ -19,7 +19,12 @@
 //             k-block; epilogue EPI_ARGMAX reduces each token column to a
 //             packed (logit, lowest index) key per 32 vocabulary rows -- the
 //             logits never reach memory
-// Every stage therefore moves 32 KB of weights.
+// Every stage therefore moves 32 KB of weights.  For large groups (prefill)
+// the same tiles are multiplied tokens-on-M: 128 token rows x 256 weight rows
+// (MODE_TGATEUP: gate|up side by side; MODE_TPAIR: two halves of W_down) into
+// one 256-column accumulator, which halves the shared-memory operand traffic
+// per MMA; its epilogues (EPI_SWIGLU_ROWS, EPI_STORE_ROWS) write whole row
+// segments with 16-byte stores.
 //
 // Scheduling: persistent CTAs (at most one per SM) claim work units (group,
 // M tile, N tile) from a global atomic counter in list order -- sets in order,
@@ -280,9 +285,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             const bool two = (S.mode != MODE_SINGLE);
             mbar_arrive_expect_tx(&full_bar[stage], (two ? 2u : 1u) * kATileBytes + b_bytes);
             tma_load_2d(st, &S.a0, ks * 64, a_row0, &full_bar[stage], pol_w);
-            if (S.mode == MODE_GATEUP)
+            if (S.mode == MODE_GATEUP || S.mode == MODE_TGATEUP)
               tma_load_2d(st + kATileBytes, &S.a1, ks * 64, a_row0, &full_bar[stage], pol_w);
-            else if (S.mode == MODE_MPAIR)
+            else if (S.mode == MODE_MPAIR || S.mode == MODE_TPAIR)
               tma_load_2d(st + kATileBytes, &S.a0, ks * 64, a_row0 + 128, &full_bar[stage], pol_w);
             for (int c = 0; c < nchunk; ++c)
               tma_load_2d(b0 + c * kBBox * 128, &S.b, ks * 64, ui.b_row0 + c * kBBox, &full_bar[stage], pol_x);
@@ -318,8 +323,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         const int slot = it & 1;
         if (!mbar_wait(&tempty_bar[slot], ((it >> 1) & 1) ^ 1u, &abort_s, p.err, deadline)) break;
         tc_fence_after();
+        const bool tok_m = (S.mode == MODE_TGATEUP || S.mode == MODE_TPAIR);
         const uint32_t n_mma = static_cast<uint32_t>((ui.nvalid + 15) & ~15);
-        const uint32_t idesc = idesc_bf16_f32(128, n_mma);
+        const uint32_t idesc = tok_m ? idesc_bf16_f32(128, 256) : idesc_bf16_f32(128, n_mma);
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(slot * ACC_COLS);
         const int kblocks = S.K / 64;
         const int nstage = (S.mode == MODE_KPAIR) ? (kblocks + 1) / 2 : kblocks;
@@ -333,7 +339,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
           const uint32_t a1 = st + kATileBytes;
           const uint32_t b0 = st + 2 * kATileBytes;
-          if (S.mode == MODE_KPAIR) {
+          if (tok_m) {
+            // A = the token rows (B slot), B = the 256 weight rows of slots 0-1
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              tc_mma_bf16(d0, smem_desc_k128(b0 + kk * 32), smem_desc_k128(st + kk * 32), idesc,
+                          (ks | kk) != 0 ? 1u : 0u);
+          } else if (S.mode == MODE_KPAIR) {
             const uint32_t b1 = b0 + (NB > 1 ? B_TILE_BYTES : 0);
             const bool two = 2 * ks + 1 < kblocks;
 #pragma unroll
@@ -390,7 +402,54 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       const int row = wq * 32 + lane;  // row of the 128-row tile held by this thread
       const uint32_t tl = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + static_cast<uint32_t>(slot * ACC_COLS);
       const int n_mma = (ui.nvalid + 15) & ~15;
-      if (S.epi == EPI_SWIGLU) {
+      if (S.epi == EPI_SWIGLU_ROWS || S.epi == EPI_STORE_ROWS) {
+        // tokens on M: this thread holds token row `row` of the tile, the
+        // columns are 256 weight outputs (gate|up, or two halves of W_down)
+        const bool tvalid = row < ui.nvalid;
+        const size_t orow = static_cast<size_t>(ui.b_row0 + row) * S.ld_out;
+        if (S.epi == EPI_SWIGLU_ROWS) {
+          uint16_t* out = static_cast<uint16_t*>(S.out);
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t g[32], v[32];
+            tmem_ld32(tl + c0, g);
+            tmem_ld32(tl + 128 + c0, v);
+            tmem_ld_wait();
+            if (tvalid && ui.m0 + c0 < S.M) {
+              uint32_t packed[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                float a2[2];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                  const float gf = __uint_as_float(g[2 * j + q]);
+                  const float uf = __uint_as_float(v[2 * j + q]);
+                  a2[q] = (gf / (1.0f + expf(-gf))) * uf;
+                }
+                packed[j] = static_cast<uint32_t>(f32_to_bf16_bits(a2[0])) |
+                            (static_cast<uint32_t>(f32_to_bf16_bits(a2[1])) << 16);
+              }
+              uint4* dst = reinterpret_cast<uint4*>(out + orow + ui.m0 + c0);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+            }
+          }
+        } else {
+          float* out = static_cast<float*>(S.out);
+          for (int c0 = 0; c0 < 256; c0 += 32) {
+            uint32_t d[32];
+            tmem_ld32(tl + c0, d);
+            tmem_ld_wait();
+            if (tvalid && ui.m0 + c0 < S.M) {
+              float4* dst = reinterpret_cast<float4*>(out + orow + ui.m0 + c0);
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                dst[q] = make_float4(__uint_as_float(d[4 * q]), __uint_as_float(d[4 * q + 1]),
+                                     __uint_as_float(d[4 * q + 2]), __uint_as_float(d[4 * q + 3]));
+            }
+          }
+        }
+      } else if (S.epi == EPI_SWIGLU) {
         const int m = ui.m0 + row;
         const bool mvalid = m < S.M;
         uint16_t* out = static_cast<uint16_t*>(S.out);
@@ -509,7 +568,7 @@ static cudaError_t launch_gemm_impl(const GemmParams& p, int grid, cudaStream_t 
 
 // Tile configurations:
 //   GEMM_MOE_DECODE   BN = 32, two B k-block slots, 5 stages of 40 KB
-//   GEMM_MOE_PREFILL  BN = 128, one B slot, 4 stages of 48 KB (down in MODE_MPAIR)
+//   GEMM_MOE_PREFILL  BN = 128, one B slot, 4 stages of 48 KB (tokens-on-M modes)
 //   GEMM_LM           BN = 128, one B slot, 4 stages of 48 KB (MODE_MPAIR)
 cudaError_t launch_gemm(int config, const GemmParams& p, int grid, cudaStream_t stream) {
   switch (config) {
