@@ -356,13 +356,14 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
     S.m_tile = 128;
     S.dep_set = -1;
   };
-  const bool tokm = !decode;
+  const bool tokm = !decode;  // large groups: tokens on the MMA's M side
+  const int bbox = decode ? mv::kDecodeBBox : mv::kPrefillBBox;
   if (Ish > 0) {  // shared expert, gate/up
     mv::GemmSet& S = p.set[ns];
     base(S, tokm ? mv::MODE_TGATEUP : mv::MODE_GATEUP, tokm ? mv::EPI_SWIGLU_ROWS : mv::EPI_SWIGLU);
     MV_TRY(tmap(&S.a0, w.ws_gate, Ish, H, 128));
     MV_TRY(tmap(&S.a1, w.ws_up, Ish, H, 128));
-    MV_TRY(tmap(&S.b, x, T, H, 16));
+    MV_TRY(tmap(&S.b, x, T, H, bbox));
     S.out = ws.a_sh;
     S.ld_out = Ish;
     S.K = H;
@@ -378,7 +379,7 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
     base(S, tokm ? mv::MODE_TGATEUP : mv::MODE_GATEUP, tokm ? mv::EPI_SWIGLU_ROWS : mv::EPI_SWIGLU);
     MV_TRY(tmap(&S.a0, w.w_gate, static_cast<uint64_t>(E) * I, H, 128));
     MV_TRY(tmap(&S.a1, w.w_up, static_cast<uint64_t>(E) * I, H, 128));
-    MV_TRY(tmap(&S.b, ws.x_perm, n, H, 16));
+    MV_TRY(tmap(&S.b, ws.x_perm, n, H, bbox));
     S.out = ws.a_perm;
     S.ld_out = I;
     S.K = H;
@@ -395,15 +396,15 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
   // pairs two k-blocks per stage (MODE_KPAIR).  Prefill tiles put 128 tokens
   // on M and 256 weight rows on N (gate|up, or two halves of W_down).  Either
   // way every stage carries 32 KB of weights.
-  const int down_mode = decode ? mv::MODE_KPAIR : mv::MODE_TPAIR;
-  const int down_epi = decode ? mv::EPI_STORE_F32 : mv::EPI_STORE_ROWS;
+  const int down_mode = decode ? mv::MODE_KPAIR : (tokm ? mv::MODE_TPAIR : mv::MODE_MPAIR);
+  const int down_epi = tokm ? mv::EPI_STORE_ROWS : mv::EPI_STORE_F32;
   const int down_tile = decode ? 128 : 256;
   if (Ish > 0) {  // shared expert, down
     mv::GemmSet& S = p.set[ns++];
     base(S, down_mode, down_epi);
     S.m_tile = down_tile;
     MV_TRY(tmap(&S.a0, w.ws_down, H, Ish, 128));
-    MV_TRY(tmap(&S.b, ws.a_sh, T, Ish, 16));
+    MV_TRY(tmap(&S.b, ws.a_sh, T, Ish, bbox));
     S.a1 = S.a0;
     S.out = ws.y_sh;
     S.ld_out = H;
@@ -419,7 +420,7 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
     base(S, down_mode, down_epi);
     S.m_tile = down_tile;
     MV_TRY(tmap(&S.a0, w.w_down, static_cast<uint64_t>(E) * H, I, 128));
-    MV_TRY(tmap(&S.b, ws.a_perm, n, I, 16));
+    MV_TRY(tmap(&S.b, ws.a_perm, n, I, bbox));
     S.a1 = S.a0;
     S.out = ws.y_perm;
     S.ld_out = H;
@@ -503,6 +504,8 @@ mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, in
   p.sched = sched;
   p.timeout_ns = timeout_ns();
   const int nt = (T + 127) / 128;
+  const bool wide = T >= 128;  // whole 128-row token tiles: one TMA box per stage
+  const int bbox = wide ? mv::kLmWideBBox : mv::kLmBBox;
   const int n256 = (V + 255) / 256;
   const int sms = num_sms();
   int V0 = V;  // rows served by 256-row units
@@ -531,7 +534,7 @@ mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, in
   if (V0 > 0) {
     mv::GemmSet& S = p.set[ns++];
     MV_TRY(tmap(&S.a0, w_lm, V0, H, 128));
-    MV_TRY(tmap(&S.b, h, T, H, 16));
+    MV_TRY(tmap(&S.b, h, T, H, bbox));
     S.a1 = S.a0;
     set_up(S, w_lm, V0, 0, 0, true);
     used = (V0 + 255) / 256 * 4;
@@ -541,7 +544,7 @@ mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, in
     mv::GemmSet& S = p.set[ns++];
     const uint16_t* tail = w_lm + static_cast<size_t>(V0) * H;
     MV_TRY(tmap(&S.a0, tail, V - V0, H, 128));
-    MV_TRY(tmap(&S.b, h, T, H, 16));
+    MV_TRY(tmap(&S.b, h, T, H, bbox));
     S.a1 = S.a0;
     set_up(S, tail, V - V0, V0, used, false);
     used += (V - V0 + 127) / 128 * 4;
@@ -550,7 +553,7 @@ mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, in
   p.nsets = ns;
   if (used > ld) return fail(MV_ERR_INTERNAL, "LM key slots %d exceed the row stride %d", used, ld);
   *nparts_used = used;
-  cudaError_t e = run_kernel(KIND_LM_GEMM, st, [&] { return mv::launch_gemm(mv::GEMM_LM, p, gemm_grid(units), st); });
+  cudaError_t e = run_kernel(KIND_LM_GEMM, st, [&] { return mv::launch_gemm(wide ? mv::GEMM_LM_WIDE : mv::GEMM_LM, p, gemm_grid(units), st); });
   if (e != cudaSuccess) return cuda_fail(e, "lm_head_gemm_argmax launch");
   return MV_OK;
 }

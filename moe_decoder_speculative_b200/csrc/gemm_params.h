@@ -11,7 +11,19 @@ enum { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_ARGMAX = 2, EPI_SWIGLU_ROWS = 3, E
 // the tokens-on-M modes load the same tiles but multiply 128 token rows by 256
 // weight rows (gate|up tiles, or two halves of W_down) into one accumulator.
 enum { MODE_SINGLE = 0, MODE_GATEUP = 1, MODE_KPAIR = 2, MODE_MPAIR = 3, MODE_TGATEUP = 4, MODE_TPAIR = 5 };
-enum { GEMM_MOE_DECODE = 0, GEMM_MOE_PREFILL = 1, GEMM_LM = 2 };
+enum { GEMM_MOE_DECODE = 0, GEMM_MOE_PREFILL = 1, GEMM_LM = 2, GEMM_LM_WIDE = 3 };
+
+// B-operand TMA box height (rows) of each tile configuration; the host builds
+// the B tensor maps with it.  Whole 128-row token tiles in one box matter: on
+// the 9,248-row prefill layer 128-row boxes ran the grouped GEMM in 616 us
+// against 757 us with 16-row boxes (8 boxes per stage).
+#ifndef MV_PREFILL_BBOX
+#define MV_PREFILL_BBOX 128
+#endif
+constexpr int kDecodeBBox = 16;
+constexpr int kPrefillBBox = MV_PREFILL_BBOX;
+constexpr int kLmBBox = 16;       // GEMM_LM: few token rows
+constexpr int kLmWideBBox = 128;  // GEMM_LM_WIDE: 128 or more token rows
 
 // Sticky device error bits, OR-ed into the workspace's error word.
 constexpr int kErrTimeout = 1;

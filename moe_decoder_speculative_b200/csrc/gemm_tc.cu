@@ -54,7 +54,6 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kMaxGroups = 2 * 256 + 8;   // routed + shared groups of both phases
 constexpr int kATileBytes = 128 * 128;  // 128 rows x 64 bf16
-constexpr int kBBox = 16;               // B rows per TMA box
 constexpr int kRing = 4;                // claimed units in flight inside a CTA
 
 struct UnitInfo {
@@ -79,8 +78,10 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 }  // namespace
 
-template <int BN, int STAGES, int NB, bool LM>
+template <int BN, int STAGES, int NB, bool LM, int BBOX>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams p) {
+  constexpr int kBBox = BBOX;  // B rows per TMA box (the B tensor maps are built with this box height)
+  static_assert(BBOX % 8 == 0 && BBOX <= BN, "BBOX");
   constexpr int B_TILE_BYTES = BN * 128;
   constexpr int STAGE_BYTES = 2 * kATileBytes + NB * B_TILE_BYTES;
   constexpr int ACC_COLS = 2 * BN;  // two accumulators (D0, D1) per slot
@@ -548,13 +549,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 // ---------------------------------------------------------------------------
 // host-side launch
 // ---------------------------------------------------------------------------
-template <int BN, int STAGES, int NB, bool LM>
+template <int BN, int STAGES, int NB, bool LM, int BBOX>
 static cudaError_t launch_gemm_impl(const GemmParams& p, int grid, cudaStream_t stream) {
   constexpr int STAGE_BYTES = 2 * kATileBytes + NB * BN * 128;
   constexpr int EXTRA = LM ? 4 * 32 * 33 * 4 : 0;  // argmax epilogue transpose buffers
   constexpr int SMEM = STAGES * STAGE_BYTES + EXTRA + 1024;
   static_assert(SMEM + 12 * 1024 <= 227 * 1024, "shared memory (dynamic + static)");
-  auto kern = gemm_tc_kernel<BN, STAGES, NB, LM>;
+  auto kern = gemm_tc_kernel<BN, STAGES, NB, LM, BBOX>;
   static thread_local int configured_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -569,12 +570,14 @@ static cudaError_t launch_gemm_impl(const GemmParams& p, int grid, cudaStream_t 
 // Tile configurations:
 //   GEMM_MOE_DECODE   BN = 32, two B k-block slots, 5 stages of 40 KB
 //   GEMM_MOE_PREFILL  BN = 128, one B slot, 4 stages of 48 KB (tokens-on-M modes)
-//   GEMM_LM           BN = 128, one B slot, 4 stages of 48 KB (MODE_MPAIR)
+//   GEMM_LM           BN = 128, one B slot, 4 stages of 48 KB (MODE_MPAIR), 16-row token boxes
+//   GEMM_LM_WIDE      the same with 128-row token boxes, for 128 or more tokens
 cudaError_t launch_gemm(int config, const GemmParams& p, int grid, cudaStream_t stream) {
   switch (config) {
-    case GEMM_MOE_DECODE: return launch_gemm_impl<32, 5, 2, false>(p, grid, stream);
-    case GEMM_MOE_PREFILL: return launch_gemm_impl<128, 4, 1, false>(p, grid, stream);
-    case GEMM_LM: return launch_gemm_impl<128, 4, 1, true>(p, grid, stream);
+    case GEMM_MOE_DECODE: return launch_gemm_impl<32, 5, 2, false, kDecodeBBox>(p, grid, stream);
+    case GEMM_MOE_PREFILL: return launch_gemm_impl<128, 4, 1, false, kPrefillBBox>(p, grid, stream);
+    case GEMM_LM: return launch_gemm_impl<128, 4, 1, true, kLmBBox>(p, grid, stream);
+    case GEMM_LM_WIDE: return launch_gemm_impl<128, 4, 1, true, kLmWideBBox>(p, grid, stream);
   }
   return cudaErrorInvalidValue;
 }
