@@ -464,11 +464,45 @@ mv_status ffn_forward_impl(const uint16_t* x, int T, const mv_moe_shape& s, cons
 }
 
 // Routing of T rows: the streaming combine+route kernel in route-only mode for
-// decode-sized batches, the shared-memory-staged router otherwise (both give
-// bit-identical logits and choices).
+// decode-sized batches, the shared-memory-staged router up to 1024 rows (both
+// give bit-identical logits and choices), the tensor cores beyond (fp32 logits
+// summed in another order: choices can differ only at near-tied logits).
 mv_status route_impl(const uint16_t* x, int T, const mv_moe_shape& s, const uint16_t* wr, const float* bias,
                      int32_t* idx, float* tw, int* err, cudaStream_t st,
                      const mv::L2Prefetch& pf = mv::L2Prefetch{}) {
+  if (T > 1024 && s.E <= 128) {
+    // Large batches: the router is a [T x H] . [H x E] contraction on the tensor
+    // cores, 128 tokens x E experts per unit; each epilogue thread holds one
+    // token's logits and does the top-k and renormalised softmax in registers.
+    // Static unit schedule, so no workspace is needed.
+    mv::GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.err = err;
+    p.sched = nullptr;
+    p.timeout_ns = timeout_ns();
+    mv::GemmSet& S = p.set[0];
+    S.mode = mv::MODE_TROUTE;
+    S.epi = mv::EPI_TOPK;
+    S.m_tile = 128;
+    S.dep_set = -1;
+    MV_TRY(tmap(&S.a0, wr, s.E, s.H, 128));
+    MV_TRY(tmap(&S.b, x, T, s.H, mv::kPrefillBBox));
+    S.a1 = S.a0;
+    S.out = idx;
+    S.out2 = tw;
+    S.bias = bias;
+    S.topk = s.k;
+    S.K = s.H;
+    S.M = s.E;
+    S.groups = 1;
+    S.static_rows = T;
+    p.nsets = 1;
+    const int64_t units = (T + 127) / 128;
+    cudaError_t e = run_kernel(KIND_ROUTER, st, [&] {
+      return mv::launch_gemm(mv::GEMM_MOE_PREFILL, p, gemm_grid(units), st);
+    });
+    return e == cudaSuccess ? MV_OK : cuda_fail(e, "router_topk (tensor-core) launch");
+  }
   cudaError_t e = run_kernel(KIND_ROUTER, st, [&] {
     if (mv::combine_route_supported(T, s.H, s.E)) {
       mv::CombineRouteArgs a{};

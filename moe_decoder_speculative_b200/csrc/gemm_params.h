@@ -6,11 +6,12 @@
 
 namespace mv {
 
-enum { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_ARGMAX = 2, EPI_SWIGLU_ROWS = 3, EPI_STORE_ROWS = 4 };
+enum { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_ARGMAX = 2, EPI_SWIGLU_ROWS = 3, EPI_STORE_ROWS = 4, EPI_TOPK = 5 };
 // Operand modes.  The first four put weights on the MMA's M side (swap-AB);
 // the tokens-on-M modes load the same tiles but multiply 128 token rows by 256
 // weight rows (gate|up tiles, or two halves of W_down) into one accumulator.
-enum { MODE_SINGLE = 0, MODE_GATEUP = 1, MODE_KPAIR = 2, MODE_MPAIR = 3, MODE_TGATEUP = 4, MODE_TPAIR = 5 };
+enum { MODE_SINGLE = 0, MODE_GATEUP = 1, MODE_KPAIR = 2, MODE_MPAIR = 3, MODE_TGATEUP = 4, MODE_TPAIR = 5,
+       MODE_TROUTE = 6 };  // MODE_TROUTE: 128 token rows x the M (<= 256) router rows, one accumulator
 enum { GEMM_MOE_DECODE = 0, GEMM_MOE_PREFILL = 1, GEMM_LM = 2, GEMM_LM_WIDE = 3 };
 
 // B-operand TMA box height (rows) of each tile configuration; the host builds
@@ -58,13 +59,16 @@ struct GemmSet {
   int32_t signal;          // 1: count finished epilogue warps per group (a later set depends on it)
   int32_t key_row_base;    // EPI_ARGMAX: vocabulary index of this set's A row 0
   int32_t key_part_base;   // EPI_ARGMAX: first key slot of this set within a token's row
+  void* out2;              // EPI_TOPK: fp32 weights [rows][topk] (`out` holds int32 ids [rows][topk])
+  const float* bias;       // EPI_TOPK: fp32 [M] added to the logits, or nullptr
+  int32_t topk;            // EPI_TOPK: k
 };
 
 struct GemmParams {
   GemmSet set[4];
   int32_t nsets;
   int* err;
-  int* sched;              // kSchedInts ints, zero at launch
+  int* sched;              // kSchedInts ints, zero at launch; nullptr: static round-robin units, no dependencies
   uint64_t timeout_ns;
 };
 

@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       for (int it = 0; ok; ++it) {
         const int q = it % kRing;
         if (!mbar_wait(&uempty_bar[q], ((it / kRing) & 1) ^ 1u, &abort_s, p.err, deadline)) break;
-        int u = atomicAdd(p.sched, 1);
+        int u = p.sched ? atomicAdd(p.sched, 1) : static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
         if (u >= total_units) u = -1;
         unit_ring[q] = u;
         mbar_arrive(&ufull_bar[q]);
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                             pol_x);
             }
           } else {
-            const bool two = (S.mode != MODE_SINGLE);
+            const bool two = (S.mode != MODE_SINGLE && S.mode != MODE_TROUTE);
             mbar_arrive_expect_tx(&full_bar[stage], (two ? 2u : 1u) * kATileBytes + b_bytes);
             tma_load_2d(st, &S.a0, ks * 64, a_row0, &full_bar[stage], pol_w);
             if (S.mode == MODE_GATEUP || S.mode == MODE_TGATEUP)
@@ -324,9 +324,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         const int slot = it & 1;
         if (!mbar_wait(&tempty_bar[slot], ((it >> 1) & 1) ^ 1u, &abort_s, p.err, deadline)) break;
         tc_fence_after();
-        const bool tok_m = (S.mode == MODE_TGATEUP || S.mode == MODE_TPAIR);
+        const bool tok_m = (S.mode == MODE_TGATEUP || S.mode == MODE_TPAIR || S.mode == MODE_TROUTE);
         const uint32_t n_mma = static_cast<uint32_t>((ui.nvalid + 15) & ~15);
-        const uint32_t idesc = tok_m ? idesc_bf16_f32(128, 256) : idesc_bf16_f32(128, n_mma);
+        const uint32_t n_tok = (S.mode == MODE_TROUTE) ? static_cast<uint32_t>((S.M + 15) & ~15) : 256u;
+        const uint32_t idesc = tok_m ? idesc_bf16_f32(128, n_tok) : idesc_bf16_f32(128, n_mma);
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(slot * ACC_COLS);
         const int kblocks = S.K / 64;
         const int nstage = (S.mode == MODE_KPAIR) ? (kblocks + 1) / 2 : kblocks;
@@ -403,7 +404,67 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       const int row = wq * 32 + lane;  // row of the 128-row tile held by this thread
       const uint32_t tl = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + static_cast<uint32_t>(slot * ACC_COLS);
       const int n_mma = (ui.nvalid + 15) & ~15;
-      if (S.epi == EPI_SWIGLU_ROWS || S.epi == EPI_STORE_ROWS) {
+      if (S.epi == EPI_TOPK) {
+        // tokens on M: this thread holds all router logits of token `row`;
+        // top-k on the logits (ties to the lower id, slots in descending
+        // order), weights exp(l_j - l_max) / sum over the kept experts.  The
+        // TMEM loads are warp-collective, so every lane issues them; only the
+        // selection and the stores depend on the row being valid.
+        const bool tvalid = row < ui.nvalid;
+        constexpr int kMaxK = 8;
+        float sv[kMaxK];
+        int si[kMaxK];
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) {
+          sv[j] = -__int_as_float(0x7f800000);
+          si[j] = 0x7fffffff;
+        }
+        for (int c0 = 0; c0 < S.M; c0 += 32) {
+          uint32_t d[32];
+          tmem_ld32(tl + c0, d);
+          tmem_ld_wait();
+          if (tvalid) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int e = c0 + j;
+              float v = __uint_as_float(d[j]);
+              if (e < S.M && S.bias) v += S.bias[e];
+              if (e < S.M && v > sv[kMaxK - 1]) {  // insert, larger first; equal values keep the earlier id
+                int pos = kMaxK - 1;
+#pragma unroll
+                for (int q = kMaxK - 1; q > 0; --q)
+                  if (v > sv[q - 1]) pos = q - 1;
+#pragma unroll
+                for (int q = kMaxK - 1; q > 0; --q)
+                  if (q > pos) {
+                    sv[q] = sv[q - 1];
+                    si[q] = si[q - 1];
+                  }
+#pragma unroll
+                for (int q = 0; q < kMaxK; ++q)
+                  if (q == pos) {
+                    sv[q] = v;
+                    si[q] = e;
+                  }
+              }
+            }
+          }
+        }
+        if (tvalid) {
+          float s = 0.f;
+#pragma unroll
+          for (int j = 0; j < kMaxK; ++j)
+            if (j < S.topk) s += expf(sv[j] - sv[0]);
+          int32_t* oi = static_cast<int32_t*>(S.out) + static_cast<size_t>(ui.b_row0 + row) * S.topk;
+          float* ow = static_cast<float*>(S.out2) + static_cast<size_t>(ui.b_row0 + row) * S.topk;
+#pragma unroll
+          for (int j = 0; j < kMaxK; ++j)
+            if (j < S.topk) {
+              oi[j] = si[j];
+              ow[j] = expf(sv[j] - sv[0]) / s;
+            }
+        }
+      } else if (S.epi == EPI_SWIGLU_ROWS || S.epi == EPI_STORE_ROWS) {
         // tokens on M: this thread holds token row `row` of the tile, the
         // columns are 256 weight outputs (gate|up, or two halves of W_down)
         const bool tvalid = row < ui.nvalid;
@@ -527,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
       }
       tc_fence_before();
-      if (S.signal) {  // release this warp's stores to the units that depend on the group
+      if (S.signal && p.sched) {  // release this warp's stores to the units that depend on the group
         fence_proxy_async_global();
         __syncwarp();
         if (lane == 0) {

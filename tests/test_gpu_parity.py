@@ -62,6 +62,26 @@ def test_router_topk(wid):
     assert np.all(np.abs(tw.sum(1) - 1) < 1e-5)
 
 
+@pytest.mark.parametrize("T,bias", [(1500, False), (2049, True)])
+def test_router_topk_large_batch(T, bias):
+    """Batches above 1024 rows route on the tensor cores (top-k in the epilogue)."""
+    rng = np.random.default_rng(T)
+    H, E, k = 1280, 64, 6
+    x = wl.f32_to_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    wr = wl.f32_to_bf16_bits(rng.standard_normal((E, H)).astype(np.float32) * 0.02)
+    b = rng.standard_normal(E).astype(np.float32) * 0.5 if bias else None
+    idx_ref, w_ref, _, gap = oracle.router(x, wr, k, bias=b)
+    shape = bd.MoeShape(H, E, 896, 0, k)
+    idx, tw = bd.moe_router_topk(bd.bf16_to_device(x), shape, bd.bf16_to_device(wr),
+                                 None if b is None else torch.from_numpy(b).cuda())
+    idx, tw = to_np(idx), to_np(tw)
+    ok = gap >= GATE_GAP
+    assert same_routing(idx, idx_ref)[ok].all()
+    same = np.all(idx == idx_ref, axis=1)
+    assert same.mean() > 0.95
+    np.testing.assert_allclose(tw[same], w_ref[same], rtol=2e-5, atol=2e-6)
+
+
 @pytest.mark.parametrize("T,E,k", [(16, 8, 2), (128, 64, 6), (37, 64, 6), (1, 8, 8), (1000, 256, 8)])
 def test_expert_permute(T, E, k):
     rng = np.random.default_rng(T * 7 + E)
