@@ -1,0 +1,148 @@
+"""The pages' central claim on the GPU kernels: greedy speculative decoding emits
+exactly the plain greedy stream, whatever the drafts.
+
+A toy causal decoder (V = 64, H = 64, two MoE layers of 8 routed experts top-2
+plus a shared expert, LM head) runs every verify pass through verify_step on
+the GPU.  Its input rows h = bf16(E1[token] + E2[previous token]) are built by
+the test (token embedding is not part of the verify path).  Plain greedy
+decoding is verify_step with K = 0, one row per sequence; speculative
+decoding verifies K drafts per pass from drafters that copy the greedy stream
+with p = 0.576, are always right, always wrong, or random.  Equality needs the
+kernels to be batch-invariant: a row's result may not depend on the other
+rows of its batch or expert group, nor on the batch size.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_decoder_speculative_b200 import binding as bd
+from moe_decoder_speculative_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+V, H, E, KTOP, I, ISH, L = 64, 64, 8, 2, 64, 64, 2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from moe_decoder_speculative_b200 import build
+    build.build()
+
+
+class ToyGPU:
+    def __init__(self, seed=0):
+        rng = np.random.default_rng(seed)
+        bf = lambda shape, s: wl.f32_to_bf16_bits(rng.standard_normal(shape).astype(np.float32) * s)
+        self.e1 = rng.standard_normal((V, H)).astype(np.float32)
+        self.e2 = rng.standard_normal((V, H)).astype(np.float32)
+        self.layers_np = [{"w_router": bf((E, H), 0.3), "w_gate": bf((E, I, H), 0.2), "w_up": bf((E, I, H), 0.2),
+                           "w_down": bf((E, H, I), 0.2), "ws_gate": bf((ISH, H), 0.2), "ws_up": bf((ISH, H), 0.2),
+                           "ws_down": bf((H, ISH), 0.2), "router_bias": None} for _ in range(L)]
+        self.w_lm_np = bf((V, H), 0.3)
+        self.layers = [bd.LayerWeights(l) for l in self.layers_np]
+        self.w_lm = bd.bf16_to_device(self.w_lm_np)
+        self.shape = bd.MoeShape(H, E, I, ISH, KTOP)
+        self.plans = {}
+
+    def rows(self, cur, prev):
+        # a draft id outside [0, V) never matches, so the rows it feeds are
+        # discarded; it is embedded as id mod V
+        cur, prev = np.mod(np.asarray(cur), V), np.mod(np.asarray(prev), V)
+        return wl.f32_to_bf16_bits(self.e1[cur] + self.e2[prev])
+
+    def verify(self, cur, prev, drafts, B, K):
+        key = (B, K)
+        if key not in self.plans:
+            self.plans[key] = bd.VerifyPlan(self.shape, self.layers, self.w_lm, B, K)
+        plan = self.plans[key]
+        d = torch.from_numpy(np.ascontiguousarray(drafts, np.int32)).cuda() if K else None
+        acc, nxt, em, am = plan(bd.bf16_to_device(self.rows(cur, prev)), d)
+        plan.sync_status()
+        return acc.cpu().numpy(), em.cpu().numpy(), am.cpu().numpy()
+
+
+def greedy(toy, prompts, n):
+    seqs = [list(p) for p in prompts]
+    B = len(seqs)
+    for _ in range(n):
+        _, em, _ = toy.verify([s[-1] for s in seqs], [s[-2] for s in seqs], None, B, 0)
+        for s, t in zip(seqs, em[:, 0]):
+            s.append(int(t))
+    return seqs
+
+
+def speculative(toy, prompts, n, K, drafter):
+    seqs = [list(p) for p in prompts]
+    B = len(seqs)
+    target = len(prompts[0]) + n
+    passes = 0
+    while min(len(s) for s in seqs) < target:
+        drafts = np.array([drafter(b, s, K) for b, s in enumerate(seqs)], np.int32).reshape(B, K)
+        cur, prev = [], []
+        for b, s in enumerate(seqs):
+            cur += [s[-1]] + list(drafts[b])
+            prev += ([s[-2], s[-1]] + list(drafts[b][:-1]))[:K + 1]
+        acc, em, _ = toy.verify(cur, prev, drafts, B, K)
+        for b, s in enumerate(seqs):
+            if len(s) < target:
+                s.extend(int(t) for t in em[b][:acc[b] + 1])
+        passes += 1
+    return [s[:target] for s in seqs], passes
+
+
+@pytest.mark.parametrize("K", [1, 3])
+@pytest.mark.parametrize("kind", ["copy0.576", "right", "wrong", "random"])
+def test_gpu_speculative_loop_equals_gpu_greedy(K, kind):
+    toy = ToyGPU()
+    rng = np.random.default_rng(1)
+    prompts = [list(rng.integers(0, V, size=2)) for _ in range(16)]
+    n = 120
+    ref = greedy(toy, prompts, n + 3 * (K + 1))
+
+    def drafter(b, s, K):
+        truth = list(ref[b][len(s):len(s) + K]) + [0] * K
+        out = []
+        for t in truth[:K]:
+            if kind == "right" or (kind == "copy0.576" and rng.random() < 0.576):
+                out.append(t)
+            elif kind == "wrong":
+                out.append((t + 1) % V)
+            else:
+                out.append(int(rng.integers(-2, V + 2)))   # includes ids outside [0, V): never match
+        return out
+
+    got, passes = speculative(toy, prompts, n, K, drafter)
+    assert got == [s[:len(got[0])] for s in ref]
+    if kind == "right":
+        assert passes <= -(-n // (K + 1)) + 1
+    if kind == "wrong":
+        assert passes == n
+
+
+def test_gpu_greedy_agrees_with_oracle_greedy_until_a_near_tie():
+    """The GPU's greedy stream follows the CPU oracle's until the first step
+    whose LM or gate decision is nearly tied on the oracle (then both are
+    valid continuations of different rounding).  The margins are wider than
+    the single-kernel ones because one step runs two layers: a last-bit
+    difference in layer 0's output moves layer 1's router and the LM logits."""
+    toy = ToyGPU()
+    rng = np.random.default_rng(2)
+    prompts = [list(rng.integers(0, V, size=2)) for _ in range(8)]
+    n = 60
+    gpu = greedy(toy, prompts, n)
+    agree = 0
+    for b, p in enumerate(prompts):
+        s = list(p)
+        for t in range(n):
+            st = oracle.verify_step(toy.rows([s[-1]], [s[-2]]), None, 1, 0, toy.layers_np, KTOP, toy.w_lm_np)
+            nxt = int(st["argmax"][0])
+            flagged = st["lm_gap"][0] < 5e-2 or any(l["gap"][0] < 5e-2 for l in st["layers"])
+            if nxt != gpu[b][len(s)]:
+                assert flagged, f"sequence {b} step {t}: unflagged disagreement"
+                break
+            s.append(nxt)
+            agree += 1
+    assert agree >= 0.5 * n * len(prompts)
