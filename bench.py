@@ -55,6 +55,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="run only the first N MoE layers (a smaller case for profiling; not a bench line)")
+    ap.add_argument("--graph", action="store_true",
+                    help="time replays of the step recorded once as a CUDA graph (verify_graph_*)")
+    ap.add_argument("--latency", action="store_true",
+                    help="per-step latency of one sequence (batch 1) for K = 0, 1, 3, eager and graph")
     return ap.parse_args()
 
 
@@ -328,10 +332,15 @@ def run_ours(args):
     plan.sync_status()
 
     stream = torch.cuda.current_stream()
+    step = lambda: plan(hidden, drafts)
+    graph = None
+    if args.graph:   # the step recorded once; replays read the same (resident) input buffers
+        graph = bd.VerifyGraph(plan, hidden, drafts)
+        step = graph
     for _ in range(max(3, args.warmup)):
-        plan(hidden, drafts)
+        step()
     torch.cuda.synchronize()
-    acc, _, _, _ = plan(hidden, drafts)
+    acc, _, _, _ = step()
     committed_per_step = int((acc + 1).sum().item())
 
     with ClockSampler(gpu_uuid(torch, dev)) as clocks:
@@ -342,7 +351,7 @@ def run_ours(args):
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ev0.record(stream)
         for _ in range(args.steps):
-            plan(hidden, drafts)
+            step()
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier()
@@ -370,6 +379,10 @@ def run_ours(args):
         dr_h = torch.from_numpy(drafts_np).pin_memory()
         hid_d = torch.empty_like(hid_h, device=dev)
         dr_d = torch.empty_like(dr_h, device=dev)
+        e2e_step, e2e_graph = (lambda: plan(hid_d.view(torch.bfloat16), dr_d)), None
+        if args.graph:
+            e2e_graph = bd.VerifyGraph(plan, hid_d.view(torch.bfloat16), dr_d)
+            e2e_step = e2e_graph
         acc_h = torch.empty(w.B, dtype=torch.int32).pin_memory()
         nxt_h = torch.empty(w.B, dtype=torch.int32).pin_memory()
         em_h = torch.empty((w.B, w.K + 1), dtype=torch.int32).pin_memory()
@@ -380,7 +393,7 @@ def run_ours(args):
         for _ in range(args.steps):
             hid_d.copy_(hid_h, non_blocking=True)
             dr_d.copy_(dr_h, non_blocking=True)
-            a, nx, em, _ = plan(hid_d.view(torch.bfloat16), dr_d)
+            a, nx, em, _ = e2e_step()
             acc_h.copy_(a, non_blocking=True)
             nxt_h.copy_(nx, non_blocking=True)
             em_h.copy_(em, non_blocking=True)
@@ -421,6 +434,7 @@ def run_ours(args):
         "config": {"workload": w.name, "B": w.B, "K": w.K, "rows": T, "layers": len(layers), "H": w.H, "E": w.E,
                    "top_k": w.k, "I": w.I, "I_shared": w.I_sh, "V": w.V,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "launch": "CUDA graph replay (verify_graph_launch)" if args.graph else "eager (verify_step)",
                    "l2": "weights (5.8 GB) far larger than L2: no flush needed"},
         "rows_per_s": world * T * K / (ms / 1e3),
         "committed_per_step": committed_all,
@@ -451,9 +465,93 @@ def run_ours(args):
                                          f"accept, one pass, {dt:.1f} s"}
     if rank == 0:
         print(json.dumps(out))
-    plan = None
+    plan = graph = e2e_graph = step = e2e_step = None
     if world > 1:
         dist.destroy_process_group()
+    return 0
+
+
+def run_latency(args):
+    """One sequence (batch 1): host-to-result latency of one verify step for
+    K = 0, 1, 3 drafts, launched eagerly (verify_step) or as a replay of the
+    recorded step (verify_graph_launch).  Each step's device time runs from
+    an event recorded before the launch call to one recorded after it, with
+    the host synchronised after every step, so launch overhead counts.
+    Committed tokens per second = the mean committed tokens per step (drafts
+    copy the verifier's own argmax w.p. p, fresh drafts every step) over the
+    median step latency."""
+    import dataclasses
+
+    import torch
+
+    from moe_decoder_speculative_b200 import binding as bd
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    base = wl.workload(args.workload if args.workload != 2 else 1)
+    assert base.has_verify and base.B == 1, "the latency table is for a batch-1 verify workload"
+    layers_n = args.layers if args.layers else base.L
+    base = dataclasses.replace(base, L=max(base.L, layers_n))   # layer l has the same bytes at any depth
+    inp0 = wl.make_inputs(base, layers=layers_n)
+    shape = bd.shape_of(base)
+    layers = [bd.LayerWeights(l, dev) for l in inp0["layers"]]
+    w_lm = bd.bf16_to_device(inp0["w_lm"], dev)
+    stream = torch.cuda.current_stream()
+    n_steps = max(50, args.steps)
+    rows = []
+    for K in (0, 1, 3):
+        w = dataclasses.replace(base, K=K)
+        hidden = bd.bf16_to_device(wl.make_hidden(w), dev)
+        plan = bd.VerifyPlan(shape, layers, w_lm, 1, K, dev)
+        _, _, _, am = plan(hidden, torch.zeros((1, max(1, K)), dtype=torch.int32, device=dev))
+        am = am.cpu().numpy()
+        sets = [torch.from_numpy(wl.make_drafts(w, am, ss=np.random.SeedSequence([w.id, K, i]))
+                                 if K else np.zeros((1, 1), np.int32)).to(dev) for i in range(n_steps)]
+        dr_buf = torch.zeros((1, max(1, K)), dtype=torch.int32, device=dev)
+        graph = bd.VerifyGraph(plan, hidden, dr_buf)
+        for mode in ("eager", "graph"):
+            def one(i):
+                if mode == "eager":
+                    return plan(hidden, sets[i])
+                dr_buf.copy_(sets[i])
+                return graph()
+            for i in range(max(3, args.warmup)):
+                one(i % n_steps)
+            torch.cuda.synchronize()
+            times, committed = [], 0
+            for i in range(n_steps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                acc, _, _, _ = one(i)
+                e1.record(stream)
+                e1.synchronize()
+                times.append(e0.elapsed_time(e1))
+                committed += int(acc[0].item()) + 1
+            plan.sync_status()
+            lat = float(np.median(times))
+            row = {"K": K, "launch": mode, "latency_us": round(lat * 1e3, 2),
+                   "p90_us": round(float(np.percentile(times, 90)) * 1e3, 2),
+                   "committed_per_step": round(committed / n_steps, 4),
+                   "committed_tok_s": round(committed / n_steps / (lat / 1e3), 1),
+                   "kernels_per_step": graph.kernels}
+            if mode == "eager":   # per-kernel device time of the same steps, one event pair per launch
+                bd.profile_enable(True)
+                for i in range(n_steps):
+                    one(i)
+                torch.cuda.synchronize()
+                bd.profile_enable(False)
+                kern = bd.profile_collect()
+                row["kernels_us"] = {k: round(1e3 * v["ms"] / v["launches"], 2) for k, v in kern.items()
+                                     if v["launches"]}
+            rows.append(row)
+        graph.close()
+    best = max(rows, key=lambda r: r["committed_tok_s"])
+    print(json.dumps({
+        "metric": "batch-1 verify latency and committed tokens/s by draft count", "value": best["committed_tok_s"],
+        "unit": "tokens/s", "n_gpus": 1, "steps": n_steps, "warmup": args.warmup, "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic (seeded weights; drafts copy the verifier argmax w.p. 0.576)",
+        "config": {"workload": base.name, "B": 1, "layers": layers_n, "H": base.H, "E": base.E, "V": base.V},
+        "best": best, "table": rows}))
     return 0
 
 
@@ -533,6 +631,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.latency:
+        return run_latency(args)
     if not wl.workload(args.workload).has_verify:
         return run_prefill(args)
     return run_ours(args)

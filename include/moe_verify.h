@@ -221,6 +221,42 @@ MV_API mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int3
                       int32_t* next_token, int32_t* emitted, int32_t* argmax, void* ws,
                       size_t ws_bytes, mv_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * verify_graph_* - verify_step recorded once into a CUDA graph and replayed.
+ * The model card's decoding-speed paragraph reports that replaying the
+ * decoder as CUDA graphs changes which draft count K is fastest at batch 1,
+ * because a batch-1 step is bound by launch latency more than by bytes.
+ *
+ * verify_graph_create takes exactly verify_step's arguments (same meaning,
+ * layout and checks; the stream is replaced by the handle out-parameter) and
+ * records the step on a private stream without running it.  Every pointer,
+ * size, the weights and the device-wait bound in force
+ * (mv_set_wait_timeout_ns) are fixed in the graph: before each replay the
+ * caller writes the step's inputs into the SAME hidden and drafts buffers, and
+ * reads the outputs from the same output buffers after it.
+ * verify_graph_launch replays the step on `stream` (asynchronous, like
+ * verify_step); replays on one workspace must not overlap in time, so launch
+ * them on one stream or order them with events.  Device-side errors land in
+ * the workspace's sticky word as with verify_step (read by mv_sync_status).
+ * verify_graph_kernels gives the number of kernels one replay launches
+ * (mv_launch_count advances by it per replay); verify_graph_destroy frees the
+ * graph (NULL is allowed).  The handle is owned by the caller and belongs to
+ * the device that was current at creation.  Creation fails with
+ * MV_ERR_INVALID_ARG while mv_profile_enable is on (its per-launch events
+ * cannot be recorded into a graph) and with MV_ERR_CUDA if the CUDA runtime
+ * refuses to record or instantiate the graph.
+ * ------------------------------------------------------------------------- */
+typedef struct mv_verify_graph mv_verify_graph;
+
+MV_API mv_status verify_graph_create(const uint16_t* hidden, const int32_t* drafts, int32_t B, int32_t K,
+                                     const mv_moe_shape* shape, const mv_moe_weights* layers,
+                                     int32_t n_layers, const uint16_t* w_lm, int32_t V, int32_t* accepted,
+                                     int32_t* next_token, int32_t* emitted, int32_t* argmax, void* ws,
+                                     size_t ws_bytes, mv_verify_graph** graph);
+MV_API mv_status verify_graph_launch(mv_verify_graph* graph, mv_stream_t stream);
+MV_API int32_t verify_graph_kernels(const mv_verify_graph* graph);
+MV_API mv_status verify_graph_destroy(mv_verify_graph* graph);
+
 /* Clears the workspace's header (its sticky error word) on the stream.  Call
  * once on a freshly allocated workspace before its first use (a workspace
  * allocated zero-filled needs no call). */

@@ -24,7 +24,8 @@ EXPORTED = ["moe_router_topk", "moe_expert_permute", "moe_ffn_workspace_size", "
             "lm_head_workspace_size", "lm_head_argmax", "greedy_accept", "verify_step_workspace_size",
             "verify_step", "mv_workspace_init", "mv_sync_status", "mv_last_error", "mv_version",
             "mv_launch_count", "mv_profile_enable", "mv_profile_collect", "mv_kernel_name",
-            "mv_set_wait_timeout_ns", "lm_head_argmax_noalloc"]
+            "mv_set_wait_timeout_ns", "lm_head_argmax_noalloc", "verify_graph_create", "verify_graph_launch",
+            "verify_graph_kernels", "verify_graph_destroy"]
 
 
 class MVError(RuntimeError):
@@ -76,6 +77,11 @@ def lib():
             "mv_profile_collect": (i32, [P, P, i32]),
             "mv_kernel_name": (ctypes.c_char_p, [i32]),
             "mv_set_wait_timeout_ns": (None, [i64]),
+            "verify_graph_create": (i32, [P, P, i32, i32, S, W, i32, P, i32, P, P, P, P, P, sz,
+                                          ctypes.POINTER(ctypes.c_void_p)]),
+            "verify_graph_launch": (i32, [P, P]),
+            "verify_graph_kernels": (i32, [P]),
+            "verify_graph_destroy": (i32, [P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -251,6 +257,46 @@ class VerifyPlan:
 
     def sync_status(self, stream=None):
         sync_status(self.ws, stream)
+
+
+class VerifyGraph:
+    """A VerifyPlan's step recorded once as a CUDA graph over fixed input
+    buffers (verify_graph_create); each call replays it (verify_graph_launch).
+    Write the next step's rows into `hidden` and drafts into `drafts` (in
+    place) before a call; the outputs are the plan's output tensors."""
+
+    def __init__(self, plan: VerifyPlan, hidden, drafts=None):
+        self.plan, self.hidden = plan, hidden
+        self.drafts = drafts if plan.K > 0 else None
+        h = ctypes.c_void_p()
+        _check(lib().verify_graph_create(_p(hidden), _p(self.drafts), plan.B, plan.K, ctypes.byref(plan.shape),
+                                         plan.c_layers, len(plan.layers), _p(plan.w_lm), plan.V, _p(plan.accepted),
+                                         _p(plan.next_token), _p(plan.emitted), _p(plan.argmax), _p(plan.ws),
+                                         plan.ws.numel(), ctypes.byref(h)))
+        self._h = h
+
+    @property
+    def kernels(self) -> int:
+        return int(lib().verify_graph_kernels(self._h))
+
+    def __call__(self, stream=None):
+        _check(lib().verify_graph_launch(self._h, _stream(stream)))
+        p = self.plan
+        return p.accepted, p.next_token, p.emitted, p.argmax
+
+    def sync_status(self, stream=None):
+        self.plan.sync_status(stream)
+
+    def close(self):
+        if self._h is not None and self._h.value:
+            lib().verify_graph_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def verify_step(hidden, drafts, B, K, shape, layers, w_lm, stream=None):

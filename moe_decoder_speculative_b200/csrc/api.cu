@@ -94,10 +94,15 @@ cudaEvent_t take_event() {
   return e;
 }
 
+// Set while verify_graph_create records a step: launches then go into the
+// graph instead of running, so they are neither timed nor counted here (a
+// replay counts its kernels when it is launched).
+thread_local bool t_recording = false;
+
 template <class F>
 cudaError_t run_kernel(int kind, cudaStream_t s, F&& launch) {
   cudaEvent_t a = nullptr, b = nullptr;
-  const bool prof = g_prof_on.load(std::memory_order_relaxed);
+  const bool prof = !t_recording && g_prof_on.load(std::memory_order_relaxed);
   if (prof) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
     a = take_event();
@@ -110,7 +115,7 @@ cudaError_t run_kernel(int kind, cudaStream_t s, F&& launch) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
     g_prof_recs.push_back({kind, a, b});
   }
-  if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e == cudaSuccess && !t_recording) g_launches.fetch_add(1, std::memory_order_relaxed);
   return e;
 }
 
@@ -864,6 +869,100 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
                                        next_token, emitted, argmax, st);
   });
   return e == cudaSuccess ? MV_OK : cuda_fail(e, "greedy_accept launch");
+}
+
+}  // extern "C"
+
+struct mv_verify_graph {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  int32_t kernels = 0;
+};
+
+namespace {
+
+void free_graph(mv_verify_graph* g) {
+  if (!g) return;
+  if (g->exec) cudaGraphExecDestroy(g->exec);
+  if (g->graph) cudaGraphDestroy(g->graph);
+  delete g;
+}
+
+}  // namespace
+
+extern "C" {
+
+mv_status verify_graph_create(const uint16_t* hidden, const int32_t* drafts, int32_t B, int32_t K,
+                              const mv_moe_shape* shape, const mv_moe_weights* layers, int32_t n_layers,
+                              const uint16_t* w_lm, int32_t V, int32_t* accepted, int32_t* next_token,
+                              int32_t* emitted, int32_t* argmax, void* ws, size_t ws_bytes,
+                              mv_verify_graph** graph) {
+  if (!graph) return fail(MV_ERR_INVALID_ARG, "graph out-parameter is NULL");
+  *graph = nullptr;
+  if (g_prof_on.load()) return fail(MV_ERR_INVALID_ARG, "profiling is on: its events cannot be recorded into a graph");
+  cudaStream_t cs = nullptr;
+  cudaError_t e = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking);
+  if (e != cudaSuccess) return cuda_fail(e, "creating the recording stream");
+  // Relaxed mode: the one-time host set-up a first call may do (kernel
+  // attributes, tensor-map encoding) is not a stream operation and stays
+  // legal while this thread records.
+  e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeRelaxed);
+  if (e != cudaSuccess) {
+    cudaStreamDestroy(cs);
+    return cuda_fail(e, "beginning the graph recording");
+  }
+  t_recording = true;
+  const mv_status st = verify_step(hidden, drafts, B, K, shape, layers, n_layers, w_lm, V, accepted, next_token,
+                                   emitted, argmax, ws, ws_bytes, reinterpret_cast<mv_stream_t>(cs));
+  t_recording = false;
+  const std::string step_msg = g_last_error;
+  mv_verify_graph* g = new mv_verify_graph();
+  e = cudaStreamEndCapture(cs, &g->graph);
+  cudaStreamDestroy(cs);
+  if (st != MV_OK) {
+    free_graph(g);
+    g_last_error = step_msg;
+    return st;
+  }
+  if (e != cudaSuccess) {
+    free_graph(g);
+    return cuda_fail(e, "ending the graph recording");
+  }
+  size_t n = 0;
+  e = cudaGraphGetNodes(g->graph, nullptr, &n);
+  std::vector<cudaGraphNode_t> nodes(n);
+  if (e == cudaSuccess && n) e = cudaGraphGetNodes(g->graph, nodes.data(), &n);
+  if (e != cudaSuccess) {
+    free_graph(g);
+    return cuda_fail(e, "listing the graph's nodes");
+  }
+  for (cudaGraphNode_t node : nodes) {
+    cudaGraphNodeType t{};
+    if (cudaGraphNodeGetType(node, &t) == cudaSuccess && t == cudaGraphNodeTypeKernel) ++g->kernels;
+  }
+  e = cudaGraphInstantiateWithFlags(&g->exec, g->graph, 0);
+  if (e != cudaSuccess) {
+    g->exec = nullptr;
+    free_graph(g);
+    return cuda_fail(e, "instantiating the graph");
+  }
+  *graph = g;
+  return MV_OK;
+}
+
+mv_status verify_graph_launch(mv_verify_graph* graph, mv_stream_t stream) {
+  if (!graph || !graph->exec) return fail(MV_ERR_INVALID_ARG, "graph is NULL");
+  cudaError_t e = cudaGraphLaunch(graph->exec, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "graph launch");
+  g_launches.fetch_add(static_cast<uint64_t>(graph->kernels), std::memory_order_relaxed);
+  return MV_OK;
+}
+
+int32_t verify_graph_kernels(const mv_verify_graph* graph) { return graph ? graph->kernels : -1; }
+
+mv_status verify_graph_destroy(mv_verify_graph* graph) {
+  free_graph(graph);
+  return MV_OK;
 }
 
 mv_status mv_workspace_init(void* ws, size_t ws_bytes, mv_stream_t stream) {

@@ -357,6 +357,7 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
   pdl_trigger();
   if (blockIdx.x == 0 && tid == 0) prefetch_l2_bulk(wr, static_cast<uint32_t>(E) * H * 2);  // weights: no dependency
   prefetch_share(pf);  // the next GEMM's first weights, while HBM is otherwise idle
+  if (row0 >= T) return;  // a prefetch-only CTA (uniform across the CTA)
   pdl_wait();  // expert outputs / rows come from the previous kernel
 
   // (1) rows of h into shared memory
@@ -490,7 +491,9 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
 template <int R, int NV>
 static cudaError_t launch_combine_route_rv(const CombineRouteArgs& a, cudaStream_t s) {
   const size_t smem = static_cast<size_t>(R) * a.H * 2 + static_cast<size_t>(R) * a.E * 4;
-  return launch_pdl(combine_route_kernel<R, NV>, dim3((a.T + R - 1) / R), dim3(512), smem, s, a.x, a.y_perm, a.y_sh, a.inv,
+  const int rows_ctas = (a.T + R - 1) / R;
+  const int grid = rows_ctas > prefetch_ctas(a.pf) ? rows_ctas : prefetch_ctas(a.pf);  // extra CTAs only prefetch
+  return launch_pdl(combine_route_kernel<R, NV>, dim3(grid), dim3(512), smem, s, a.x, a.y_perm, a.y_sh, a.inv,
              a.w_prev, a.k_prev, a.T * a.k_prev, a.out, a.T, a.H, a.E, a.k, a.wr, a.bias, a.idx, a.w, a.err, a.pf);
 }
 
@@ -871,7 +874,8 @@ cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t
   if (T <= 0) return cudaSuccess;
   const long long total = static_cast<long long>(T) * (H / 8);
   const long long blocks = (total + 255) / 256;
-  const int grid = static_cast<int>(blocks < 148LL * 8 ? blocks : 148LL * 8);
+  int grid = static_cast<int>(blocks < 148LL * 8 ? blocks : 148LL * 8);
+  if (grid < prefetch_ctas(pf)) grid = prefetch_ctas(pf);  // the grid-stride loop leaves the extra CTAs idle
   return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, s, y_perm, y_sh, inv, w, res, out, T, H, k, T * k, err,
                     pf);
 }

@@ -40,6 +40,16 @@ struct L2Prefetch {
   int n;
 };
 
+// CTAs a kernel needs so that no CTA issues more than 256 KB of the prefetch:
+// one SM issues bulk prefetches at roughly 200 GB/s, so a kernel with few
+// rows (one CTA per row at batch 1) launches extra CTAs that only prefetch.
+inline int prefetch_ctas(const L2Prefetch& pf) {
+  uint64_t total = 0;
+  for (int i = 0; i < pf.n; ++i) total += pf.bytes[i];
+  const uint64_t n = (total + (256u << 10) - 1) >> 18;
+  return static_cast<int>(n < 148 ? n : 148);
+}
+
 // Small CUDA-core kernels (kernels_small.cu).
 struct CombineRouteArgs {
   const uint16_t* x;        // residual rows (combine) or the rows to route (route only)

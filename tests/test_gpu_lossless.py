@@ -7,7 +7,9 @@ the GPU.  Its input rows h = bf16(E1[token] + E2[previous token]) are built by
 the test (token embedding is not part of the verify path).  Plain greedy
 decoding is verify_step with K = 0, one row per sequence; speculative
 decoding verifies K drafts per pass from drafters that copy the greedy stream
-with p = 0.576, are always right, always wrong, or random.  Equality needs the
+with p = 0.576, are always right, always wrong, or random.  Each loop runs
+once with eager verify_step calls and once with replays of recorded
+verify_graph handles.  Equality needs the
 kernels to be batch-invariant: a row's result may not depend on the other
 rows of its batch or expert group, nor on the batch size.
 """
@@ -33,7 +35,8 @@ def _need_gpu():
 
 
 class ToyGPU:
-    def __init__(self, seed=0):
+    def __init__(self, seed=0, use_graph=False):
+        self.use_graph = use_graph
         rng = np.random.default_rng(seed)
         bf = lambda shape, s: wl.f32_to_bf16_bits(rng.standard_normal(shape).astype(np.float32) * s)
         self.e1 = rng.standard_normal((V, H)).astype(np.float32)
@@ -56,10 +59,24 @@ class ToyGPU:
     def verify(self, cur, prev, drafts, B, K):
         key = (B, K)
         if key not in self.plans:
-            self.plans[key] = bd.VerifyPlan(self.shape, self.layers, self.w_lm, B, K)
-        plan = self.plans[key]
+            plan = bd.VerifyPlan(self.shape, self.layers, self.w_lm, B, K)
+            graph = None
+            if self.use_graph:   # fixed input buffers, refilled before every replay
+                hid = torch.empty((B * (K + 1), H), dtype=torch.bfloat16, device="cuda")
+                dr = torch.empty((B, max(1, K)), dtype=torch.int32, device="cuda")
+                graph = (bd.VerifyGraph(plan, hid, dr), hid, dr)
+            self.plans[key] = (plan, graph)
+        plan, graph = self.plans[key]
+        hidden = bd.bf16_to_device(self.rows(cur, prev))
         d = torch.from_numpy(np.ascontiguousarray(drafts, np.int32)).cuda() if K else None
-        acc, nxt, em, am = plan(bd.bf16_to_device(self.rows(cur, prev)), d)
+        if graph is None:
+            acc, nxt, em, am = plan(hidden, d)
+        else:
+            g, hid, dr = graph
+            hid.copy_(hidden)
+            if K:
+                dr.copy_(d)
+            acc, nxt, em, am = g()
         plan.sync_status()
         return acc.cpu().numpy(), em.cpu().numpy(), am.cpu().numpy()
 
@@ -93,13 +110,16 @@ def speculative(toy, prompts, n, K, drafter):
     return [s[:target] for s in seqs], passes
 
 
+@pytest.mark.parametrize("mode", ["eager", "graph"])
 @pytest.mark.parametrize("K", [1, 3])
 @pytest.mark.parametrize("kind", ["copy0.576", "right", "wrong", "random"])
-def test_gpu_speculative_loop_equals_gpu_greedy(K, kind):
-    toy = ToyGPU()
+def test_gpu_speculative_loop_equals_gpu_greedy(K, kind, mode):
+    """200 tokens from 16 seeded prompts; in graph mode every verify pass (and
+    the K = 0 greedy reference) is a replay of a recorded verify_graph."""
+    toy = ToyGPU(use_graph=(mode == "graph"))
     rng = np.random.default_rng(1)
     prompts = [list(rng.integers(0, V, size=2)) for _ in range(16)]
-    n = 120
+    n = 200
     ref = greedy(toy, prompts, n + 3 * (K + 1))
 
     def drafter(b, s, K):
