@@ -261,22 +261,39 @@ struct Carve {
 
 struct FfnWs {
   int32_t *counts, *offsets, *perm, *inv, *sort;
+  int32_t* inv_alt;  // slab layout: the other layer's inverse map (layers alternate)
   uint16_t *x_perm, *a_perm, *a_sh;
   float *y_perm, *y_sh;
+  int64_t n_pos;     // rows of x_perm / a_perm / y_perm
 };
 
-FfnWs carve_ffn(Carve& c, int64_t T, const mv_moe_shape& s) {
+// Decode-sized verify steps group the routed rows by expert inside the
+// routing kernel (combine_route) instead of a permute launch: expert e owns
+// rows [e*T, (e+1)*T) of x_perm, a_perm and y_perm (a row selects an expert
+// at most once, so T rows always suffice) and its row count is an atomic
+// counter in the layer's scheduling block.  Larger batches keep the compact
+// stable permutation.
+bool use_slabs(int64_t T, const mv_moe_shape& s) {
+  return T * s.k <= 16LL * s.E && mv::combine_route_supported(static_cast<int>(T), s.H, s.E);
+}
+constexpr int kSlabCountOff = 768;  // per-expert slab counters within a layer's scheduling block
+static_assert(1 + mv::kMaxGroups <= kSlabCountOff && kSlabCountOff + 256 <= mv::kSchedInts, "scheduling block");
+
+FfnWs carve_ffn(Carve& c, int64_t T, const mv_moe_shape& s, bool slabs = false) {
   FfnWs w;
   const size_t n = static_cast<size_t>(T) * s.k;
+  const size_t rows = slabs ? static_cast<size_t>(T) * s.E : n;
+  w.n_pos = static_cast<int64_t>(rows);
   w.counts = c.take<int32_t>(s.E);
   w.offsets = c.take<int32_t>(s.E + 1);
   w.perm = c.take<int32_t>(n);
   w.inv = c.take<int32_t>(n);
+  w.inv_alt = slabs ? c.take<int32_t>(n) : nullptr;
   w.sort = c.take<int32_t>(mv::permute_uses_sort(static_cast<int>(T), s.k) ? mv::sort_scratch_ints(static_cast<int>(T), s.E, s.k) : 1);
-  w.x_perm = c.take<uint16_t>(n * s.H);
-  w.a_perm = c.take<uint16_t>(n * s.I);
+  w.x_perm = c.take<uint16_t>(rows * s.H);
+  w.a_perm = c.take<uint16_t>(rows * s.I);
   w.a_sh = c.take<uint16_t>(static_cast<size_t>(T) * s.I_shared);
-  w.y_perm = c.take<float>(n * s.H);
+  w.y_perm = c.take<float>(rows * s.H);
   w.y_sh = c.take<float>(static_cast<size_t>(T) * s.H);
   return w;
 }
@@ -342,7 +359,8 @@ constexpr uint64_t kPrefetchBudget = static_cast<uint64_t>(MV_PREFETCH_BUDGET_MB
 // projection (fp32 rows) of the shared expert and the routed experts in one
 // persistent launch; a down unit waits for its expert's gate/up units.
 mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const mv_moe_weights& w,
-                        const FfnWs& ws, int* err, int* sched, cudaStream_t st) {
+                        const FfnWs& ws, int* err, int* sched, cudaStream_t st,
+                        const int32_t* slab_counts = nullptr) {
   const int H = s.H, E = s.E, I = s.I, Ish = s.I_shared, k = s.k;
   const int n = T * k;
   const bool decode = static_cast<int64_t>(n) <= 16LL * E;  // routed groups average <= 16 rows
@@ -384,14 +402,15 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
     base(S, tokm ? mv::MODE_TGATEUP : mv::MODE_GATEUP, tokm ? mv::EPI_SWIGLU_ROWS : mv::EPI_SWIGLU);
     MV_TRY(tmap(&S.a0, w.w_gate, static_cast<uint64_t>(E) * I, H, 128));
     MV_TRY(tmap(&S.a1, w.w_up, static_cast<uint64_t>(E) * I, H, 128));
-    MV_TRY(tmap(&S.b, ws.x_perm, n, H, bbox));
+    MV_TRY(tmap(&S.b, ws.x_perm, ws.n_pos, H, bbox));
     S.out = ws.a_perm;
     S.ld_out = I;
     S.K = H;
     S.M = I;
     S.groups = E;
-    S.counts = ws.counts;
-    S.offsets = ws.offsets;
+    S.counts = slab_counts ? slab_counts : ws.counts;
+    S.offsets = slab_counts ? nullptr : ws.offsets;
+    S.slab_rows = slab_counts ? T : 0;
     S.a_group_stride = I;
     S.signal = 1;
     units += int64_t((I + 127) / 128) * (std::min(E, n) + (n + BN - 1) / BN);
@@ -425,15 +444,16 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
     base(S, down_mode, down_epi);
     S.m_tile = down_tile;
     MV_TRY(tmap(&S.a0, w.w_down, static_cast<uint64_t>(E) * H, I, 128));
-    MV_TRY(tmap(&S.b, ws.a_perm, n, I, bbox));
+    MV_TRY(tmap(&S.b, ws.a_perm, ws.n_pos, I, bbox));
     S.a1 = S.a0;
     S.out = ws.y_perm;
     S.ld_out = H;
     S.K = I;
     S.M = H;
     S.groups = E;
-    S.counts = ws.counts;
-    S.offsets = ws.offsets;
+    S.counts = slab_counts ? slab_counts : ws.counts;
+    S.offsets = slab_counts ? nullptr : ws.offsets;
+    S.slab_rows = slab_counts ? T : 0;
     S.a_group_stride = H;
     S.dep_set = rt1;
     units += int64_t((H + 127) / 128) * (std::min(E, n) + (n + BN - 1) / BN);
@@ -450,19 +470,26 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
 mv_status ffn_forward_impl(const uint16_t* x, int T, const mv_moe_shape& s, const mv_moe_weights& w,
                            const int32_t* idx, const float* tw, const uint16_t* res, uint16_t* out,
                            const FfnWs& ws, int* err, int* sched, cudaStream_t st, bool do_combine = true,
-                           const mv::L2Prefetch& combine_pf = mv::L2Prefetch{}) {
-  cudaError_t e = run_kernel(KIND_PERMUTE, st, [&] {
-    if (mv::permute_uses_sort(T, s.k))
-      return mv::launch_permute_sorted(idx, T, s.E, s.k, ws.counts, ws.offsets, ws.perm, ws.inv, x, s.H, ws.x_perm,
-                                       ws.sort, st);
-    return mv::launch_permute(idx, T, s.E, s.k, ws.counts, ws.offsets, ws.perm, ws.inv, x, s.H, ws.x_perm, st);
-  });
-  if (e != cudaSuccess) return cuda_fail(e, "expert_permute launch");
-  MV_TRY(moe_gemm_impl(x, T, s, w, ws, err, sched, st));
+                           const mv::L2Prefetch& combine_pf = mv::L2Prefetch{},
+                           const int32_t* slab_counts = nullptr, const int32_t* slab_inv = nullptr) {
+  // With slab_counts the routing kernel has already grouped the rows (slab
+  // layout; slab_inv is its inverse map) and no permute launch is needed.
+  cudaError_t e = cudaSuccess;
+  if (!slab_counts) {
+    e = run_kernel(KIND_PERMUTE, st, [&] {
+      if (mv::permute_uses_sort(T, s.k))
+        return mv::launch_permute_sorted(idx, T, s.E, s.k, ws.counts, ws.offsets, ws.perm, ws.inv, x, s.H, ws.x_perm,
+                                         ws.sort, st);
+      return mv::launch_permute(idx, T, s.E, s.k, ws.counts, ws.offsets, ws.perm, ws.inv, x, s.H, ws.x_perm, st);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "expert_permute launch");
+  }
+  MV_TRY(moe_gemm_impl(x, T, s, w, ws, err, sched, st, slab_counts));
   if (!do_combine) return MV_OK;
+  const int32_t* inv = slab_counts ? slab_inv : ws.inv;
   e = run_kernel(KIND_COMBINE, st, [&] {
-    return mv::launch_combine(ws.y_perm, s.I_shared > 0 ? ws.y_sh : nullptr, ws.inv, tw, res, out, T, s.H, s.k,
-                              err, combine_pf, st);
+    return mv::launch_combine(ws.y_perm, s.I_shared > 0 ? ws.y_sh : nullptr, inv, tw, res, out, T, s.H, s.k,
+                              static_cast<int>(ws.n_pos), err, combine_pf, st);
   });
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   return MV_OK;
@@ -768,7 +795,7 @@ size_t verify_step_workspace_size(int32_t B, int32_t K, const mv_moe_shape* shap
   c.take<float>(static_cast<size_t>(T) * shape->k * 2);
   c.take<uint64_t>(static_cast<size_t>(lm_parts_alloc(V)) * T);
   c.take<char>(kSchedBytes * (kMaxLayers + 1));
-  carve_ffn(c, T, *shape);
+  carve_ffn(c, T, *shape, use_slabs(T, *shape));
   return kHeader + c.off + 1024;
 }
 
@@ -808,17 +835,46 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
   float* tw_buf = c.take<float>(tk * 2);
   uint64_t* parts = c.take<uint64_t>(static_cast<size_t>(lm_parts_alloc(V)) * T);
   int* sched = c.take<int>(static_cast<size_t>(mv::kSchedInts) * (kMaxLayers + 1));
-  FfnWs fw = carve_ffn(c, T, *shape);
+  const bool slabs = use_slabs(T, *shape);
+  FfnWs fw = carve_ffn(c, T, *shape, slabs);
   cudaError_t e0 = cudaMemsetAsync(sched, 0, kSchedBytes * (n_layers + 1), st);
   if (e0 != cudaSuccess) return cuda_fail(e0, "clearing the scheduling state");
+  auto slab_counts = [&](int l) -> int32_t* {
+    return slabs ? sched + static_cast<size_t>(l) * mv::kSchedInts + kSlabCountOff : nullptr;
+  };
+  auto slab_inv = [&](int l) -> int32_t* { return slabs ? ((l & 1) ? fw.inv_alt : fw.inv) : nullptr; };
 
   // Layer l's combine runs fused with layer l+1's routing (combine_route) when
   // the batch is decode-sized; otherwise as its own kernel before the router.
+  // Decode-sized batches also group the routed rows by expert in that kernel
+  // (slab layout) instead of a permute launch.
   const bool fused = mv::combine_route_supported(static_cast<int>(T), shape->H, shape->E);
   const uint16_t* h = hidden;
-  if (n_layers > 0)
+  if (n_layers > 0 && slabs) {
+    cudaError_t e = run_kernel(KIND_ROUTER, st, [&] {
+      mv::CombineRouteArgs a{};
+      a.x = h;
+      a.T = static_cast<int>(T);
+      a.H = shape->H;
+      a.E = shape->E;
+      a.k = shape->k;
+      a.wr = layers[0].w_router;
+      a.bias = layers[0].router_bias;
+      a.idx = idx_buf;
+      a.w = tw_buf;
+      a.err = err;
+      a.pf = moe_first_wave(*shape, layers[0], kPrefetchBudget);
+      a.slab_counts = slab_counts(0);
+      a.inv_out = slab_inv(0);
+      a.x_slab = fw.x_perm;
+      a.slab_rows = static_cast<int>(T);
+      return mv::launch_combine_route(a, st);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "router_topk launch");
+  } else if (n_layers > 0) {
     MV_TRY(route_impl(h, static_cast<int>(T), *shape, layers[0].w_router, layers[0].router_bias, idx_buf, tw_buf, err,
                       st, moe_first_wave(*shape, layers[0], kPrefetchBudget)));
+  }
   for (int l = 0; l < n_layers; ++l) {
     const mv_moe_weights& w = layers[l];
     int32_t* idx = idx_buf + (l & 1) * tk;
@@ -827,7 +883,8 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
     const bool last = (l + 1 == n_layers);
     MV_TRY(ffn_forward_impl(h, static_cast<int>(T), *shape, w, idx, tw, h, next, fw, err,
                             sched + static_cast<size_t>(l) * mv::kSchedInts, st, last || !fused,
-                            last ? lm_first_wave(w_lm, V, shape->H, kPrefetchBudget) : mv::L2Prefetch{}));
+                            last ? lm_first_wave(w_lm, V, shape->H, kPrefetchBudget) : mv::L2Prefetch{},
+                            slab_counts(l), slab_inv(l)));
     if (!last) {
       int32_t* idx_n = idx_buf + ((l + 1) & 1) * tk;
       float* tw_n = tw_buf + ((l + 1) & 1) * tk;
@@ -838,7 +895,8 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
           a.x = h;
           a.y_perm = fw.y_perm;
           a.y_sh = shape->I_shared > 0 ? fw.y_sh : nullptr;
-          a.inv = fw.inv;
+          a.inv = slabs ? slab_inv(l) : fw.inv;
+          a.n_pos = static_cast<int>(fw.n_pos);
           a.w_prev = tw;
           a.k_prev = shape->k;
           a.out = next;
@@ -852,6 +910,10 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
           a.w = tw_n;
           a.err = err;
           a.pf = moe_first_wave(*shape, wn, kPrefetchBudget);
+          a.slab_counts = slab_counts(l + 1);
+          a.inv_out = slab_inv(l + 1);
+          a.x_slab = fw.x_perm;
+          a.slab_rows = static_cast<int>(T);
           return mv::launch_combine_route(a, st);
         });
         if (e != cudaSuccess) return cuda_fail(e, "combine_route launch");

@@ -33,6 +33,7 @@ constexpr int kErrInternal = 2;
 // Ints of scheduling state one grouped-GEMM launch uses (claim counter plus one
 // completion counter per group); zeroed before the launch.
 constexpr int kSchedInts = 1024;
+constexpr int kMaxGroups = 2 * 256 + 8;  // routed + shared groups of both phases
 
 // One operand set of the grouped GEMM: `groups` groups that share tensor maps.
 // Group gi multiplies A rows [gi*a_group_stride, +M) by the B rows
@@ -45,7 +46,8 @@ struct GemmSet {
   CUtensorMap b;           // B operand, box of 16 rows x 64 columns
   void* out;
   const int32_t* counts;   // device [groups] or nullptr (static_rows)
-  const int32_t* offsets;  // device [groups] or nullptr (0)
+  const int32_t* offsets;  // device [groups], or nullptr: group g starts at row g * slab_rows
+  int32_t slab_rows;       // rows reserved per group when offsets is nullptr (0: one group at row 0)
   int32_t ld_out;
   int32_t K;               // reduction length, multiple of 64
   int32_t M;               // valid A rows per group

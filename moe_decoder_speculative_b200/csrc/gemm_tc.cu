@@ -52,7 +52,6 @@ namespace mv {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kMaxGroups = 2 * 256 + 8;   // routed + shared groups of both phases
 constexpr int kATileBytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kRing = 4;                // claimed units in flight inside a CTA
 
@@ -140,9 +139,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     while (g >= set_base[s + 1]) ++s;
     const int gi = g - set_base[s];
     const GemmSet& S = p.set[s];
-    const int rows = S.counts ? S.counts[gi] : S.static_rows;
+    int rows = S.counts ? S.counts[gi] : S.static_rows;
+    if (S.slab_rows > 0 && rows > S.slab_rows) rows = S.slab_rows;  // a slab never holds more
     g_rows[g] = rows;
-    g_row0[g] = S.offsets ? S.offsets[gi] : 0;
+    g_row0[g] = S.offsets ? S.offsets[gi] : gi * S.slab_rows;
     g_set[g] = static_cast<unsigned char>(s);
     g_gi[g] = static_cast<short>(gi);
     const int mt = (S.M + S.m_tile - 1) / S.m_tile;

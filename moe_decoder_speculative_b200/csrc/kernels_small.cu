@@ -58,7 +58,7 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
 // of a warp argmax (larger logit wins, equal logits -> lower expert id), then
 // the renormalised softmax weights exp(l_j - l_max) / sum_selected.
 __device__ __forceinline__ void topk_select_row(const float* lrow, int E, int k, int lane,
-                                                int32_t* idx_out, float* w_out) {
+                                                int32_t* idx_out, float* w_out, int32_t* sel_s = nullptr) {
   constexpr int kMaxPer = 8;  // E <= 256
   float v[kMaxPer];
   const int per = (E + 31) / 32;
@@ -108,6 +108,7 @@ __device__ __forceinline__ void topk_select_row(const float* lrow, int E, int k,
       }
     idx_out[lane] = my_e;
     w_out[lane] = expf(my_v - mx) / s;
+    if (sel_s) sel_s[lane] = my_e;
   }
 }
 
@@ -338,7 +339,13 @@ cudaError_t launch_router(const uint16_t* x, int T, int H, int E, int k, const u
 //      (+ bias) in fp32, warp w owning experts w, w+8, ...; the router rows
 //      stream from L2 four experts at a time, all loads of a batch issued
 //      before any is used (NV 16-byte vectors per lane per expert row);
-//  (3) top-k with renormalised softmax weights, one warp per row.
+//  (3) top-k with renormalised softmax weights, one warp per row;
+//  (4) with slab_counts: the grouping by expert of the next layer, done here
+//      instead of by a separate permute launch.  Each routed entry claims the
+//      next free row of its expert's slab (an atomic counter per expert) and
+//      the CTA copies its rows there from shared memory.  A claim past the
+//      slab's capacity (only possible for rows whose logits are all -inf or
+//      NaN) is undone, reported as an internal error and its entry skipped.
 // ---------------------------------------------------------------------------
 template <int R, int NV>
 __global__ void __launch_bounds__(512) combine_route_kernel(
@@ -346,8 +353,11 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
     const int32_t* __restrict__ inv, const float* __restrict__ w_prev, int k_prev, int n_pos,
     uint16_t* __restrict__ out, int T, int H, int E, int k, const uint16_t* __restrict__ wr,
     const float* __restrict__ bias, int32_t* __restrict__ idx, float* __restrict__ wout, int* err,
-    const L2Prefetch pf) {
+    const L2Prefetch pf, int32_t* __restrict__ slab_counts, int32_t* __restrict__ inv_out,
+    uint16_t* __restrict__ x_slab, int slab_rows) {
   extern __shared__ __align__(16) uint8_t sm[];
+  __shared__ int32_t sel_s[R * 8];  // the experts each row selected
+  __shared__ int32_t pos_s[R * 8];  // their slab rows (-1: skipped)
   uint16_t* hs = reinterpret_cast<uint16_t*>(sm);                         // [R][H]
   float* ls = reinterpret_cast<float*>(hs + static_cast<size_t>(R) * H);  // [R][E]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -485,7 +495,36 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
   // (3) top-k
   if (warp < nrows)
     topk_select_row(ls + warp * E, E, k, lane, idx + static_cast<size_t>(row0 + warp) * k,
-                    wout + static_cast<size_t>(row0 + warp) * k);
+                    wout + static_cast<size_t>(row0 + warp) * k, slab_counts ? sel_s + warp * 8 : nullptr);
+  if (!slab_counts) return;  // uniform across the CTA
+
+  // (4) slab placement of the routed rows
+  __syncthreads();
+  if (tid < nrows * k) {
+    const int r = tid / k, j = tid % k;
+    const int e = sel_s[r * 8 + j];
+    int p = -1;
+    if (e >= 0 && e < E) {
+      const int c = atomicAdd(&slab_counts[e], 1);
+      if (c < slab_rows) {
+        p = e * slab_rows + c;
+      } else {
+        atomicSub(&slab_counts[e], 1);
+      }
+    }
+    if (p < 0 && err) atomicOr(err, kErrInternal);
+    pos_s[r * 8 + j] = p;
+    inv_out[static_cast<size_t>(row0 + r) * k + j] = p;
+  }
+  __syncthreads();
+  for (int i = tid; i < nrows * k * hv; i += blockDim.x) {
+    const int q = i / hv, c = i % hv;
+    const int r = q / k, j = q % k;
+    const int p = pos_s[r * 8 + j];
+    if (p >= 0)
+      reinterpret_cast<uint4*>(x_slab + static_cast<size_t>(p) * H)[c] =
+          reinterpret_cast<const uint4*>(hs + static_cast<size_t>(r) * H)[c];
+  }
 }
 
 template <int R, int NV>
@@ -494,7 +533,8 @@ static cudaError_t launch_combine_route_rv(const CombineRouteArgs& a, cudaStream
   const int rows_ctas = (a.T + R - 1) / R;
   const int grid = rows_ctas > prefetch_ctas(a.pf) ? rows_ctas : prefetch_ctas(a.pf);  // extra CTAs only prefetch
   return launch_pdl(combine_route_kernel<R, NV>, dim3(grid), dim3(512), smem, s, a.x, a.y_perm, a.y_sh, a.inv,
-             a.w_prev, a.k_prev, a.T * a.k_prev, a.out, a.T, a.H, a.E, a.k, a.wr, a.bias, a.idx, a.w, a.err, a.pf);
+                    a.w_prev, a.k_prev, a.n_pos > 0 ? a.n_pos : a.T * a.k_prev, a.out, a.T, a.H, a.E, a.k, a.wr,
+                    a.bias, a.idx, a.w, a.err, a.pf, a.slab_counts, a.inv_out, a.x_slab, a.slab_rows);
 }
 
 // Larger batches route with the shared-memory-staged router instead (each of
@@ -870,13 +910,13 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t* inv,
                            const float* w, const uint16_t* res, uint16_t* out, int T, int H,
-                           int k, int* err, const L2Prefetch& pf, cudaStream_t s) {
+                           int k, int n_pos, int* err, const L2Prefetch& pf, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   const long long total = static_cast<long long>(T) * (H / 8);
   const long long blocks = (total + 255) / 256;
   int grid = static_cast<int>(blocks < 148LL * 8 ? blocks : 148LL * 8);
   if (grid < prefetch_ctas(pf)) grid = prefetch_ctas(pf);  // the grid-stride loop leaves the extra CTAs idle
-  return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, s, y_perm, y_sh, inv, w, res, out, T, H, k, T * k, err,
+  return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, s, y_perm, y_sh, inv, w, res, out, T, H, k, n_pos, err,
                     pf);
 }
 

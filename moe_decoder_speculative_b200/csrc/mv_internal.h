@@ -66,6 +66,17 @@ struct CombineRouteArgs {
   float* w;
   int* err;
   L2Prefetch pf;
+  int n_pos;                // entries of y_perm (positions valid in inv); 0: T * k_prev
+  // Grouping by expert fused into the routing (slab layout), or nullptr: each
+  // routed entry (row r, slot j -> expert e) takes the next free row of expert
+  // e's slab of slab_rows rows: p = e * slab_rows + atomicAdd(&slab_counts[e], 1),
+  // x_slab[p] = the routed row, inv_out[r * k + j] = p.  slab_counts must be
+  // zero at launch.  Rows land in a slab in any order; every consumer reads
+  // them through slab_counts and inv_out, and no result depends on the order.
+  int32_t* slab_counts;
+  int32_t* inv_out;
+  uint16_t* x_slab;
+  int slab_rows;
 };
 bool combine_route_supported(int T, int H, int E);
 cudaError_t launch_combine_route(const CombineRouteArgs& a, cudaStream_t s);
@@ -80,9 +91,10 @@ size_t sort_scratch_ints(int T, int E, int k);
 cudaError_t launch_permute_sorted(const int32_t* idx, int T, int E, int k, int32_t* counts, int32_t* offsets,
                                   int32_t* perm, int32_t* inv, const uint16_t* x, int H, uint16_t* x_perm,
                                   int32_t* scratch, cudaStream_t s);
+// n_pos: the number of y_perm rows (positions in inv are checked against it).
 cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t* inv,
                            const float* w, const uint16_t* res, uint16_t* out, int T, int H,
-                           int k, int* err, const L2Prefetch& pf, cudaStream_t s);
+                           int k, int n_pos, int* err, const L2Prefetch& pf, cudaStream_t s);
 cudaError_t launch_lm_finalize(const uint64_t* keys, int nparts, int ld, int T, int32_t* argmax,
                                cudaStream_t s);
 cudaError_t launch_accept(const int32_t* argmax, const int32_t* drafts, int B, int K,
