@@ -33,7 +33,7 @@ import numpy as np
 __all__ = [
     "Workload", "WORKLOADS", "workload", "f32_to_bf16_bits", "bf16_bits_to_f32",
     "normal_bf16", "make_layer", "make_hidden", "make_lm_head", "make_inputs",
-    "make_drafts", "hot_experts", "router_bias",
+    "make_drafts", "hot_experts", "router_bias", "make_draft_block",
 ]
 
 
@@ -143,9 +143,10 @@ def normal_bf16(ss: np.random.SeedSequence, shape, std: float) -> np.ndarray:
 
 
 def _tree(wid: int):
-    """Fixed seed tree: root(seed=workload id) -> [hidden, layers, lm_head, drafts, hot, ties]."""
+    """Fixed seed tree: root(seed=workload id) -> [hidden, layers, lm_head, drafts, hot, ties,
+    draft_block].  (Child i does not depend on how many siblings are spawned.)"""
     root = np.random.SeedSequence(int(wid))
-    return root.spawn(6)
+    return root.spawn(7)
 
 
 def make_layer(w: Workload, layer_ss: np.random.SeedSequence) -> dict:
@@ -168,6 +169,29 @@ def make_layer(w: Workload, layer_ss: np.random.SeedSequence) -> dict:
 
 def make_hidden(w: Workload) -> np.ndarray:
     return normal_bf16(_tree(w.id)[0], (w.T, w.H), w.x_std)
+
+
+def make_draft_block(w: Workload, I_d: int | None = None) -> dict:
+    """Synthetic weights of the FastMTP draft block, bf16 bits: token embedding
+    w_emb [V][H] ~ N(0, 1); RMSNorm gains g_hidden, g_embed [H] ~ 1 + N(0, 0.1^2);
+    projection w_proj [H][2H] and a dense SwiGLU FFN (w_gate, w_up [I_d][H],
+    w_down [H][I_d]) ~ N(0, w_std^2).  I_d defaults to the shared expert's
+    width I_sh."""
+    s = _tree(w.id)[6].spawn(7)
+    H, Id = w.H, (I_d or w.I_sh)
+
+    def gain(ss):
+        return f32_to_bf16_bits(1.0 + bf16_bits_to_f32(normal_bf16(ss, (H,), 0.1)))
+
+    return {
+        "w_emb": normal_bf16(s[0], (w.V, H), 1.0),
+        "g_hidden": gain(s[1]),
+        "g_embed": gain(s[2]),
+        "w_proj": normal_bf16(s[3], (H, 2 * H), w.w_std),
+        "w_gate": normal_bf16(s[4], (Id, H), w.w_std),
+        "w_up": normal_bf16(s[5], (Id, H), w.w_std),
+        "w_down": normal_bf16(s[6], (H, Id), w.w_std),
+    }
 
 
 def make_lm_head(w: Workload) -> np.ndarray | None:

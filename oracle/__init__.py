@@ -54,8 +54,12 @@ def _load():
             lib.oracle_swiglu.argtypes = [P, i, i, P, P, P, P, P, i]
             lib.oracle_lm_head_argmax.argtypes = [P, i, i, P, i, P, P, P, i, i]
             lib.oracle_greedy_accept.argtypes = [P, P, i, i, P, P, P]
+            f32 = ctypes.c_float
+            lib.oracle_rmsnorm.argtypes = [P, i, i, P, f32, P, i]
+            lib.oracle_fastmtp_draft.argtypes = [P, P, i, i, i, i, i, P, P, P, P, P, P, P, P, f32, P, P, P, i, i]
             for f in ("oracle_router", "oracle_moe_ffn", "oracle_swiglu",
-                      "oracle_lm_head_argmax", "oracle_greedy_accept", "oracle_num_threads"):
+                      "oracle_lm_head_argmax", "oracle_greedy_accept", "oracle_num_threads",
+                      "oracle_rmsnorm", "oracle_fastmtp_draft"):
                 getattr(lib, f).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -195,4 +199,61 @@ def verify_step(hidden, drafts, B, K, layers, k, w_lm, acc_double=False, n_threa
     am, zmax, lm_gap = lm_head_argmax(st["h"], w_lm, acc_double=acc_double, n_threads=n_threads)
     acc, nxt, em = greedy_accept(am, drafts, B, K)
     st.update(argmax=am, zmax=zmax, lm_gap=lm_gap, accepted=acc, next_token=nxt, emitted=em)
+    return st
+
+
+RMS_EPS = 1e-6   # RMSNorm epsilon of the draft block (a reading; the pages give none)
+
+DRAFT_KEYS = ("w_emb", "g_hidden", "g_embed", "w_proj", "w_gate", "w_up", "w_down")
+
+
+def rmsnorm(x, gain, eps=RMS_EPS, acc_double=False):
+    """RMSNorm of every row of x [T][n] (bf16 bits): bf16((x * r) * gain),
+    r = 1 / sqrt(mean(x^2) + eps).  Returns bf16 bits [T][n]."""
+    x = _u16(np.atleast_2d(x))
+    T, n = x.shape
+    g = _u16(gain)
+    out = np.zeros_like(x)
+    rc = _load().oracle_rmsnorm(_p(x), T, n, _p(g), float(eps), _p(out), int(acc_double))
+    if rc:
+        raise ValueError("oracle_rmsnorm: invalid arguments")
+    return out
+
+
+def fastmtp_draft(h0, t0, K, draft, w_lm, eps=RMS_EPS, acc_double=False, n_threads=0):
+    """K recursive steps of the FastMTP draft block from the verifier's last
+    hidden state h0 [B][H] and next token t0 [B].  ``draft`` holds the block's
+    weights (DRAFT_KEYS: w_emb [V][H], g_hidden [H], g_embed [H],
+    w_proj [H][2H], w_gate [I_d][H], w_up [I_d][H], w_down [H][I_d], bf16 bits).
+    Returns {"drafts" int32 [B][K], "h_steps" bf16 [K][B][H], "gaps" fp32 [K][B]}."""
+    h0 = _u16(h0)
+    B, H = h0.shape
+    t0 = np.ascontiguousarray(t0, np.int32)
+    w = {k: _u16(draft[k]) for k in DRAFT_KEYS}
+    w_lm = _u16(w_lm)
+    V = w_lm.shape[0]
+    Id = w["w_gate"].shape[0]
+    drafts = np.zeros((B, K), np.int32)
+    h_steps = np.zeros((K, B, H), np.uint16)
+    gaps = np.zeros((K, B), np.float32)
+    rc = _load().oracle_fastmtp_draft(_p(h0), _p(t0), B, int(K), H, Id, V, *[_p(w[k]) for k in DRAFT_KEYS],
+                                      _p(w_lm), float(eps), _p(drafts), _p(h_steps), _p(gaps),
+                                      int(acc_double), int(n_threads))
+    if rc:
+        raise ValueError("oracle_fastmtp_draft: invalid arguments")
+    return {"drafts": drafts, "h_steps": h_steps, "gaps": gaps}
+
+
+def speculative_step(hidden, drafts, B, K, layers, k, w_lm, draft, eps=RMS_EPS, acc_double=False,
+                     n_threads=0):
+    """One iteration of the draft-and-verify loop: verify_step on the rows,
+    then the draft block from the verifier's final hidden state at each
+    sequence's last kept row (row b*(K+1) + accepted[b]) and its next token,
+    giving the K drafts of the next iteration."""
+    st = verify_step(hidden, drafts, B, K, layers, k, w_lm, acc_double=acc_double, n_threads=n_threads)
+    rows = np.arange(B) * (K + 1) + st["accepted"]
+    h0 = st["h"][rows]
+    nxt = fastmtp_draft(h0, st["next_token"], K, draft, w_lm, eps=eps, acc_double=acc_double,
+                        n_threads=n_threads)
+    st.update(draft_h0=h0, next_drafts=nxt["drafts"], draft_h_steps=nxt["h_steps"], draft_gaps=nxt["gaps"])
     return st

@@ -16,6 +16,10 @@
 //     decoding; the verifier commits up to K+1 tokens per pass.
 //   * tldrocket write-up ("Jina AI Releases jina-ocr-v1 ..."), speculative
 //     paragraph: the decoder keeps only the drafts that match its own choice.
+//   * model card, decoding-speed paragraph, and the write-up's speculative
+//     paragraph: the drafts come from FastMTP, one dense draft block applied
+//     recursively for K steps (not K separate heads).  The pages give the
+//     block no shape; the reading taken is in fastmtp_draft_row below.
 // The pages give no formulas; the readings taken where they are silent are:
 //   gating = softmax over the E routed logits, keep the top k (selected on the
 //   logits, ties to the lower expert id, slots in descending-logit order), then
@@ -190,6 +194,46 @@ void lm_row(const uint16_t* h, int H, const uint16_t* w_lm, int V, int32_t* am, 
   if (gap) gap[0] = (V > 1) ? static_cast<float>(bz - second) : std::numeric_limits<float>::infinity();
 }
 
+// RMSNorm of one row: out_i = bf16((x_i * r) * gain_i) with
+// r = 1 / sqrt(sum_i x_i^2 / n + eps), the sum in Acc in ascending order.
+template <class Acc>
+void rmsnorm_row(const uint16_t* x, int n, const uint16_t* gain, float eps, uint16_t* out) {
+  Acc ss = 0;
+  for (int i = 0; i < n; ++i) {
+    const Acc v = static_cast<Acc>(bf16_to_float(x[i]));
+    ss += v * v;
+  }
+  const Acc r = static_cast<Acc>(1) / std::sqrt(ss / static_cast<Acc>(n) + static_cast<Acc>(eps));
+  for (int i = 0; i < n; ++i)
+    out[i] = float_to_bf16(static_cast<float>((static_cast<Acc>(bf16_to_float(x[i])) * r) *
+                                              static_cast<Acc>(bf16_to_float(gain[i]))));
+}
+
+// One step of the FastMTP draft block on one row (the reading of "a single
+// dense draft block applied recursively"): the block takes the previous
+// hidden state h (the verifier's last hidden state at the first step, the
+// block's own output after that) and the token t drafted last (the verifier's
+// next token at the first step), and returns the next hidden state:
+//   u  = [ RMSNorm(h) * g_h ; RMSNorm(E[t]) * g_e ]      (2H, bf16)
+//   z  = bf16(u . W_proj^T)                              (W_proj [H][2H])
+//   h' = bf16(z + SwiGLU(z))                             (dense, intermediate I_d)
+// and the draft is the shared LM head's greedy choice on h'.
+template <class Acc>
+void draft_step_row(const uint16_t* h, int32_t t, int H, int Id, const uint16_t* w_emb,
+                    const uint16_t* g_h, const uint16_t* g_e, const uint16_t* w_proj,
+                    const uint16_t* wg, const uint16_t* wu, const uint16_t* wd, float eps,
+                    uint16_t* h_out) {
+  std::vector<uint16_t> u(2 * static_cast<size_t>(H)), z(H), a(Id);
+  rmsnorm_row<Acc>(h, H, g_h, eps, u.data());
+  rmsnorm_row<Acc>(w_emb + static_cast<size_t>(t) * H, H, g_e, eps, u.data() + H);
+  for (int i = 0; i < H; ++i)
+    z[i] = float_to_bf16(static_cast<float>(dot_bf16<Acc>(u.data(), w_proj + static_cast<size_t>(i) * 2 * H, 2 * H)));
+  std::vector<Acc> y(H);
+  swiglu_row<Acc>(z.data(), H, Id, wg, wu, wd, a.data(), y.data());
+  for (int i = 0; i < H; ++i)
+    h_out[i] = float_to_bf16(static_cast<float>(static_cast<Acc>(bf16_to_float(z[i])) + y[i]));
+}
+
 void set_threads(int n_threads) {
 #ifdef _OPENMP
   if (n_threads > 0) omp_set_num_threads(n_threads);
@@ -303,6 +347,59 @@ int oracle_greedy_accept(const int32_t* argmax, const int32_t* drafts, int B, in
     next_token[b] = g[a];
     if (emitted) {
       for (int j = 0; j <= K; ++j) emitted[static_cast<size_t>(b) * (K + 1) + j] = (j <= a) ? g[j] : -1;
+    }
+  }
+  return 0;
+}
+
+// RMSNorm of T rows of n values (see rmsnorm_row).
+int oracle_rmsnorm(const uint16_t* x, int T, int n, const uint16_t* gain, float eps, uint16_t* out,
+                   int acc_double) {
+  if (!x || !gain || !out || T < 0 || n <= 0 || !(eps >= 0.f)) return 1;
+  for (int r = 0; r < T; ++r) {
+    const size_t o = static_cast<size_t>(r) * n;
+    if (acc_double)
+      rmsnorm_row<double>(x + o, n, gain, eps, out + o);
+    else
+      rmsnorm_row<float>(x + o, n, gain, eps, out + o);
+  }
+  return 0;
+}
+
+// FastMTP drafting: K recursive steps of the draft block (draft_step_row) per
+// sequence, starting from h0[b] and t0[b]; drafts[b][j] = the LM head's greedy
+// choice on the j-th step's output.  h_steps[j][b][H] (nullable) receives the
+// step outputs, gaps[j][b] (nullable) the LM top-2 gap of each step.
+int oracle_fastmtp_draft(const uint16_t* h0, const int32_t* t0, int B, int K, int H, int Id, int V,
+                         const uint16_t* w_emb, const uint16_t* g_h, const uint16_t* g_e,
+                         const uint16_t* w_proj, const uint16_t* wg, const uint16_t* wu,
+                         const uint16_t* wd, const uint16_t* w_lm, float eps, int32_t* drafts,
+                         uint16_t* h_steps, float* gaps, int acc_double, int n_threads) {
+  if (!h0 || !t0 || !w_emb || !g_h || !g_e || !w_proj || !wg || !wu || !wd || !w_lm || B < 0 ||
+      K < 0 || H <= 0 || Id <= 0 || V <= 0 || !(eps >= 0.f) || (K > 0 && B > 0 && !drafts))
+    return 1;
+  for (int b = 0; b < B; ++b)
+    if (t0[b] < 0 || t0[b] >= V) return 1;
+  set_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int b = 0; b < B; ++b) {
+    std::vector<uint16_t> h(h0 + static_cast<size_t>(b) * H, h0 + static_cast<size_t>(b + 1) * H), hn(H);
+    int32_t t = t0[b];
+    for (int j = 0; j < K; ++j) {
+      int32_t d = 0;
+      float gp = 0.f;
+      if (acc_double) {
+        draft_step_row<double>(h.data(), t, H, Id, w_emb, g_h, g_e, w_proj, wg, wu, wd, eps, hn.data());
+        lm_row<double>(hn.data(), H, w_lm, V, &d, nullptr, &gp);
+      } else {
+        draft_step_row<float>(h.data(), t, H, Id, w_emb, g_h, g_e, w_proj, wg, wu, wd, eps, hn.data());
+        lm_row<float>(hn.data(), H, w_lm, V, &d, nullptr, &gp);
+      }
+      drafts[static_cast<size_t>(b) * K + j] = d;
+      if (h_steps) std::copy(hn.begin(), hn.end(), h_steps + (static_cast<size_t>(j) * B + b) * H);
+      if (gaps) gaps[static_cast<size_t>(j) * B + b] = gp;
+      h.swap(hn);
+      t = d;
     }
   }
   return 0;
