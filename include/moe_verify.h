@@ -222,6 +222,66 @@ MV_API mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int3
                       size_t ws_bytes, mv_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * FastMTP draft block (jina-ocr-v1 model card, decoding-speed paragraph, and
+ * the tldrocket write-up's speculative paragraph: the drafts come from one
+ * dense draft block applied recursively for K steps, not K separate heads).
+ * The pages give the block no shape; this library's reading is:
+ *   u_j  = [ RMSNorm(h_{j-1}) * g_hidden ; RMSNorm(w_emb[t_{j-1}]) * g_embed ]
+ *   z_j  = bf16(u_j . w_proj^T)                      w_proj [H][2H]
+ *   h_j  = bf16(z_j + SwiGLU(z_j))                   dense, intermediate I_d
+ *   t_j  = argmax_v h_j . w_lm[v]  (the verifier's LM head; ties to lower v)
+ * for j = 1..K, from h_0 = the verifier's last hidden state and t_0 = the
+ * verifier's next token; drafts = t_1..t_K.  RMSNorm(x) = x / sqrt(mean(x^2)
+ * + 1e-6) in fp32; u, z and the SwiGLU activation are rounded to bf16 (they
+ * feed bf16 MMAs).
+ * All weights are bf16 device pointers, row-major, 16-byte aligned:
+ *   w_emb [V][H], g_hidden [H], g_embed [H], w_proj [H][2H],
+ *   w_gate [I_d][H], w_up [I_d][H], w_down [H][I_d];  I_d a multiple of 64.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  const uint16_t* w_emb;
+  const uint16_t* g_hidden;
+  const uint16_t* g_embed;
+  const uint16_t* w_proj;
+  const uint16_t* w_gate;
+  const uint16_t* w_up;
+  const uint16_t* w_down;
+  int32_t I_d;
+} mv_draft_weights;
+
+/* Bytes of workspace fastmtp_draft needs. */
+MV_API size_t fastmtp_draft_workspace_size(int32_t B, int32_t K, int32_t H, int32_t I_d, int32_t V);
+
+/* fastmtp_draft - K recursive draft-block steps for B sequences.
+ *   h0 [B][H] bf16 (the verifier's last hidden state of each sequence),
+ *   t0 [B] int32 (its next token, in [0, V); another value is reported as
+ *   MV_ERR_INTERNAL by mv_sync_status and drafts from embedding row 0),
+ *   w_lm [V][H] bf16 (the verifier's LM head), drafts [B][K] int32 output,
+ *   h_steps [K][B][H] bf16 output of every step (nullable).
+ * Asynchronous on `stream`; device-side errors land in the workspace's sticky
+ * word (mv_sync_status).  K = 0 or B = 0 launches nothing. */
+MV_API mv_status fastmtp_draft(const uint16_t* h0, const int32_t* t0, int32_t B, int32_t K, int32_t H,
+                               const mv_draft_weights* draft, const uint16_t* w_lm, int32_t V,
+                               int32_t* drafts, uint16_t* h_steps, void* ws, size_t ws_bytes,
+                               mv_stream_t stream);
+
+/* Bytes of workspace speculative_step needs. */
+MV_API size_t speculative_step_workspace_size(int32_t B, int32_t K, const mv_moe_shape* shape, int32_t I_d,
+                                              int32_t V);
+
+/* speculative_step - one iteration of the draft-and-verify loop on the GPU:
+ * verify_step (same arguments and outputs), then fastmtp_draft from the
+ * verifier's final hidden state at each sequence's last kept row
+ * (row b*(K+1) + accepted[b] of h_L) and its next token, writing the K
+ * drafts the next iteration verifies to next_drafts [B][K] (may not alias
+ * drafts).  One stream of launches, no host synchronisation. */
+MV_API mv_status speculative_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, int32_t K,
+                                  const mv_moe_shape* shape, const mv_moe_weights* layers, int32_t n_layers,
+                                  const uint16_t* w_lm, int32_t V, const mv_draft_weights* draft,
+                                  int32_t* accepted, int32_t* next_token, int32_t* emitted, int32_t* argmax,
+                                  int32_t* next_drafts, void* ws, size_t ws_bytes, mv_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * verify_graph_* - verify_step recorded once into a CUDA graph and replayed.
  * The model card's decoding-speed paragraph reports that replaying the
  * decoder as CUDA graphs changes which draft count K is fastest at batch 1,

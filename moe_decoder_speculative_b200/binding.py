@@ -25,7 +25,8 @@ EXPORTED = ["moe_router_topk", "moe_expert_permute", "moe_ffn_workspace_size", "
             "verify_step", "mv_workspace_init", "mv_sync_status", "mv_last_error", "mv_version",
             "mv_launch_count", "mv_profile_enable", "mv_profile_collect", "mv_kernel_name",
             "mv_set_wait_timeout_ns", "lm_head_argmax_noalloc", "verify_graph_create", "verify_graph_launch",
-            "verify_graph_kernels", "verify_graph_destroy"]
+            "verify_graph_kernels", "verify_graph_destroy", "fastmtp_draft_workspace_size", "fastmtp_draft",
+            "speculative_step_workspace_size", "speculative_step"]
 
 
 class MVError(RuntimeError):
@@ -42,6 +43,13 @@ class MoeShape(ctypes.Structure):
 class MoeWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("w_router", "router_bias", "w_gate", "w_up", "w_down",
                                                 "ws_gate", "ws_up", "ws_down")]
+
+
+DRAFT_KEYS = ("w_emb", "g_hidden", "g_embed", "w_proj", "w_gate", "w_up", "w_down")
+
+
+class DraftWeightsC(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in DRAFT_KEYS] + [("I_d", ctypes.c_int32)]
 
 
 _lib = None
@@ -82,6 +90,11 @@ def lib():
             "verify_graph_launch": (i32, [P, P]),
             "verify_graph_kernels": (i32, [P]),
             "verify_graph_destroy": (i32, [P]),
+            "fastmtp_draft_workspace_size": (sz, [i32, i32, i32, i32, i32]),
+            "fastmtp_draft": (i32, [P, P, i32, i32, i32, ctypes.POINTER(DraftWeightsC), P, i32, P, P, P, sz, P]),
+            "speculative_step_workspace_size": (sz, [i32, i32, S, i32, i32]),
+            "speculative_step": (i32, [P, P, i32, i32, S, W, i32, P, i32, ctypes.POINTER(DraftWeightsC), P, P, P, P,
+                                       P, P, sz, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -254,6 +267,63 @@ class VerifyPlan:
                                  _p(self.accepted), _p(self.next_token), _p(self.emitted), _p(self.argmax),
                                  _p(self.ws), self.ws.numel(), _stream(stream)))
         return self.accepted, self.next_token, self.emitted, self.argmax
+
+    def sync_status(self, stream=None):
+        sync_status(self.ws, stream)
+
+
+class DraftWeights:
+    """Device copies of the FastMTP draft block's weights plus the C struct."""
+
+    def __init__(self, draft: dict, device="cuda"):
+        self.t = {n: (draft[n] if isinstance(draft[n], torch.Tensor) else bf16_to_device(draft[n], device))
+                  for n in DRAFT_KEYS}
+        self.I_d = int(self.t["w_gate"].shape[0])
+        self.c = DraftWeightsC(*[self.t[n].data_ptr() for n in DRAFT_KEYS], self.I_d)
+
+
+def fastmtp_draft(h0, t0, K: int, draft: DraftWeights, w_lm, keep_steps=False, ws=None, stream=None):
+    """K recursive draft-block steps from h0 [B][H] (bf16) and t0 [B] (int32).
+    Returns drafts int32 [B][K] (and the step outputs bf16 [K][B][H] when
+    keep_steps)."""
+    B, H = h0.shape
+    V = w_lm.shape[0]
+    drafts = torch.empty((B, K), dtype=torch.int32, device=h0.device)
+    steps = torch.empty((K, B, H), dtype=torch.bfloat16, device=h0.device) if keep_steps else None
+    if ws is None:
+        ws = workspace(int(lib().fastmtp_draft_workspace_size(B, K, H, draft.I_d, V)), h0.device)
+    _check(lib().fastmtp_draft(_p(h0), _p(t0), B, K, H, ctypes.byref(draft.c), _p(w_lm), V, _p(drafts), _p(steps),
+                               _p(ws), ws.numel(), _stream(stream)))
+    return (drafts, steps) if keep_steps else drafts
+
+
+class SpeculativePlan:
+    """speculative_step: verify_step, then the draft block from the verifier's
+    state, giving the next iteration's drafts -- one loop iteration on the GPU."""
+
+    def __init__(self, shape: MoeShape, layers: list, w_lm, draft: DraftWeights, B: int, K: int, device="cuda"):
+        self.shape, self.layers, self.w_lm, self.draft, self.B, self.K = shape, layers, w_lm, draft, B, K
+        self.V = w_lm.shape[0]
+        arr = (MoeWeights * max(1, len(layers)))()
+        for i, lw in enumerate(layers):
+            arr[i] = lw.c
+        self.c_layers = arr
+        n = int(lib().speculative_step_workspace_size(B, K, ctypes.byref(shape), draft.I_d, self.V))
+        self.ws = workspace(n, device)
+        T = B * (K + 1)
+        self.accepted = torch.empty(B, dtype=torch.int32, device=device)
+        self.next_token = torch.empty(B, dtype=torch.int32, device=device)
+        self.emitted = torch.empty((B, K + 1), dtype=torch.int32, device=device)
+        self.argmax = torch.empty(T, dtype=torch.int32, device=device)
+        self.next_drafts = torch.empty((B, max(1, K)), dtype=torch.int32, device=device)
+
+    def __call__(self, hidden, drafts, stream=None):
+        _check(lib().speculative_step(_p(hidden), _p(drafts) if self.K > 0 else None, self.B, self.K,
+                                      ctypes.byref(self.shape), self.c_layers, len(self.layers), _p(self.w_lm),
+                                      self.V, ctypes.byref(self.draft.c), _p(self.accepted), _p(self.next_token),
+                                      _p(self.emitted), _p(self.argmax), _p(self.next_drafts), _p(self.ws),
+                                      self.ws.numel(), _stream(stream)))
+        return self.accepted, self.next_token, self.emitted, self.argmax, self.next_drafts
 
     def sync_status(self, stream=None):
         sync_status(self.ws, stream)

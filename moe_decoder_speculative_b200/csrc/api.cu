@@ -68,11 +68,15 @@ enum Kind {
   KIND_LM_GEMM,
   KIND_LM_FINALIZE,
   KIND_ACCEPT,
+  KIND_DRAFT_GEMM,
+  KIND_DRAFT_LM,
+  KIND_DRAFT_STEP,
   KIND_COUNT
 };
 const char* kKindNames[KIND_COUNT] = {"router_topk",       "expert_permute",     "grouped_moe_gemm",
                                       "combine_unpermute", "combine_route",      "lm_head_gemm_argmax",
-                                      "lm_argmax_finalize", "greedy_accept"};
+                                      "lm_argmax_finalize", "greedy_accept",     "draft_block_gemm",
+                                      "draft_lm_head_argmax", "draft_step"};
 
 struct ProfRec {
   int kind;
@@ -563,7 +567,8 @@ mv_status route_impl(const uint16_t* x, int T, const mv_moe_shape& s, const uint
 // lm_parts_alloc(V) slots per token.  Returns the key slots used per token
 // (the row stride of `parts` is `ld`).
 mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, int V, uint64_t* parts, int ld,
-                       int* err, int* sched, cudaStream_t st, bool balance, int* nparts_used) {
+                       int* err, int* sched, cudaStream_t st, bool balance, int* nparts_used,
+                       int kind = KIND_LM_GEMM) {
   mv::GemmParams p;
   std::memset(&p, 0, sizeof(p));
   p.err = err;
@@ -619,7 +624,7 @@ mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, in
   p.nsets = ns;
   if (used > ld) return fail(MV_ERR_INTERNAL, "LM key slots %d exceed the row stride %d", used, ld);
   *nparts_used = used;
-  cudaError_t e = run_kernel(KIND_LM_GEMM, st, [&] { return mv::launch_gemm(wide ? mv::GEMM_LM_WIDE : mv::GEMM_LM, p, gemm_grid(units), st); });
+  cudaError_t e = run_kernel(kind, st, [&] { return mv::launch_gemm(wide ? mv::GEMM_LM_WIDE : mv::GEMM_LM, p, gemm_grid(units), st); });
   if (e != cudaSuccess) return cuda_fail(e, "lm_head_gemm_argmax launch");
   return MV_OK;
 }
@@ -799,10 +804,13 @@ size_t verify_step_workspace_size(int32_t B, int32_t K, const mv_moe_shape* shap
   return kHeader + c.off + 1024;
 }
 
-mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, int32_t K, const mv_moe_shape* shape,
-                      const mv_moe_weights* layers, int32_t n_layers, const uint16_t* w_lm, int32_t V,
-                      int32_t* accepted, int32_t* next_token, int32_t* emitted, int32_t* argmax, void* ws,
-                      size_t ws_bytes, mv_stream_t stream) {
+// The verify step; *h_final (when given) receives the device address of the
+// last layer's hidden rows (inside the workspace, or `hidden` with no layers).
+static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts, int32_t B, int32_t K,
+                                  const mv_moe_shape* shape, const mv_moe_weights* layers, int32_t n_layers,
+                                  const uint16_t* w_lm, int32_t V, int32_t* accepted, int32_t* next_token,
+                                  int32_t* emitted, int32_t* argmax, void* ws, size_t ws_bytes, mv_stream_t stream,
+                                  const uint16_t** h_final) {
   MV_TRY(check_shape(shape));
   if (B < 0 || K < 0 || K > 32 || n_layers < 0 || n_layers > kMaxLayers || V <= 0)
     return fail(MV_ERR_INVALID_ARG, "bad sizes B=%d K=%d (K <= 32) n_layers=%d (<= %d) V=%d", B, K, n_layers,
@@ -923,6 +931,7 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
     }
     h = next;
   }
+  if (h_final) *h_final = h;
   int used = 0;
   MV_TRY(lm_gemm_impl(h, static_cast<int>(T), shape->H, w_lm, V, parts, lm_parts_alloc(V), err,
                       sched + static_cast<size_t>(n_layers) * mv::kSchedInts, st, true, &used));
@@ -931,6 +940,239 @@ mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, 
                                        next_token, emitted, argmax, st);
   });
   return e == cudaSuccess ? MV_OK : cuda_fail(e, "greedy_accept launch");
+}
+
+mv_status verify_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, int32_t K, const mv_moe_shape* shape,
+                      const mv_moe_weights* layers, int32_t n_layers, const uint16_t* w_lm, int32_t V,
+                      int32_t* accepted, int32_t* next_token, int32_t* emitted, int32_t* argmax, void* ws,
+                      size_t ws_bytes, mv_stream_t stream) {
+  return verify_step_impl(hidden, drafts, B, K, shape, layers, n_layers, w_lm, V, accepted, next_token, emitted,
+                          argmax, ws, ws_bytes, stream, nullptr);
+}
+
+// ---------------------------------------------------------------------------
+// FastMTP draft block
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+constexpr float kDraftRmsEps = 1e-6f;
+
+struct DraftWs {
+  int* sched;       // 2 GEMM launches per step
+  uint16_t* u;      // [B][2H] block input
+  uint16_t* z;      // [B][H] projection
+  uint16_t* a;      // [B][I_d] SwiGLU activation
+  uint16_t* h[2];   // step outputs (ping-pong) when the caller keeps none
+  uint64_t* keys;   // [B][lm_parts_alloc(V)] LM argmax keys
+};
+
+DraftWs carve_draft(Carve& c, int64_t B, int K, int H, int Id, int V) {
+  DraftWs w;
+  w.sched = c.take<int>(static_cast<size_t>(mv::kSchedInts) * 2 * std::max(K, 1));
+  w.u = c.take<uint16_t>(static_cast<size_t>(B) * 2 * H);
+  w.z = c.take<uint16_t>(static_cast<size_t>(B) * H);
+  w.a = c.take<uint16_t>(static_cast<size_t>(B) * Id);
+  w.h[0] = c.take<uint16_t>(static_cast<size_t>(B) * H);
+  w.h[1] = c.take<uint16_t>(static_cast<size_t>(B) * H);
+  w.keys = c.take<uint64_t>(static_cast<size_t>(lm_parts_alloc(V)) * B);
+  return w;
+}
+
+mv_status check_draft(const mv_draft_weights* d, int H) {
+  if (!d) return fail(MV_ERR_INVALID_ARG, "draft weights are NULL");
+  if (d->I_d <= 0 || d->I_d % 64) return fail(MV_ERR_UNSUPPORTED_SHAPE, "I_d=%d must be a positive multiple of 64", d->I_d);
+  if (H % 64) return fail(MV_ERR_UNSUPPORTED_SHAPE, "H=%d must be a multiple of 64", H);
+  MV_TRY(check_ptr(d->w_emb, "draft.w_emb"));
+  MV_TRY(check_ptr(d->g_hidden, "draft.g_hidden"));
+  MV_TRY(check_ptr(d->g_embed, "draft.g_embed"));
+  MV_TRY(check_ptr(d->w_proj, "draft.w_proj"));
+  MV_TRY(check_ptr(d->w_gate, "draft.w_gate"));
+  MV_TRY(check_ptr(d->w_up, "draft.w_up"));
+  MV_TRY(check_ptr(d->w_down, "draft.w_down"));
+  return MV_OK;
+}
+
+// One launch of the draft block's dense part for B rows, three dependent sets
+// of swap-AB tiles: z = bf16(u . W_proj^T); a = bf16(silu(z Wg^T) * (z Wu^T));
+// h' = bf16(z + a . Wd^T).  Each later set waits for the earlier one through
+// the launch's completion counters.
+mv_status draft_gemm_impl(const uint16_t* u, int B, int H, const mv_draft_weights& d, uint16_t* z, uint16_t* a,
+                          uint16_t* hout, int* err, int* sched, cudaStream_t st) {
+  mv::GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.err = err;
+  p.sched = sched;
+  p.timeout_ns = timeout_ns();
+  const int Id = d.I_d, BN = 32, bbox = mv::kDecodeBBox;
+  const int64_t ntile = (B + BN - 1) / BN;
+  mv::GemmSet& P = p.set[0];
+  P.mode = mv::MODE_KPAIR;
+  P.epi = mv::EPI_STORE_BF16;
+  P.m_tile = 128;
+  P.dep_set = -1;
+  MV_TRY(tmap(&P.a0, d.w_proj, H, 2 * static_cast<uint64_t>(H), 128));
+  P.a1 = P.a0;
+  MV_TRY(tmap(&P.b, u, B, 2 * static_cast<uint64_t>(H), bbox));
+  P.out = z;
+  P.ld_out = H;
+  P.K = 2 * H;
+  P.M = H;
+  P.groups = 1;
+  P.static_rows = B;
+  P.signal = 1;
+  mv::GemmSet& G = p.set[1];
+  G.mode = mv::MODE_GATEUP;
+  G.epi = mv::EPI_SWIGLU;
+  G.m_tile = 128;
+  G.dep_set = 0;
+  MV_TRY(tmap(&G.a0, d.w_gate, Id, H, 128));
+  MV_TRY(tmap(&G.a1, d.w_up, Id, H, 128));
+  MV_TRY(tmap(&G.b, z, B, H, bbox));
+  G.out = a;
+  G.ld_out = Id;
+  G.K = H;
+  G.M = Id;
+  G.groups = 1;
+  G.static_rows = B;
+  G.signal = 1;
+  mv::GemmSet& D = p.set[2];
+  D.mode = mv::MODE_KPAIR;
+  D.epi = mv::EPI_STORE_BF16;
+  D.m_tile = 128;
+  D.dep_set = 1;
+  MV_TRY(tmap(&D.a0, d.w_down, H, Id, 128));
+  D.a1 = D.a0;
+  MV_TRY(tmap(&D.b, a, B, Id, bbox));
+  D.out = hout;
+  D.res = z;
+  D.ld_out = H;
+  D.K = Id;
+  D.M = H;
+  D.groups = 1;
+  D.static_rows = B;
+  p.nsets = 3;
+  const int64_t units = ntile * ((H + 127) / 128 * 2 + (Id + 127) / 128);
+  cudaError_t e = run_kernel(KIND_DRAFT_GEMM, st, [&] {
+    return mv::launch_gemm(mv::GEMM_MOE_DECODE, p, gemm_grid(units), st);
+  });
+  return e == cudaSuccess ? MV_OK : cuda_fail(e, "draft_block_gemm launch");
+}
+
+// K recursive draft-block steps from h (row b*row_stride + acc[b] of h_src)
+// and t0; drafts[b][j-1] is step j's greedy choice.
+mv_status draft_impl(const uint16_t* h_src, int row_stride, const int32_t* acc, const int32_t* t0, int B, int K,
+                     int H, const mv_draft_weights& d, const uint16_t* w_lm, int V, int32_t* drafts,
+                     uint16_t* h_steps, const DraftWs& w, int* err, cudaStream_t st) {
+  if (B == 0 || K == 0) return MV_OK;
+  cudaError_t e = cudaMemsetAsync(w.sched, 0, kSchedBytes * 2 * K, st);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the draft scheduling state");
+  mv::MtpStepArgs a{};
+  a.t0 = t0;
+  a.drafts = drafts;
+  a.K = K;
+  a.w_emb = d.w_emb;
+  a.V = V;
+  a.g_h = d.g_hidden;
+  a.g_e = d.g_embed;
+  a.H = H;
+  a.eps = kDraftRmsEps;
+  a.err = err;
+  a.B = B;
+  a.j = 0;
+  a.h_src = h_src;
+  a.row_stride = row_stride;
+  a.acc = acc;
+  a.u = w.u;
+  e = run_kernel(KIND_DRAFT_STEP, st, [&] { return mv::launch_mtp_step(a, st); });
+  if (e != cudaSuccess) return cuda_fail(e, "draft_step launch");
+  const int ld = lm_parts_alloc(V);
+  for (int j = 1; j <= K; ++j) {
+    uint16_t* hout = h_steps ? h_steps + static_cast<size_t>(j - 1) * B * H : w.h[(j - 1) & 1];
+    int* sched = w.sched + static_cast<size_t>(2 * (j - 1)) * mv::kSchedInts;
+    MV_TRY(draft_gemm_impl(w.u, B, H, d, w.z, w.a, hout, err, sched, st));
+    int used = 0;
+    MV_TRY(lm_gemm_impl(hout, B, H, w_lm, V, w.keys, ld, err, sched + mv::kSchedInts, st, true, &used,
+                        KIND_DRAFT_LM));
+    a.keys = w.keys;
+    a.nparts = used;
+    a.ld = ld;
+    a.j = j;
+    a.h_src = hout;
+    a.row_stride = 1;
+    a.acc = nullptr;
+    a.u = (j < K) ? w.u : nullptr;
+    e = run_kernel(KIND_DRAFT_STEP, st, [&] { return mv::launch_mtp_step(a, st); });
+    if (e != cudaSuccess) return cuda_fail(e, "draft_step launch");
+  }
+  return MV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fastmtp_draft_workspace_size(int32_t B, int32_t K, int32_t H, int32_t I_d, int32_t V) {
+  if (B < 0 || K < 0 || H <= 0 || I_d <= 0 || V <= 0) return 0;
+  Carve c{nullptr};
+  carve_draft(c, B, K, H, I_d, V);
+  return kHeader + c.off + 1024;
+}
+
+mv_status fastmtp_draft(const uint16_t* h0, const int32_t* t0, int32_t B, int32_t K, int32_t H,
+                        const mv_draft_weights* draft, const uint16_t* w_lm, int32_t V, int32_t* drafts,
+                        uint16_t* h_steps, void* ws, size_t ws_bytes, mv_stream_t stream) {
+  if (B < 0 || K < 0 || K > 32 || H <= 0 || V <= 0)
+    return fail(MV_ERR_INVALID_ARG, "bad sizes B=%d K=%d (K <= 32) H=%d V=%d", B, K, H, V);
+  MV_TRY(check_draft(draft, H));
+  if (V % 8) return fail(MV_ERR_UNSUPPORTED_SHAPE, "V=%d must be a multiple of 8", V);
+  const bool none = (B == 0 || K == 0);
+  MV_TRY(check_ptr(h0, "h0", none));
+  MV_TRY(check_ptr(t0, "t0", none));
+  MV_TRY(check_ptr(w_lm, "w_lm"));
+  MV_TRY(check_ptr(drafts, "drafts", none));
+  MV_TRY(check_ptr(h_steps, "h_steps", true));
+  MV_TRY(check_ptr(ws, "workspace"));
+  const size_t need = fastmtp_draft_workspace_size(B, K, H, draft->I_d, V);
+  if (ws_bytes < need) return fail(MV_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+  if (none) return MV_OK;
+  Carve c{static_cast<char*>(ws) + kHeader};
+  const DraftWs w = carve_draft(c, B, K, H, draft->I_d, V);
+  return draft_impl(h0, 1, nullptr, t0, B, K, H, *draft, w_lm, V, drafts, h_steps, w, static_cast<int*>(ws),
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t speculative_step_workspace_size(int32_t B, int32_t K, const mv_moe_shape* shape, int32_t I_d, int32_t V) {
+  if (!shape) return 0;
+  const size_t v = verify_step_workspace_size(B, K, shape, V);
+  const size_t d = fastmtp_draft_workspace_size(B, K, shape->H, I_d, V);
+  if (!v || !d) return 0;
+  return align_up(v, 1024) + d;
+}
+
+mv_status speculative_step(const uint16_t* hidden, const int32_t* drafts, int32_t B, int32_t K,
+                           const mv_moe_shape* shape, const mv_moe_weights* layers, int32_t n_layers,
+                           const uint16_t* w_lm, int32_t V, const mv_draft_weights* draft, int32_t* accepted,
+                           int32_t* next_token, int32_t* emitted, int32_t* argmax, int32_t* next_drafts, void* ws,
+                           size_t ws_bytes, mv_stream_t stream) {
+  MV_TRY(check_shape(shape));
+  MV_TRY(check_draft(draft, shape->H));
+  MV_TRY(check_ptr(next_drafts, "next_drafts", K == 0 || B == 0));
+  if (next_drafts && drafts && next_drafts == drafts) return fail(MV_ERR_INVALID_ARG, "next_drafts may not alias drafts");
+  const size_t need = speculative_step_workspace_size(B, K, shape, draft->I_d, V);
+  if (!need) return fail(MV_ERR_INVALID_ARG, "bad sizes B=%d K=%d V=%d", B, K, V);
+  MV_TRY(check_ptr(ws, "workspace"));
+  if (ws_bytes < need) return fail(MV_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+  const size_t vbytes = align_up(verify_step_workspace_size(B, K, shape, V), 1024);
+  const uint16_t* h_last = nullptr;
+  MV_TRY(verify_step_impl(hidden, drafts, B, K, shape, layers, n_layers, w_lm, V, accepted, next_token, emitted,
+                          argmax, ws, vbytes, stream, &h_last));
+  if (B == 0 || K == 0) return MV_OK;
+  Carve c{static_cast<char*>(ws) + vbytes + kHeader};
+  const DraftWs w = carve_draft(c, B, K, shape->H, draft->I_d, V);
+  return draft_impl(h_last, K + 1, accepted, next_token, B, K, shape->H, *draft, w_lm, V, next_drafts, nullptr, w,
+                    static_cast<int*>(ws), reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

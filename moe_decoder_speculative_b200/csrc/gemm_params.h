@@ -6,7 +6,8 @@
 
 namespace mv {
 
-enum { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_ARGMAX = 2, EPI_SWIGLU_ROWS = 3, EPI_STORE_ROWS = 4, EPI_TOPK = 5 };
+enum { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_ARGMAX = 2, EPI_SWIGLU_ROWS = 3, EPI_STORE_ROWS = 4, EPI_TOPK = 5,
+       EPI_STORE_BF16 = 6 };  // EPI_STORE_BF16: bf16(res + acc), res nullable (swap-AB tiles)
 // Operand modes.  The first four put weights on the MMA's M side (swap-AB);
 // the tokens-on-M modes load the same tiles but multiply 128 token rows by 256
 // weight rows (gate|up tiles, or two halves of W_down) into one accumulator.
@@ -64,6 +65,7 @@ struct GemmSet {
   void* out2;              // EPI_TOPK: fp32 weights [rows][topk] (`out` holds int32 ids [rows][topk])
   const float* bias;       // EPI_TOPK: fp32 [M] added to the logits, or nullptr
   int32_t topk;            // EPI_TOPK: k
+  const uint16_t* res;     // EPI_STORE_BF16: bf16 [rows][ld_out] added before rounding, or nullptr
 };
 
 struct GemmParams {

@@ -549,6 +549,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
           }
         }
+      } else if (S.epi == EPI_STORE_BF16) {
+        // out[n][m] = bf16(res[n][m] + acc) (res nullable).  res was written
+        // by an earlier set of this launch (a dependency): read it from L2.
+        uint16_t* out = static_cast<uint16_t*>(S.out);
+        const int m = ui.m0 + row;
+        const bool mvalid = m < S.M;
+        for (int c0 = 0; c0 < n_mma; c0 += 32) {
+          uint32_t d[32];
+          tmem_ld32(tl + c0, d);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int n = c0 + j;
+            if (mvalid && n < ui.nvalid) {
+              const size_t o = static_cast<size_t>(ui.b_row0 + n) * S.ld_out + m;
+              float v = __uint_as_float(d[j]);
+              if (S.res) v = __fadd_rn(bf16_bits_to_f32(__ldcg(S.res + o)), v);
+              out[o] = f32_to_bf16_bits(v);
+            }
+          }
+        }
       } else if (LM) {  // EPI_ARGMAX over the tile's 128 (MODE_SINGLE) or 256 (MODE_MPAIR) vocabulary rows
         const int halves = (S.mode == MODE_MPAIR) ? 2 : 1;
         uint64_t* out = static_cast<uint64_t*>(S.out);

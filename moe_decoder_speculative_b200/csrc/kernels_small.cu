@@ -968,6 +968,115 @@ cudaError_t launch_lm_finalize(const uint64_t* keys, int nparts, int ld, int T, 
 }
 
 // ---------------------------------------------------------------------------
+// FastMTP draft block: the per-sequence step between its GEMMs (jina-ocr-v1
+// model card, decoding-speed paragraph: one dense draft block applied
+// recursively).  One CTA of 256 threads per sequence b:
+//  (1) the token t: with keys, the previous step's draft = the greedy choice
+//      of the LM head (largest packed key of row b), written to
+//      drafts[b][j-1]; without, t0[b] (the verifier's next token);
+//  (2) with u, the block's next input row
+//        u[b] = [ bf16((h * r_h) * g_h) ; bf16((e * r_e) * g_e) ],  e = w_emb[t],
+//        r = 1 / sqrt(sum(x^2) / H + eps)  (products and sums rounded singly),
+//      h = row b*row_stride + (acc ? acc[b] : 0) of h_src.
+// A token outside [0, V) (a failed LM step, or a bad t0) is reported as an
+// internal error, written as -1, and embeds row 0.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float block_sum_256(float v, float* red8, int lane, int wid) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) red8[wid] = v;
+  __syncthreads();
+  float s = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) s = __fadd_rn(s, red8[w]);
+  return s;
+}
+
+__global__ void __launch_bounds__(256) mtp_step_kernel(
+    const uint64_t* __restrict__ keys, int nparts, int ld, const int32_t* __restrict__ t0,
+    int32_t* __restrict__ drafts, int K, int j, const uint16_t* __restrict__ h_src, int row_stride,
+    const int32_t* __restrict__ acc, const uint16_t* __restrict__ w_emb, int V, const uint16_t* __restrict__ g_h,
+    const uint16_t* __restrict__ g_e, int H, float eps, uint16_t* __restrict__ u, int* err) {
+  __shared__ uint64_t red[8];
+  __shared__ float red_h[8], red_e[8];
+  __shared__ int t_s;
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (keys) {
+    row_max_key(keys + static_cast<size_t>(b) * ld, nparts, tid, 256, red, lane, wid);
+    __syncthreads();
+    if (tid == 0) {
+      uint64_t best = red[0];
+      for (int w = 1; w < 8; ++w) best = umax64(best, red[w]);
+      int t = static_cast<int>(argmax_key_index(best));
+      if (t < 0 || t >= V) {
+        t = -1;
+        if (err) atomicOr(err, kErrInternal);
+      }
+      drafts[static_cast<size_t>(b) * K + (j - 1)] = t;
+      t_s = t;
+    }
+  } else if (tid == 0) {
+    int t = t0[b];
+    if (t < 0 || t >= V) {
+      t = -1;
+      if (err) atomicOr(err, kErrInternal);
+    }
+    t_s = t;
+  }
+  __syncthreads();
+  if (!u) return;  // uniform: the last step only writes its draft
+  const int t = t_s < 0 ? 0 : t_s;
+  int a = acc ? acc[b] : 0;
+  a = a < 0 ? 0 : (a >= row_stride ? row_stride - 1 : a);
+  const uint4* hrow = reinterpret_cast<const uint4*>(h_src + (static_cast<size_t>(b) * row_stride + a) * H);
+  const uint4* erow = reinterpret_cast<const uint4*>(w_emb + static_cast<size_t>(t) * H);
+  const int hv = H / 8;
+  float sh = 0.f, se = 0.f;
+  for (int c = tid; c < hv; c += 256) {
+    float fh[8], fe[8];
+    bf16x8_to_f32(hrow[c], fh);
+    bf16x8_to_f32(__ldg(erow + c), fe);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      sh = __fadd_rn(sh, __fmul_rn(fh[i], fh[i]));
+      se = __fadd_rn(se, __fmul_rn(fe[i], fe[i]));
+    }
+  }
+  sh = block_sum_256(sh, red_h, lane, wid);
+  se = block_sum_256(se, red_e, lane, wid);
+  const float rh = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(sh, static_cast<float>(H)), eps)));
+  const float re = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(se, static_cast<float>(H)), eps)));
+  uint4* urow = reinterpret_cast<uint4*>(u + static_cast<size_t>(b) * 2 * H);
+  const uint4* gh = reinterpret_cast<const uint4*>(g_h);
+  const uint4* ge = reinterpret_cast<const uint4*>(g_e);
+  for (int c = tid; c < hv; c += 256) {
+    float fh[8], fe[8], gfh[8], gfe[8];
+    bf16x8_to_f32(hrow[c], fh);
+    bf16x8_to_f32(__ldg(erow + c), fe);
+    bf16x8_to_f32(__ldg(gh + c), gfh);
+    bf16x8_to_f32(__ldg(ge + c), gfe);
+    uint32_t oh[4], oe[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      oh[i] = static_cast<uint32_t>(f32_to_bf16_bits(__fmul_rn(__fmul_rn(fh[2 * i], rh), gfh[2 * i]))) |
+              (static_cast<uint32_t>(f32_to_bf16_bits(__fmul_rn(__fmul_rn(fh[2 * i + 1], rh), gfh[2 * i + 1]))) << 16);
+      oe[i] = static_cast<uint32_t>(f32_to_bf16_bits(__fmul_rn(__fmul_rn(fe[2 * i], re), gfe[2 * i]))) |
+              (static_cast<uint32_t>(f32_to_bf16_bits(__fmul_rn(__fmul_rn(fe[2 * i + 1], re), gfe[2 * i + 1]))) << 16);
+    }
+    urow[c] = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+    urow[hv + c] = make_uint4(oe[0], oe[1], oe[2], oe[3]);
+  }
+}
+
+cudaError_t launch_mtp_step(const MtpStepArgs& a, cudaStream_t s) {
+  if (a.B <= 0) return cudaSuccess;
+  return launch_pdl(mtp_step_kernel, dim3(a.B), dim3(256), 0, s, a.keys, a.nparts, a.ld, a.t0, a.drafts, a.K, a.j,
+                    a.h_src, a.row_stride, a.acc, a.w_emb, a.V, a.g_h, a.g_e, a.H, a.eps, a.u, a.err);
+}
+
+// ---------------------------------------------------------------------------
 // Greedy acceptance (one thread per sequence).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void accept_one(const int32_t* g, const int32_t* d, int K, int b,

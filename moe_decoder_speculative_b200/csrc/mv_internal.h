@@ -95,6 +95,26 @@ cudaError_t launch_permute_sorted(const int32_t* idx, int T, int E, int k, int32
 cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t* inv,
                            const float* w, const uint16_t* res, uint16_t* out, int T, int H,
                            int k, int n_pos, int* err, const L2Prefetch& pf, cudaStream_t s);
+// The FastMTP draft block's per-sequence step (kernels_small.cu, mtp_step_kernel).
+struct MtpStepArgs {
+  const uint64_t* keys;   // previous step's LM keys [B][ld] (nparts used), or nullptr: take t0
+  int nparts, ld;
+  const int32_t* t0;      // [B] first tokens (when keys is nullptr)
+  int32_t* drafts;        // [B][K]; step j writes column j-1
+  int K, j;
+  const uint16_t* h_src;  // previous hidden states, row b*row_stride + (acc ? acc[b] : 0)
+  int row_stride;
+  const int32_t* acc;
+  const uint16_t* w_emb;  // [V][H]
+  int V;
+  const uint16_t *g_h, *g_e;
+  int H;
+  float eps;
+  uint16_t* u;            // [B][2H] next input rows, or nullptr (last step)
+  int* err;
+  int B;
+};
+cudaError_t launch_mtp_step(const MtpStepArgs& a, cudaStream_t s);
 cudaError_t launch_lm_finalize(const uint64_t* keys, int nparts, int ld, int T, int32_t* argmax,
                                cudaStream_t s);
 cudaError_t launch_accept(const int32_t* argmax, const int32_t* drafts, int B, int K,
