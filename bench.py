@@ -59,6 +59,8 @@ def parse_args():
                     help="time replays of the step recorded once as a CUDA graph (verify_graph_*)")
     ap.add_argument("--latency", action="store_true",
                     help="per-step latency of one sequence (batch 1) for K = 0, 1, 3, eager and graph")
+    ap.add_argument("--spec", action="store_true",
+                    help="the draft-and-verify loop step (speculative_step) and the FastMTP draft block alone")
     return ap.parse_args()
 
 
@@ -555,6 +557,102 @@ def run_latency(args):
     return 0
 
 
+def draft_step_bytes(w, B, I_d):
+    """Algorithmic bytes of one FastMTP draft step for B rows: the projection,
+    the dense SwiGLU and the LM head weights once, the embedding rows, and the
+    bf16 rows in and out of each GEMM."""
+    H, V = w.H, w.V
+    weights = 2 * H * H * 2 + 3 * I_d * H * 2 + V * H * 2
+    rows = B * (2 * H * 2 + H * 2 * 4 + I_d * 2 * 2 + H * 2)   # u, z (w+r twice), a (w+r), h'
+    return weights + rows + B * H * 2
+
+
+def run_spec(args):
+    """speculative_step on the concurrency-32 workload: one draft-and-verify
+    loop iteration (verify_step, then K FastMTP draft-block steps from the
+    verifier's state) with inputs resident, and fastmtp_draft alone.  The
+    draft block's weights are synthetic, so its drafts rarely match the
+    verifier (the committed tokens per iteration are reported as measured)."""
+    import torch
+
+    from moe_decoder_speculative_b200 import binding as bd
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    w = wl.workload(args.workload)
+    assert w.has_verify, "a verify workload"
+    inp = wl.make_inputs(w, layers=args.layers)
+    shape = bd.shape_of(w)
+    layers = [bd.LayerWeights(l, dev) for l in inp["layers"]]
+    w_lm = bd.bf16_to_device(inp["w_lm"], dev)
+    hidden = bd.bf16_to_device(inp["hidden"], dev)
+    dw = bd.DraftWeights(wl.make_draft_block(w), dev)
+    vplan = bd.VerifyPlan(shape, layers, w_lm, w.B, w.K, dev)
+    _, _, _, am = vplan(hidden, torch.zeros((w.B, w.K), dtype=torch.int32, device=dev))
+    drafts = torch.from_numpy(wl.make_drafts(w, am.cpu().numpy())).to(dev)
+    sp = bd.SpeculativePlan(shape, layers, w_lm, dw, w.B, w.K, dev)
+    h0 = hidden[:: w.K + 1].contiguous()
+    t0 = am[:: w.K + 1].contiguous()
+    dws = bd.workspace(int(bd.lib().fastmtp_draft_workspace_size(w.B, w.K, w.H, dw.I_d, w.V)), dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n0 = bd.launch_count()
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n, (bd.launch_count() - n0) // n
+
+    n = max(20, args.steps)
+    with ClockSampler(gpu_uuid(torch, dev)) as clocks:
+        ms_spec, l_spec = timed(lambda: sp(hidden, drafts), n)
+        ms_verify, l_verify = timed(lambda: vplan(hidden, drafts), n)
+        ms_draft, l_draft = timed(lambda: bd.fastmtp_draft(h0, t0, w.K, dw, w_lm, ws=dws), n)
+        bd.profile_enable(True)
+        for _ in range(n):
+            sp(hidden, drafts)
+        torch.cuda.synchronize()
+        bd.profile_enable(False)
+        kern = bd.profile_collect()
+    sp.sync_status()
+    bd.sync_status(dws)
+    acc = sp.accepted.cpu().numpy()
+    nd = sp.next_drafts.cpu().numpy()
+    step_bytes = draft_step_bytes(w, w.B, dw.I_d)
+    peak, peak_kind = measured_peaks()
+    kernels = {k: {"launches": v["launches"], "avg_us": round(1e3 * v["ms"] / v["launches"], 2)}
+               for k, v in kern.items() if v["launches"]}
+    d_gemm = kern.get("draft_block_gemm", {"ms": 0, "launches": 1})
+    d_lm = kern.get("draft_lm_head_argmax", {"ms": 0, "launches": 1})
+    draft_bytes = w.K * step_bytes
+    print(json.dumps({
+        "metric": "draft-and-verify loop iteration (speculative_step) at 32 sequences x K=3",
+        "value": ms_spec * 1e3, "unit": "us per iteration", "higher_is_better": False, "n_gpus": 1,
+        "steps": n, "warmup": args.warmup, "dtype": "bf16",
+        "data": "synthetic (seeded weights; draft block weights random, so its drafts rarely match)",
+        "config": {"workload": w.name, "B": w.B, "K": w.K, "layers": len(layers), "I_d": dw.I_d},
+        "verify_us": ms_verify * 1e3, "draft_us": ms_draft * 1e3,
+        "launches": {"speculative_step": l_spec, "verify_step": l_verify, "fastmtp_draft": l_draft},
+        "draft_roofline": {"bound": "hbm", "alg_bytes": int(draft_bytes),
+                           "achieved_gbs": round(draft_bytes / (ms_draft / 1e3) / 1e9, 1), "peak_gbs": peak,
+                           "frac": round(draft_bytes / (ms_draft / 1e3) / 1e9 / peak, 4), "peak_source": peak_kind},
+        "draft_kernels": {"draft_block_gemm_gbs": round((2 * w.H * w.H * 2 + 3 * dw.I_d * w.H * 2) /
+                                                        (d_gemm["ms"] / d_gemm["launches"] / 1e3) / 1e9, 1)
+                          if d_gemm["ms"] else None,
+                          "draft_lm_gbs": round(w.V * w.H * 2 / (d_lm["ms"] / d_lm["launches"] / 1e3) / 1e9, 1)
+                          if d_lm["ms"] else None},
+        "kernels": kernels, "committed_per_iteration": int((acc + 1).sum()),
+        "next_drafts_valid": bool(np.all((nd >= 0) & (nd < w.V))), "clocks": clocks.summary(),
+    }))
+    return 0
+
+
 def run_prefill(args):
     """A MoE layer over prefill-sized batches (routing + grouped SwiGLU experts +
     combine), tensor-bound: reports rows/s and the grouped GEMM's TFLOP/s."""
@@ -633,6 +731,8 @@ def main():
         return run_reference(args)
     if args.latency:
         return run_latency(args)
+    if args.spec:
+        return run_spec(args)
     if not wl.workload(args.workload).has_verify:
         return run_prefill(args)
     return run_ours(args)

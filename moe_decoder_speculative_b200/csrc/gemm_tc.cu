@@ -59,6 +59,7 @@ struct UnitInfo {
   int set, g, gi, m0, nvalid, b_row0;
 };
 
+
 __device__ __forceinline__ int upper_pow2_cols(int c) {
   int n = 32;
   while (n < c) n <<= 1;
@@ -112,6 +113,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
+  // Each tile configuration compiles only the epilogues it is launched with
+  // (a smaller kernel keeps its hot loops in the instruction cache): the
+  // weights-on-M tiles (BN = 32) the SwiGLU / fp32 / bf16 stores,
+  // the tokens-on-M tiles (BN = 128) the row stores and the router top-k, the
+  // LM head the argmax.
+  constexpr bool kSwapAB = !LM && BN == 32;
+  constexpr bool kTokM = !LM && BN == 128;
 
   pdl_trigger();
   if (warp == 0 && lane == 0) {
@@ -284,14 +292,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
           } else {
             const bool two = (S.mode != MODE_SINGLE && S.mode != MODE_TROUTE);
+            const int kx = ks * 64;
             mbar_arrive_expect_tx(&full_bar[stage], (two ? 2u : 1u) * kATileBytes + b_bytes);
-            tma_load_2d(st, &S.a0, ks * 64, a_row0, &full_bar[stage], pol_w);
+            tma_load_2d(st, &S.a0, kx, a_row0, &full_bar[stage], pol_w);
             if (S.mode == MODE_GATEUP || S.mode == MODE_TGATEUP)
-              tma_load_2d(st + kATileBytes, &S.a1, ks * 64, a_row0, &full_bar[stage], pol_w);
+              tma_load_2d(st + kATileBytes, &S.a1, kx, a_row0, &full_bar[stage], pol_w);
             else if (S.mode == MODE_MPAIR || S.mode == MODE_TPAIR)
-              tma_load_2d(st + kATileBytes, &S.a0, ks * 64, a_row0 + 128, &full_bar[stage], pol_w);
+              tma_load_2d(st + kATileBytes, &S.a0, kx, a_row0 + 128, &full_bar[stage], pol_w);
             for (int c = 0; c < nchunk; ++c)
-              tma_load_2d(b0 + c * kBBox * 128, &S.b, ks * 64, ui.b_row0 + c * kBBox, &full_bar[stage], pol_x);
+              tma_load_2d(b0 + c * kBBox * 128, &S.b, kx, ui.b_row0 + c * kBBox, &full_bar[stage], pol_x);
           }
           fills[stage]++;
           if (++stage == STAGES) {
@@ -404,7 +413,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       const int row = wq * 32 + lane;  // row of the 128-row tile held by this thread
       const uint32_t tl = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + static_cast<uint32_t>(slot * ACC_COLS);
       const int n_mma = (ui.nvalid + 15) & ~15;
-      if (S.epi == EPI_TOPK) {
+      // The accumulator slot goes back to the MMA warp as soon as this warp
+      // has read its last TMEM columns of the unit, before the stores: slow
+      // stores then delay only this warp, not the next unit's MMAs.
+      bool released = false;
+      auto release_tmem = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty_bar[slot]);
+        released = true;
+      };
+      if (kTokM && S.epi == EPI_TOPK) {
         // tokens on M: this thread holds all router logits of token `row`;
         // top-k on the logits (ties to the lower id, slots in descending
         // order), weights exp(l_j - l_max) / sum over the kept experts.  The
@@ -464,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
               ow[j] = expf(sv[j] - sv[0]) / s;
             }
         }
-      } else if (S.epi == EPI_SWIGLU_ROWS || S.epi == EPI_STORE_ROWS) {
+      } else if (kTokM && (S.epi == EPI_SWIGLU_ROWS || S.epi == EPI_STORE_ROWS)) {
         // tokens on M: this thread holds token row `row` of the tile, the
         // columns are 256 weight outputs (gate|up, or two halves of W_down)
         const bool tvalid = row < ui.nvalid;
@@ -511,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
           }
         }
-      } else if (S.epi == EPI_SWIGLU) {
+      } else if (kSwapAB && S.epi == EPI_SWIGLU) {
         const int m = ui.m0 + row;
         const bool mvalid = m < S.M;
         uint16_t* out = static_cast<uint16_t*>(S.out);
@@ -520,6 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           tmem_ld32(tl + c0, g);
           tmem_ld32(tl + BN + c0, v);
           tmem_ld_wait();
+          if (c0 + 32 >= n_mma) release_tmem();
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int n = c0 + j;
@@ -531,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
           }
         }
-      } else if (S.epi == EPI_STORE_F32) {
+      } else if (kSwapAB && S.epi == EPI_STORE_F32) {
         float* out = static_cast<float*>(S.out);
         const int halves = (S.mode == MODE_MPAIR) ? 2 : 1;
         for (int h = 0; h < halves; ++h) {
@@ -541,6 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             uint32_t d[32];
             tmem_ld32(tl + h * BN + c0, d);
             tmem_ld_wait();
+            if (h + 1 == halves && c0 + 32 >= n_mma) release_tmem();
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int n = c0 + j;
@@ -549,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
           }
         }
-      } else if (S.epi == EPI_STORE_BF16) {
+      } else if (kSwapAB && S.epi == EPI_STORE_BF16) {
         // out[n][m] = bf16(res[n][m] + acc) (res nullable).  res was written
         // by an earlier set of this launch (a dependency): read it from L2.
         uint16_t* out = static_cast<uint16_t*>(S.out);
@@ -559,6 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           uint32_t d[32];
           tmem_ld32(tl + c0, d);
           tmem_ld_wait();
+          if (c0 + 32 >= n_mma) release_tmem();
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int n = c0 + j;
@@ -607,8 +629,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             out[static_cast<size_t>(ui.b_row0 + n) * S.ld_out + part] = best_key;
           }
         }
+      } else if (lane == 0) {
+        atomicOr(p.err, kErrInternal);  // a set this tile configuration is not compiled for
       }
-      tc_fence_before();
+      if (!released) tc_fence_before();
       if (S.signal && p.sched) {  // release this warp's stores to the units that depend on the group
         fence_proxy_async_global();
         __syncwarp();
@@ -618,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty_bar[slot]);
+      if (!released && lane == 0) mbar_arrive(&tempty_bar[slot]);
     }
   }
 
