@@ -122,6 +122,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   constexpr bool kTokM = !LM && BN == 128;
 
   pdl_trigger();
+  // ---- set-up that needs nothing from the previous kernel ----------------
+  // Barriers, TMEM (one CTA per SM by shared memory, so two GEMM launches
+  // never hold TMEM on one SM) and descriptors.
+  if (tid == 0) {
+    abort_s = 0;
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull_bar[i], 1);
+      mbar_init(&tempty_bar[i], 4);
+    }
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&ufull_bar[i], 1);
+      mbar_init(&uempty_bar[i], 5);  // the MMA thread + 4 epilogue warps
+    }
+    mbar_init(&mma_done_bar, 1);
+    fence_barrier_init();
+  }
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < p.nsets; ++s) {
       tma_prefetch_desc(&p.set[s].a0);
@@ -129,6 +149,98 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       tma_prefetch_desc(&p.set[s].b);
     }
   }
+  const int tmem_cols = upper_pow2_cols(2 * ACC_COLS);
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_s, tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+
+  // TMA issue of one stage of a unit: the weights (A) part with the stage's
+  // full byte count, and/or the token-row (B) part.
+  const uint64_t pol_w = policy_evict_first();
+  const uint64_t pol_x = policy_evict_last();
+  auto issue_stage = [&](const GemmSet& S, const UnitInfo& ui, int ks, int stg, bool wts, bool toks) {
+    uint8_t* st = smem + stg * STAGE_BYTES;
+    uint8_t* b0 = st + 2 * kATileBytes;
+    const int a_row0 = ui.gi * S.a_group_stride + ui.m0;
+    const int nchunk = (ui.nvalid + kBBox - 1) / kBBox;
+    const uint32_t b_bytes = nchunk * kBBox * 128;
+    const int kblocks = S.K / 64;
+    if (S.mode == MODE_KPAIR) {
+      const int kb0 = 2 * ks;
+      const bool two = kb0 + 1 < kblocks;
+      uint8_t* b1 = b0 + (NB > 1 ? B_TILE_BYTES : 0);
+      if (wts) {
+        mbar_arrive_expect_tx(&full_bar[stg], (two ? 2u : 1u) * (kATileBytes + b_bytes));
+        tma_load_2d(st, &S.a0, kb0 * 64, a_row0, &full_bar[stg], pol_w);
+        if (two) tma_load_2d(st + kATileBytes, &S.a0, (kb0 + 1) * 64, a_row0, &full_bar[stg], pol_w);
+      }
+      if (toks) {
+        for (int c = 0; c < nchunk; ++c)
+          tma_load_2d(b0 + c * kBBox * 128, &S.b, kb0 * 64, ui.b_row0 + c * kBBox, &full_bar[stg], pol_x);
+        if (two)
+          for (int c = 0; c < nchunk; ++c)
+            tma_load_2d(b1 + c * kBBox * 128, &S.b, (kb0 + 1) * 64, ui.b_row0 + c * kBBox, &full_bar[stg], pol_x);
+      }
+    } else {
+      const bool two = (S.mode != MODE_SINGLE && S.mode != MODE_TROUTE);
+      const int kx = ks * 64;
+      if (wts) {
+        mbar_arrive_expect_tx(&full_bar[stg], (two ? 2u : 1u) * kATileBytes + b_bytes);
+        tma_load_2d(st, &S.a0, kx, a_row0, &full_bar[stg], pol_w);
+        if (S.mode == MODE_GATEUP || S.mode == MODE_TGATEUP)
+          tma_load_2d(st + kATileBytes, &S.a1, kx, a_row0, &full_bar[stg], pol_w);
+        else if (S.mode == MODE_MPAIR || S.mode == MODE_TPAIR)
+          tma_load_2d(st + kATileBytes, &S.a0, kx, a_row0 + 128, &full_bar[stg], pol_w);
+      }
+      if (toks)
+        for (int c = 0; c < nchunk; ++c)
+          tma_load_2d(b0 + c * kBBox * 128, &S.b, kx, ui.b_row0 + c * kBBox, &full_bar[stg], pol_x);
+    }
+  };
+  auto unit_stages = [](const GemmSet& S) {
+    const int kblocks = S.K / 64;
+    return (S.mode == MODE_KPAIR) ? (kblocks + 1) / 2 : kblocks;
+  };
+
+  // The first set, when its rows are static and it depends on nothing, gives
+  // CTA b its first unit b (the others are claimed in order after them), so
+  // the weights of that unit can stream before the previous kernel ends: its
+  // first stages are issued here, weights only; the token rows follow the wait.
+  const GemmSet& S0 = p.set[0];
+  const bool first_static = !S0.counts && !S0.offsets && S0.groups == 1 && S0.dep_set < 0 && S0.static_rows > 0;
+  const int nt0 = first_static ? (S0.static_rows + BN - 1) / BN : 0;
+  const int units0 = first_static ? (S0.M + S0.m_tile - 1) / S0.m_tile * nt0 : 0;
+  const int nstatic = min(units0, static_cast<int>(gridDim.x));
+  const bool early = static_cast<int>(blockIdx.x) < nstatic;
+  UnitInfo ui0{};
+  if (early) {
+    const int u0 = static_cast<int>(blockIdx.x);
+    const int n0 = (u0 % nt0) * BN;
+    ui0.g = 0;
+    ui0.set = 0;
+    ui0.gi = 0;
+    ui0.m0 = (u0 / nt0) * S0.m_tile;
+    ui0.nvalid = min(BN, S0.static_rows - n0);
+    ui0.b_row0 = n0;
+  }
+  int stage = 0;  // producer state (warp 0, lane 0)
+  uint32_t phase = 0;
+  int fills[STAGES];
+#pragma unroll
+  for (int i = 0; i < STAGES; ++i) fills[i] = 0;
+  const int npre = early ? min(STAGES, unit_stages(S0)) : 0;
+  if (warp == 0 && lane == 0) {
+    for (int ks = 0; ks < npre; ++ks) {  // fresh barriers: no empty-slot wait
+      issue_stage(S0, ui0, ks, ks, true, false);
+      fills[ks]++;
+    }
+  }
+
   pdl_wait();  // the group sizes and the B operands come from the previous kernels
 
   // ---- group table (every CTA builds the same one) -----------------------
@@ -158,24 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     g_nt[g] = nt;
     g_begin[g + 1] = mt * nt;  // unit count, scanned below
   }
-  if (tid == 0) {
-    g_begin[0] = 0;
-    abort_s = 0;
-    for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&tfull_bar[i], 1);
-      mbar_init(&tempty_bar[i], 4);
-    }
-    for (int i = 0; i < kRing; ++i) {
-      mbar_init(&ufull_bar[i], 1);
-      mbar_init(&uempty_bar[i], 5);  // the MMA thread + 4 epilogue warps
-    }
-    mbar_init(&mma_done_bar, 1);
-    fence_barrier_init();
-  }
+  if (tid == 0) g_begin[0] = 0;
   __syncthreads();
   if (warp == 0) {  // inclusive scan of unit counts, 32 groups at a time
     int carry = 0;
@@ -193,7 +288,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   }
   __syncthreads();
   const int total_units = g_begin[ng];
-  if (total_units == 0) return;  // uniform across the CTA
 
   auto decode = [&](int u) -> UnitInfo {
     int lo = 0, hi = ng;  // g with g_begin[g] <= u < g_begin[g+1]
@@ -215,31 +309,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   };
   auto group_units = [&](int g) { return g_begin[g + 1] - g_begin[g]; };
 
-  const int tmem_cols = upper_pow2_cols(2 * ACC_COLS);
-  if (warp == 1) {
-    tmem_alloc(&tmem_base_s, tmem_cols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = tmem_base_s;
-
-  if (warp == 0) {
+  if (total_units == 0) {
+    // nothing to do (uniform across the CTA); no copy was issued early, since
+    // an early unit implies a non-empty first set
+  } else if (warp == 0) {
     // ======================= claimer + TMA producer ========================
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_x = policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
-      int fills[STAGES];
-#pragma unroll
-      for (int i = 0; i < STAGES; ++i) fills[i] = 0;
       bool ok = true;
       for (int it = 0; ok; ++it) {
         const int q = it % kRing;
         if (!mbar_wait(&uempty_bar[q], ((it / kRing) & 1) ^ 1u, &abort_s, p.err, deadline)) break;
-        int u = p.sched ? atomicAdd(p.sched, 1) : static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
+        int u;
+        if (it == 0 && early)
+          u = static_cast<int>(blockIdx.x);
+        else
+          u = p.sched ? nstatic + atomicAdd(p.sched, 1) : static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
         if (u >= total_units) u = -1;
         unit_ring[q] = u;
         mbar_arrive(&ufull_bar[q]);
@@ -264,45 +348,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           if (!ok) break;
           fence_proxy_async_global();
         }
-        const int a_row0 = ui.gi * S.a_group_stride + ui.m0;
-        const int nchunk = (ui.nvalid + kBBox - 1) / kBBox;
-        const uint32_t b_bytes = nchunk * kBBox * 128;
-        const int kblocks = S.K / 64;
-        const int nstage = (S.mode == MODE_KPAIR) ? (kblocks + 1) / 2 : kblocks;
+        const int nstage = unit_stages(S);
         for (int ks = 0; ks < nstage; ++ks) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_s, p.err, deadline)) {
+          const bool pre = (it == 0 && ks < npre);  // weights already issued before the wait
+          if (!pre && !mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_s, p.err, deadline)) {
             ok = false;
             break;
           }
-          uint8_t* st = smem + stage * STAGE_BYTES;
-          uint8_t* b0 = st + 2 * kATileBytes;
-          if (S.mode == MODE_KPAIR) {
-            const int kb0 = 2 * ks;
-            const bool two = kb0 + 1 < kblocks;
-            mbar_arrive_expect_tx(&full_bar[stage], (two ? 2u : 1u) * (kATileBytes + b_bytes));
-            tma_load_2d(st, &S.a0, kb0 * 64, a_row0, &full_bar[stage], pol_w);
-            for (int c = 0; c < nchunk; ++c)
-              tma_load_2d(b0 + c * kBBox * 128, &S.b, kb0 * 64, ui.b_row0 + c * kBBox, &full_bar[stage], pol_x);
-            if (two) {
-              tma_load_2d(st + kATileBytes, &S.a0, (kb0 + 1) * 64, a_row0, &full_bar[stage], pol_w);
-              uint8_t* b1 = b0 + (NB > 1 ? B_TILE_BYTES : 0);
-              for (int c = 0; c < nchunk; ++c)
-                tma_load_2d(b1 + c * kBBox * 128, &S.b, (kb0 + 1) * 64, ui.b_row0 + c * kBBox, &full_bar[stage],
-                            pol_x);
-            }
-          } else {
-            const bool two = (S.mode != MODE_SINGLE && S.mode != MODE_TROUTE);
-            const int kx = ks * 64;
-            mbar_arrive_expect_tx(&full_bar[stage], (two ? 2u : 1u) * kATileBytes + b_bytes);
-            tma_load_2d(st, &S.a0, kx, a_row0, &full_bar[stage], pol_w);
-            if (S.mode == MODE_GATEUP || S.mode == MODE_TGATEUP)
-              tma_load_2d(st + kATileBytes, &S.a1, kx, a_row0, &full_bar[stage], pol_w);
-            else if (S.mode == MODE_MPAIR || S.mode == MODE_TPAIR)
-              tma_load_2d(st + kATileBytes, &S.a0, kx, a_row0 + 128, &full_bar[stage], pol_w);
-            for (int c = 0; c < nchunk; ++c)
-              tma_load_2d(b0 + c * kBBox * 128, &S.b, kx, ui.b_row0 + c * kBBox, &full_bar[stage], pol_x);
-          }
-          fills[stage]++;
+          issue_stage(S, ui, ks, stage, !pre, true);
+          if (!pre) fills[stage]++;
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
