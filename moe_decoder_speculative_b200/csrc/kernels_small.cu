@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const uint16_t* __rest
                                                           const float* __restrict__ bias,
                                                           int32_t* __restrict__ idx,
                                                           float* __restrict__ wout) {
-  extern __shared__ __align__(16) uint8_t sm[];
+  extern __shared__ __align__(128) uint8_t sm[];
   uint16_t* xs = reinterpret_cast<uint16_t*>(sm);                        // [R][H]
   float* ls = reinterpret_cast<float*>(sm + static_cast<size_t>(R) * H * 2);  // [R][E]
   pdl_trigger();
@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
     const float* __restrict__ bias, int32_t* __restrict__ idx, float* __restrict__ wout, int* err,
     const L2Prefetch pf, int32_t* __restrict__ slab_counts, int32_t* __restrict__ inv_out,
     uint16_t* __restrict__ x_slab, int slab_rows) {
-  extern __shared__ __align__(16) uint8_t sm[];
+  extern __shared__ __align__(128) uint8_t sm[];
   __shared__ int32_t sel_s[R * 8];  // the experts each row selected
   __shared__ int32_t pos_s[R * 8];  // their slab rows (-1: skipped)
   uint16_t* hs = reinterpret_cast<uint16_t*>(sm);                         // [R][H]

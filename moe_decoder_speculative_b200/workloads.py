@@ -149,9 +149,10 @@ def _tree(wid: int):
     return root.spawn(7)
 
 
-def make_layer(w: Workload, layer_ss: np.random.SeedSequence) -> dict:
-    """One MoE layer's weights, all N(0, w_std^2) in bf16."""
-    s = layer_ss.spawn(7)
+def make_layer(w: Workload, layer_ss: np.random.SeedSequence, norm: bool = False) -> dict:
+    """One MoE layer's weights, all N(0, w_std^2) in bf16; with norm, also the
+    gain of the pre-RMSNorm variant, norm_gain [H] ~ 1 + N(0, 0.1^2)."""
+    s = layer_ss.spawn(8)
     H, E, I, Ish = w.H, w.E, w.I, w.I_sh
     d = {
         "w_router": normal_bf16(s[0], (E, H), w.w_std),
@@ -164,6 +165,8 @@ def make_layer(w: Workload, layer_ss: np.random.SeedSequence) -> dict:
         d["ws_up"] = normal_bf16(s[5], (Ish, H), w.w_std)
         d["ws_down"] = normal_bf16(s[6], (H, Ish), w.w_std)
     d["router_bias"] = None
+    if norm:
+        d["norm_gain"] = f32_to_bf16_bits(1.0 + bf16_bits_to_f32(normal_bf16(s[7], (H,), 0.1)))
     return d
 
 
@@ -200,7 +203,7 @@ def make_lm_head(w: Workload) -> np.ndarray | None:
     return normal_bf16(_tree(w.id)[2], (w.V, w.H), w.w_std)
 
 
-def make_inputs(w: Workload, layers: int | None = None) -> dict:
+def make_inputs(w: Workload, layers: int | None = None, norm: bool = False) -> dict:
     """All tensors of a workload except the drafts (which need the verifier's argmax).
 
     ``layers`` limits how many of the L layers are drawn (for partial tests); the
@@ -211,7 +214,7 @@ def make_inputs(w: Workload, layers: int | None = None) -> dict:
     layer_ss = t[1].spawn(w.L)
     out = {
         "hidden": make_hidden(w),
-        "layers": [make_layer(w, layer_ss[l]) for l in range(L)],
+        "layers": [make_layer(w, layer_ss[l], norm) for l in range(L)],
         "w_lm": make_lm_head(w),
     }
     if w.n_hot:

@@ -172,21 +172,26 @@ def greedy_accept(argmax, drafts, B, K):
 
 
 def moe_stack(hidden, layers, k, acc_double=False, n_threads=0, keep=False):
-    """Run the stacked MoE layers with a residual: h_{l+1} = bf16(h_l + MoE_l(h_l)).
+    """Run the stacked MoE layers with a residual: h_{l+1} = bf16(h_l + MoE_l(x_l)).
 
+    x_l = h_l, or, when the layer carries a "norm_gain" (the pre-RMSNorm
+    variant of the decoder block), x_l = rmsnorm(h_l, norm_gain): the router
+    and the experts see the normalised rows, the residual stays h_l.
     Returns a dict with the final h, and per layer the routing (idx, w), the
     6th-vs-7th logit gap and the MoE output m (when keep=True).
     """
     h = _u16(hidden)
     per_layer = []
     for layer in layers:
-        idx, w, logits, gap = router(h, layer["w_router"], k, bias=layer.get("router_bias"),
+        g = layer.get("norm_gain")
+        x = h if g is None else rmsnorm(h, g, acc_double=acc_double)
+        idx, w, logits, gap = router(x, layer["w_router"], k, bias=layer.get("router_bias"),
                                      acc_double=acc_double, n_threads=n_threads)
-        m, h_next = moe_ffn(h, layer, idx, w, residual=h, acc_double=acc_double,
+        m, h_next = moe_ffn(x, layer, idx, w, residual=h, acc_double=acc_double,
                             n_threads=n_threads)
         rec = {"idx": idx, "w": w, "gap": gap}
         if keep:
-            rec.update(h_in=h, m=m, logits=logits)
+            rec.update(h_in=h, m=m, logits=logits, x_in=x)
         per_layer.append(rec)
         h = h_next
     return {"h": h, "layers": per_layer}
