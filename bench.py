@@ -59,6 +59,8 @@ def parse_args():
                     help="time replays of the step recorded once as a CUDA graph (verify_graph_*)")
     ap.add_argument("--latency", action="store_true",
                     help="per-step latency of one sequence (batch 1) for K = 0, 1, 3, eager and graph")
+    ap.add_argument("--norm", action="store_true",
+                    help="the pre-RMSNorm variant of every layer (seeded norm gains)")
     ap.add_argument("--spec", action="store_true",
                     help="the draft-and-verify loop step (speculative_step) and the FastMTP draft block alone")
     return ap.parse_args()
@@ -308,7 +310,7 @@ def run_ours(args):
 
     w = wl.workload(args.workload)
     assert w.has_verify, "the benchmark times the verify step"
-    inp = wl.make_inputs(w, layers=args.layers)
+    inp = wl.make_inputs(w, layers=args.layers, norm=args.norm)
     if rank > 0:   # each replica verifies its own batch of sequences
         inp["hidden"] = wl.normal_bf16(np.random.SeedSequence([w.id, rank]), (w.T, w.H), w.x_std)
     shape = bd.shape_of(w)
@@ -437,6 +439,7 @@ def run_ours(args):
                    "top_k": w.k, "I": w.I, "I_shared": w.I_sh, "V": w.V,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "launch": "CUDA graph replay (verify_graph_launch)" if args.graph else "eager (verify_step)",
+                   "layer": "pre-RMSNorm variant" if args.norm else "residual, no norm",
                    "l2": "weights (5.8 GB) far larger than L2: no flush needed"},
         "rows_per_s": world * T * K / (ms / 1e3),
         "committed_per_step": committed_all,

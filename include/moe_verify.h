@@ -93,6 +93,15 @@ typedef struct {
   const uint16_t* ws_gate;   /* [I_shared][H]  (NULL when I_shared == 0) */
   const uint16_t* ws_up;     /* [I_shared][H] */
   const uint16_t* ws_down;   /* [H][I_shared] */
+  /* [H] gain of the pre-RMSNorm variant of the layer, or NULL (plain layer).
+   * With it, verify_step and speculative_step route and run the experts on
+   * x = bf16(RMSNorm(h) * norm_gain) and keep the residual h:
+   * h' = bf16(h + MoE(x)).  The pages name no norm (the model card's
+   * architecture paragraph gives only the decoder's shape); this is the
+   * DeepSeek-style decoder block without its attention.  moe_ffn_forward
+   * ignores it: compose moe_rmsnorm, moe_router_topk and moe_ffn_forward
+   * (x = the normalised rows, residual = h) instead. */
+  const uint16_t* norm_gain;
 } mv_moe_weights;
 
 /* ---------------------------------------------------------------------------
@@ -122,6 +131,15 @@ MV_API mv_status moe_router_topk(const uint16_t* x, int32_t T, const mv_moe_shap
  * ------------------------------------------------------------------------- */
 MV_API mv_status moe_expert_permute(const int32_t* topk_idx, int32_t T, int32_t E, int32_t k,
                              int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                             mv_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_rmsnorm - out[r] = bf16((x[r] * s_r) * gain), s_r = 1 / sqrt(sum_h
+ * x[r][h]^2 / H + 1e-6) in fp32 (products and sums singly rounded), for the
+ * pre-RMSNorm layer variant (see mv_moe_weights.norm_gain).
+ *   x, out [T][H] bf16 (may not alias), gain [H] bf16.  H a multiple of 8.
+ * ------------------------------------------------------------------------- */
+MV_API mv_status moe_rmsnorm(const uint16_t* x, int32_t T, int32_t H, const uint16_t* gain, uint16_t* out,
                              mv_stream_t stream);
 
 /* Bytes of workspace moe_ffn_forward needs for T rows. */

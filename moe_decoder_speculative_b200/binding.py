@@ -26,7 +26,7 @@ EXPORTED = ["moe_router_topk", "moe_expert_permute", "moe_ffn_workspace_size", "
             "mv_launch_count", "mv_profile_enable", "mv_profile_collect", "mv_kernel_name",
             "mv_set_wait_timeout_ns", "lm_head_argmax_noalloc", "verify_graph_create", "verify_graph_launch",
             "verify_graph_kernels", "verify_graph_destroy", "fastmtp_draft_workspace_size", "fastmtp_draft",
-            "speculative_step_workspace_size", "speculative_step"]
+            "speculative_step_workspace_size", "speculative_step", "moe_rmsnorm"]
 
 
 class MVError(RuntimeError):
@@ -42,7 +42,7 @@ class MoeShape(ctypes.Structure):
 
 class MoeWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("w_router", "router_bias", "w_gate", "w_up", "w_down",
-                                                "ws_gate", "ws_up", "ws_down")]
+                                                "ws_gate", "ws_up", "ws_down", "norm_gain")]
 
 
 DRAFT_KEYS = ("w_emb", "g_hidden", "g_embed", "w_proj", "w_gate", "w_up", "w_down")
@@ -68,6 +68,7 @@ def lib():
         sig = {
             "moe_router_topk": (i32, [P, i32, S, P, P, P, P, P]),
             "moe_expert_permute": (i32, [P, i32, i32, i32, P, P, P, P, P]),
+            "moe_rmsnorm": (i32, [P, i32, i32, P, P, P]),
             "moe_ffn_workspace_size": (sz, [i32, S]),
             "moe_ffn_forward": (i32, [P, i32, S, W, P, P, P, P, P, sz, P]),
             "lm_head_workspace_size": (sz, [i32, i32]),
@@ -146,7 +147,7 @@ class LayerWeights:
 
     def __init__(self, layer: dict, device="cuda"):
         self.t = {}
-        for n in ("w_router", "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down"):
+        for n in ("w_router", "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down", "norm_gain"):
             v = layer.get(n)
             self.t[n] = None if v is None else (v if isinstance(v, torch.Tensor) else bf16_to_device(v, device))
         b = layer.get("router_bias")
@@ -154,6 +155,15 @@ class LayerWeights:
             b if isinstance(b, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(b, np.float32)).to(device))
         self.c = MoeWeights(*[None if self.t[n] is None else self.t[n].data_ptr()
                               for n, _ in MoeWeights._fields_])
+
+
+def moe_rmsnorm(x, gain, out=None, stream=None):
+    """bf16((x * s) * gain) per row, s = 1 / sqrt(mean(x^2) + 1e-6) (the
+    pre-RMSNorm layer variant's input)."""
+    T, H = x.shape
+    out = torch.empty_like(x) if out is None else out
+    _check(lib().moe_rmsnorm(_p(x), T, H, _p(gain), _p(out), _stream(stream)))
+    return out
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:

@@ -71,12 +71,13 @@ enum Kind {
   KIND_DRAFT_GEMM,
   KIND_DRAFT_LM,
   KIND_DRAFT_STEP,
+  KIND_RMSNORM,
   KIND_COUNT
 };
 const char* kKindNames[KIND_COUNT] = {"router_topk",       "expert_permute",     "grouped_moe_gemm",
                                       "combine_unpermute", "combine_route",      "lm_head_gemm_argmax",
                                       "lm_argmax_finalize", "greedy_accept",     "draft_block_gemm",
-                                      "draft_lm_head_argmax", "draft_step"};
+                                      "draft_lm_head_argmax", "draft_step", "rmsnorm"};
 
 struct ProfRec {
   int kind;
@@ -243,6 +244,7 @@ mv_status check_weights(const mv_moe_weights* w, const mv_moe_shape* s) {
     MV_TRY(check_ptr(w->ws_up, "ws_up"));
     MV_TRY(check_ptr(w->ws_down, "ws_down"));
   }
+  MV_TRY(check_ptr(w->norm_gain, "norm_gain", true));
   return MV_OK;
 }
 
@@ -708,6 +710,19 @@ mv_status moe_expert_permute(const int32_t* topk_idx, int32_t T, int32_t E, int3
   return e == cudaSuccess ? MV_OK : cuda_fail(e, "expert_permute launch");
 }
 
+mv_status moe_rmsnorm(const uint16_t* x, int32_t T, int32_t H, const uint16_t* gain, uint16_t* out,
+                      mv_stream_t stream) {
+  if (T < 0 || H <= 0) return fail(MV_ERR_INVALID_ARG, "bad sizes T=%d H=%d", T, H);
+  if (H % 8) return fail(MV_ERR_UNSUPPORTED_SHAPE, "H=%d must be a multiple of 8", H);
+  MV_TRY(check_ptr(x, "x", T == 0));
+  MV_TRY(check_ptr(gain, "gain"));
+  MV_TRY(check_ptr(out, "out", T == 0));
+  if (T > 0 && out == x) return fail(MV_ERR_INVALID_ARG, "out may not alias x");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = run_kernel(KIND_RMSNORM, st, [&] { return mv::launch_rmsnorm(x, T, H, gain, out, st); });
+  return e == cudaSuccess ? MV_OK : cuda_fail(e, "rmsnorm launch");
+}
+
 size_t moe_ffn_workspace_size(int32_t T, const mv_moe_shape* shape) {
   if (!shape || T < 0) return 0;
   Carve c{nullptr};
@@ -801,6 +816,7 @@ size_t verify_step_workspace_size(int32_t B, int32_t K, const mv_moe_shape* shap
   c.take<uint64_t>(static_cast<size_t>(lm_parts_alloc(V)) * T);
   c.take<char>(kSchedBytes * (kMaxLayers + 1));
   carve_ffn(c, T, *shape, use_slabs(T, *shape));
+  c.take<uint16_t>(static_cast<size_t>(T) * shape->H);  // normalised rows (pre-RMSNorm layers)
   return kHeader + c.off + 1024;
 }
 
@@ -845,6 +861,7 @@ static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts,
   int* sched = c.take<int>(static_cast<size_t>(mv::kSchedInts) * (kMaxLayers + 1));
   const bool slabs = use_slabs(T, *shape);
   FfnWs fw = carve_ffn(c, T, *shape, slabs);
+  uint16_t* xn_buf = c.take<uint16_t>(static_cast<size_t>(T) * shape->H);  // RMSNorm(h) * g of the current layer
   cudaError_t e0 = cudaMemsetAsync(sched, 0, kSchedBytes * (n_layers + 1), st);
   if (e0 != cudaSuccess) return cuda_fail(e0, "clearing the scheduling state");
   auto slab_counts = [&](int l) -> int32_t* {
@@ -856,9 +873,19 @@ static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts,
   // the batch is decode-sized; otherwise as its own kernel before the router.
   // Decode-sized batches also group the routed rows by expert in that kernel
   // (slab layout) instead of a permute launch.
+  // A layer with a norm gain (the pre-RMSNorm variant) routes and runs its
+  // experts on xn_buf = bf16(RMSNorm(h) * g), written by the routing kernel
+  // (or by the RMSNorm kernel when the routing is not fused), and keeps the
+  // residual h.
   const bool fused = mv::combine_route_supported(static_cast<int>(T), shape->H, shape->E);
   const uint16_t* h = hidden;
-  if (n_layers > 0 && slabs) {
+  auto rmsnorm = [&](const uint16_t* src, const uint16_t* g) -> mv_status {
+    cudaError_t e = run_kernel(KIND_RMSNORM, st, [&] {
+      return mv::launch_rmsnorm(src, static_cast<int>(T), shape->H, g, xn_buf, st);
+    });
+    return e == cudaSuccess ? MV_OK : cuda_fail(e, "rmsnorm launch");
+  };
+  if (n_layers > 0 && fused) {
     cudaError_t e = run_kernel(KIND_ROUTER, st, [&] {
       mv::CombineRouteArgs a{};
       a.x = h;
@@ -876,12 +903,16 @@ static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts,
       a.inv_out = slab_inv(0);
       a.x_slab = fw.x_perm;
       a.slab_rows = static_cast<int>(T);
+      a.norm_gain = layers[0].norm_gain;
+      a.xn_out = xn_buf;
       return mv::launch_combine_route(a, st);
     });
     if (e != cudaSuccess) return cuda_fail(e, "router_topk launch");
   } else if (n_layers > 0) {
-    MV_TRY(route_impl(h, static_cast<int>(T), *shape, layers[0].w_router, layers[0].router_bias, idx_buf, tw_buf, err,
-                      st, moe_first_wave(*shape, layers[0], kPrefetchBudget)));
+    if (layers[0].norm_gain) MV_TRY(rmsnorm(h, layers[0].norm_gain));
+    MV_TRY(route_impl(layers[0].norm_gain ? xn_buf : h, static_cast<int>(T), *shape, layers[0].w_router,
+                      layers[0].router_bias, idx_buf, tw_buf, err, st,
+                      moe_first_wave(*shape, layers[0], kPrefetchBudget)));
   }
   for (int l = 0; l < n_layers; ++l) {
     const mv_moe_weights& w = layers[l];
@@ -889,7 +920,8 @@ static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts,
     float* tw = tw_buf + (l & 1) * tk;
     uint16_t* next = hbuf[l & 1];
     const bool last = (l + 1 == n_layers);
-    MV_TRY(ffn_forward_impl(h, static_cast<int>(T), *shape, w, idx, tw, h, next, fw, err,
+    const uint16_t* x_in = w.norm_gain ? xn_buf : h;
+    MV_TRY(ffn_forward_impl(x_in, static_cast<int>(T), *shape, w, idx, tw, h, next, fw, err,
                             sched + static_cast<size_t>(l) * mv::kSchedInts, st, last || !fused,
                             last ? lm_first_wave(w_lm, V, shape->H, kPrefetchBudget) : mv::L2Prefetch{},
                             slab_counts(l), slab_inv(l)));
@@ -922,11 +954,15 @@ static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts,
           a.inv_out = slab_inv(l + 1);
           a.x_slab = fw.x_perm;
           a.slab_rows = static_cast<int>(T);
+          a.norm_gain = wn.norm_gain;
+          a.xn_out = xn_buf;
           return mv::launch_combine_route(a, st);
         });
         if (e != cudaSuccess) return cuda_fail(e, "combine_route launch");
       } else {
-        MV_TRY(route_impl(next, static_cast<int>(T), *shape, wn.w_router, wn.router_bias, idx_n, tw_n, err, st));
+        if (wn.norm_gain) MV_TRY(rmsnorm(next, wn.norm_gain));
+        MV_TRY(route_impl(wn.norm_gain ? xn_buf : next, static_cast<int>(T), *shape, wn.w_router, wn.router_bias,
+                          idx_n, tw_n, err, st));
       }
     }
     h = next;

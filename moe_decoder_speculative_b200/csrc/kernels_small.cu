@@ -354,10 +354,12 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
     uint16_t* __restrict__ out, int T, int H, int E, int k, const uint16_t* __restrict__ wr,
     const float* __restrict__ bias, int32_t* __restrict__ idx, float* __restrict__ wout, int* err,
     const L2Prefetch pf, int32_t* __restrict__ slab_counts, int32_t* __restrict__ inv_out,
-    uint16_t* __restrict__ x_slab, int slab_rows) {
+    uint16_t* __restrict__ x_slab, int slab_rows, const uint16_t* __restrict__ norm_gain,
+    uint16_t* __restrict__ xn_out) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ int32_t sel_s[R * 8];  // the experts each row selected
   __shared__ int32_t pos_s[R * 8];  // their slab rows (-1: skipped)
+  __shared__ float nred[R][16];     // RMSNorm partial sums, one per warp
   uint16_t* hs = reinterpret_cast<uint16_t*>(sm);                         // [R][H]
   float* ls = reinterpret_cast<float*>(hs + static_cast<size_t>(R) * H);  // [R][E]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -438,6 +440,46 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
     reinterpret_cast<uint4*>(hs + static_cast<size_t>(r) * H)[c] = o;
   }
   __syncthreads();
+
+  // (1b) pre-RMSNorm variant: the router and the experts take
+  //      x = bf16((h * s) * g), s = 1 / sqrt(sum(h^2) / H + eps); the rows are
+  //      normalised in shared memory and written to xn_out (the shared
+  //      expert's input); the combined rows written above stay the residual.
+  if (norm_gain) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float ss = 0.f;
+      for (int c = tid; c < hv; c += blockDim.x) {
+        float f[8];
+        bf16x8_to_f32(reinterpret_cast<const uint4*>(hs + static_cast<size_t>(r) * H)[c], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = __fadd_rn(ss, __fmul_rn(f[i], f[i]));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+      if (lane == 0) nred[r][warp] = ss;
+    }
+    __syncthreads();
+    for (int i = tid; i < R * hv; i += blockDim.x) {
+      const int r = i / hv, c = i % hv;
+      if (r >= nrows) continue;
+      float tot = 0.f;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot = __fadd_rn(tot, nred[r][w]);
+      const float sc = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot, static_cast<float>(H)), kRmsNormEps)));
+      float f[8], g[8];
+      bf16x8_to_f32(reinterpret_cast<const uint4*>(hs + static_cast<size_t>(r) * H)[c], f);
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(norm_gain) + c), g);
+      uint32_t ow[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        ow[q] = static_cast<uint32_t>(f32_to_bf16_bits(__fmul_rn(__fmul_rn(f[2 * q], sc), g[2 * q]))) |
+                (static_cast<uint32_t>(f32_to_bf16_bits(__fmul_rn(__fmul_rn(f[2 * q + 1], sc), g[2 * q + 1]))) << 16);
+      const uint4 o = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      reinterpret_cast<uint4*>(hs + static_cast<size_t>(r) * H)[c] = o;
+      reinterpret_cast<uint4*>(xn_out + static_cast<size_t>(row0 + r) * H)[c] = o;
+    }
+    __syncthreads();
+  }
 
   // (2) router logits: warp w owns experts w, w+16, w+32, w+48 (one batch of
   //     loads for E <= 64); each x vector is converted once and reused.
@@ -534,7 +576,8 @@ static cudaError_t launch_combine_route_rv(const CombineRouteArgs& a, cudaStream
   const int grid = rows_ctas > prefetch_ctas(a.pf) ? rows_ctas : prefetch_ctas(a.pf);  // extra CTAs only prefetch
   return launch_pdl(combine_route_kernel<R, NV>, dim3(grid), dim3(512), smem, s, a.x, a.y_perm, a.y_sh, a.inv,
                     a.w_prev, a.k_prev, a.n_pos > 0 ? a.n_pos : a.T * a.k_prev, a.out, a.T, a.H, a.E, a.k, a.wr,
-                    a.bias, a.idx, a.w, a.err, a.pf, a.slab_counts, a.inv_out, a.x_slab, a.slab_rows);
+                    a.bias, a.idx, a.w, a.err, a.pf, a.slab_counts, a.inv_out, a.x_slab, a.slab_rows, a.norm_gain,
+                    a.xn_out);
 }
 
 // Larger batches route with the shared-memory-staged router instead (each of
@@ -965,6 +1008,53 @@ cudaError_t launch_lm_finalize(const uint64_t* keys, int nparts, int ld, int T, 
                                cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   return launch_pdl(lm_finalize_kernel, dim3(T), dim3(128), 0, s, keys, nparts, ld, T, argmax);
+}
+
+// ---------------------------------------------------------------------------
+// RMSNorm of T rows (the pre-RMSNorm layer variant): one CTA of 256 threads
+// per row, out = bf16((x * s) * g), s = 1 / sqrt(sum(x^2) / H + eps), with the
+// products and sums singly rounded.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* __restrict__ x, int H,
+                                                      const uint16_t* __restrict__ gain, uint16_t* __restrict__ out) {
+  __shared__ float red[8];
+  pdl_trigger();
+  pdl_wait();
+  const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(r) * H);
+  const int hv = H / 8;
+  float ss = 0.f;
+  for (int c = tid; c < hv; c += 256) {
+    float f[8];
+    bf16x8_to_f32(xr[c], f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss = __fadd_rn(ss, __fmul_rn(f[i], f[i]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+  if (lane == 0) red[wid] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) tot = __fadd_rn(tot, red[w]);
+  const float sc = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot, static_cast<float>(H)), kRmsNormEps)));
+  uint4* orow = reinterpret_cast<uint4*>(out + static_cast<size_t>(r) * H);
+  for (int c = tid; c < hv; c += 256) {
+    float f[8], g[8];
+    bf16x8_to_f32(xr[c], f);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(gain) + c), g);
+    uint32_t ow[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      ow[q] = static_cast<uint32_t>(f32_to_bf16_bits(__fmul_rn(__fmul_rn(f[2 * q], sc), g[2 * q]))) |
+              (static_cast<uint32_t>(f32_to_bf16_bits(__fmul_rn(__fmul_rn(f[2 * q + 1], sc), g[2 * q + 1]))) << 16);
+    orow[c] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+  }
+}
+
+cudaError_t launch_rmsnorm(const uint16_t* x, int T, int H, const uint16_t* gain, uint16_t* out, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  return launch_pdl(rmsnorm_kernel, dim3(T), dim3(256), 0, s, x, H, gain, out);
 }
 
 // ---------------------------------------------------------------------------

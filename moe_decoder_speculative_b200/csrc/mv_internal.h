@@ -77,7 +77,13 @@ struct CombineRouteArgs {
   int32_t* inv_out;
   uint16_t* x_slab;
   int slab_rows;
+  // Pre-RMSNorm variant, or nullptr: the rows are routed (and placed) as
+  // bf16(RMSNorm(row) * norm_gain), also written to xn_out [T][H].
+  const uint16_t* norm_gain;
+  uint16_t* xn_out;
 };
+constexpr float kRmsNormEps = 1e-6f;
+cudaError_t launch_rmsnorm(const uint16_t* x, int T, int H, const uint16_t* gain, uint16_t* out, cudaStream_t s);
 bool combine_route_supported(int T, int H, int E);
 cudaError_t launch_combine_route(const CombineRouteArgs& a, cudaStream_t s);
 cudaError_t launch_router(const uint16_t* x, int T, int H, int E, int k, const uint16_t* wr,
