@@ -822,11 +822,12 @@ size_t verify_step_workspace_size(int32_t B, int32_t K, const mv_moe_shape* shap
 
 // The verify step; *h_final (when given) receives the device address of the
 // last layer's hidden rows (inside the workspace, or `hidden` with no layers).
-static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts, int32_t B, int32_t K,
-                                  const mv_moe_shape* shape, const mv_moe_weights* layers, int32_t n_layers,
-                                  const uint16_t* w_lm, int32_t V, int32_t* accepted, int32_t* next_token,
-                                  int32_t* emitted, int32_t* argmax, void* ws, size_t ws_bytes, mv_stream_t stream,
-                                  const uint16_t** h_final) {
+// The host-side argument checks of verify_step (shared with the graph
+// executor, which must reject bad arguments before touching the GPU).
+static mv_status verify_step_check(const uint16_t* hidden, const int32_t* drafts, int32_t B, int32_t K,
+                                   const mv_moe_shape* shape, const mv_moe_weights* layers, int32_t n_layers,
+                                   const uint16_t* w_lm, int32_t V, int32_t* accepted, int32_t* next_token,
+                                   int32_t* emitted, int32_t* argmax, void* ws, size_t ws_bytes) {
   MV_TRY(check_shape(shape));
   if (B < 0 || K < 0 || K > 32 || n_layers < 0 || n_layers > kMaxLayers || V <= 0)
     return fail(MV_ERR_INVALID_ARG, "bad sizes B=%d K=%d (K <= 32) n_layers=%d (<= %d) V=%d", B, K, n_layers,
@@ -847,6 +848,17 @@ static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts,
   const size_t need = verify_step_workspace_size(B, K, shape, V);
   if (ws_bytes < need)
     return fail(MV_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+  return MV_OK;
+}
+
+static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts, int32_t B, int32_t K,
+                                  const mv_moe_shape* shape, const mv_moe_weights* layers, int32_t n_layers,
+                                  const uint16_t* w_lm, int32_t V, int32_t* accepted, int32_t* next_token,
+                                  int32_t* emitted, int32_t* argmax, void* ws, size_t ws_bytes, mv_stream_t stream,
+                                  const uint16_t** h_final) {
+  MV_TRY(verify_step_check(hidden, drafts, B, K, shape, layers, n_layers, w_lm, V, accepted, next_token, emitted,
+                           argmax, ws, ws_bytes));
+  const int64_t T = int64_t(B) * (K + 1);
   if (B == 0) return MV_OK;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -1240,6 +1252,8 @@ mv_status verify_graph_create(const uint16_t* hidden, const int32_t* drafts, int
   if (!graph) return fail(MV_ERR_INVALID_ARG, "graph out-parameter is NULL");
   *graph = nullptr;
   if (g_prof_on.load()) return fail(MV_ERR_INVALID_ARG, "profiling is on: its events cannot be recorded into a graph");
+  MV_TRY(verify_step_check(hidden, drafts, B, K, shape, layers, n_layers, w_lm, V, accepted, next_token, emitted,
+                           argmax, ws, ws_bytes));
   cudaStream_t cs = nullptr;
   cudaError_t e = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking);
   if (e != cudaSuccess) return cuda_fail(e, "creating the recording stream");
