@@ -433,7 +433,7 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
     mv::GemmSet& S = p.set[ns++];
     base(S, down_mode, down_epi);
     S.m_tile = down_tile;
-    MV_TRY(tmap(&S.a0, w.ws_down, H, Ish, 128));
+    MV_TRY(tmap(&S.a0, w.ws_down, H, Ish, decode ? 128 : 256));  // MODE_TPAIR: one 256-row box
     MV_TRY(tmap(&S.b, ws.a_sh, T, Ish, bbox));
     S.a1 = S.a0;
     S.out = ws.y_sh;
@@ -449,7 +449,7 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
     mv::GemmSet& S = p.set[ns++];
     base(S, down_mode, down_epi);
     S.m_tile = down_tile;
-    MV_TRY(tmap(&S.a0, w.w_down, static_cast<uint64_t>(E) * H, I, 128));
+    MV_TRY(tmap(&S.a0, w.w_down, static_cast<uint64_t>(E) * H, I, decode ? 128 : 256));
     MV_TRY(tmap(&S.b, ws.a_perm, ws.n_pos, I, bbox));
     S.a1 = S.a0;
     S.out = ws.y_perm;
@@ -606,7 +606,7 @@ mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, in
   int64_t units = 0;
   if (V0 > 0) {
     mv::GemmSet& S = p.set[ns++];
-    MV_TRY(tmap(&S.a0, w_lm, V0, H, 128));
+    MV_TRY(tmap(&S.a0, w_lm, V0, H, 256));  // MODE_MPAIR: both 128-row halves in one box
     MV_TRY(tmap(&S.b, h, T, H, bbox));
     S.a1 = S.a0;
     set_up(S, w_lm, V0, 0, 0, true);
