@@ -132,8 +132,9 @@ struct TmKey {
   const void* ptr;
   uint64_t rows, cols;
   uint32_t box_rows;
+  uint32_t rank;  // 2: [rows][cols] tiles; 3: [k-block][rows][64] view, two k-blocks per box
   bool operator==(const TmKey& o) const {
-    return ptr == o.ptr && rows == o.rows && cols == o.cols && box_rows == o.box_rows;
+    return ptr == o.ptr && rows == o.rows && cols == o.cols && box_rows == o.box_rows && rank == o.rank;
   }
 };
 struct TmHash {
@@ -142,6 +143,7 @@ struct TmHash {
     h ^= (k.rows * 0x9E3779B97F4A7C15ull) + (h << 6) + (h >> 2);
     h ^= (k.cols * 0xC2B2AE3D27D4EB4Full) + (h << 6) + (h >> 2);
     h ^= k.box_rows + (h << 6) + (h >> 2);
+    h ^= k.rank + (h << 6) + (h >> 2);
     return h;
   }
 };
@@ -162,8 +164,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 std::mutex g_tm_mu;
 std::unordered_map<TmKey, CUtensorMap, TmHash> g_tm_cache;
 
-mv_status tmap(CUtensorMap* out, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  TmKey key{ptr, rows, cols, box_rows};
+mv_status tmap_rank(CUtensorMap* out, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                    uint32_t rank) {
+  TmKey key{ptr, rows, cols, box_rows, rank};
   {
     std::lock_guard<std::mutex> lk(g_tm_mu);
     auto it = g_tm_cache.find(key);
@@ -176,13 +179,26 @@ mv_status tmap(CUtensorMap* out, const void* ptr, uint64_t rows, uint64_t cols, 
   if (!fn) return fail(MV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   CUtensorMap m;
   std::memset(&m, 0, sizeof(m));
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {64, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r;
+  if (rank == 3) {
+    // element (x, y, z) = row y, column 64 z + x: each box is two consecutive
+    // 64-wide k-blocks of box_rows rows, stored k-block after k-block
+    const cuuint64_t dims[3] = {64, rows, cols / 64};
+    const cuuint64_t strides[2] = {cols * 2, 128};
+    const cuuint32_t box[3] = {64, box_rows, 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
   if (r != CUDA_SUCCESS)
     return fail(MV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for [%llu x %llu] box %u", static_cast<int>(r),
                 static_cast<unsigned long long>(rows), static_cast<unsigned long long>(cols), box_rows);
@@ -191,6 +207,16 @@ mv_status tmap(CUtensorMap* out, const void* ptr, uint64_t rows, uint64_t cols, 
   g_tm_cache[key] = m;
   *out = m;
   return MV_OK;
+}
+
+mv_status tmap(CUtensorMap* out, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  return tmap_rank(out, ptr, rows, cols, box_rows, 2);
+}
+
+// The weights-on-M GEMM tiles (GEMM_MOE_DECODE) read every operand through 3D
+// maps, two k-blocks per box.
+mv_status tmap3(CUtensorMap* out, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  return tmap_rank(out, ptr, rows, cols, box_rows, 3);
 }
 
 // ---------------------------------------------------------------------------
@@ -387,12 +413,15 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
   };
   const bool tokm = !decode;  // large groups: tokens on the MMA's M side
   const int bbox = decode ? mv::kDecodeBBox : mv::kPrefillBBox;
+  auto map = [decode](CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box) {
+    return decode ? tmap3(m, ptr, rows, cols, box) : tmap(m, ptr, rows, cols, box);
+  };
   if (Ish > 0) {  // shared expert, gate/up
     mv::GemmSet& S = p.set[ns];
     base(S, tokm ? mv::MODE_TGATEUP : mv::MODE_GATEUP, tokm ? mv::EPI_SWIGLU_ROWS : mv::EPI_SWIGLU);
-    MV_TRY(tmap(&S.a0, w.ws_gate, Ish, H, 128));
-    MV_TRY(tmap(&S.a1, w.ws_up, Ish, H, 128));
-    MV_TRY(tmap(&S.b, x, T, H, bbox));
+    MV_TRY(map(&S.a0, w.ws_gate, Ish, H, 128));
+    MV_TRY(map(&S.a1, w.ws_up, Ish, H, 128));
+    MV_TRY(map(&S.b, x, T, H, bbox));
     S.out = ws.a_sh;
     S.ld_out = Ish;
     S.K = H;
@@ -406,9 +435,9 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
   {  // routed experts, gate/up
     mv::GemmSet& S = p.set[ns];
     base(S, tokm ? mv::MODE_TGATEUP : mv::MODE_GATEUP, tokm ? mv::EPI_SWIGLU_ROWS : mv::EPI_SWIGLU);
-    MV_TRY(tmap(&S.a0, w.w_gate, static_cast<uint64_t>(E) * I, H, 128));
-    MV_TRY(tmap(&S.a1, w.w_up, static_cast<uint64_t>(E) * I, H, 128));
-    MV_TRY(tmap(&S.b, ws.x_perm, ws.n_pos, H, bbox));
+    MV_TRY(map(&S.a0, w.w_gate, static_cast<uint64_t>(E) * I, H, 128));
+    MV_TRY(map(&S.a1, w.w_up, static_cast<uint64_t>(E) * I, H, 128));
+    MV_TRY(map(&S.b, ws.x_perm, ws.n_pos, H, bbox));
     S.out = ws.a_perm;
     S.ld_out = I;
     S.K = H;
@@ -433,8 +462,8 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
     mv::GemmSet& S = p.set[ns++];
     base(S, down_mode, down_epi);
     S.m_tile = down_tile;
-    MV_TRY(tmap(&S.a0, w.ws_down, H, Ish, decode ? 128 : 256));  // MODE_TPAIR: one 256-row box
-    MV_TRY(tmap(&S.b, ws.a_sh, T, Ish, bbox));
+    MV_TRY(map(&S.a0, w.ws_down, H, Ish, decode ? 128 : 256));  // MODE_TPAIR: one 256-row box
+    MV_TRY(map(&S.b, ws.a_sh, T, Ish, bbox));
     S.a1 = S.a0;
     S.out = ws.y_sh;
     S.ld_out = H;
@@ -449,8 +478,8 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
     mv::GemmSet& S = p.set[ns++];
     base(S, down_mode, down_epi);
     S.m_tile = down_tile;
-    MV_TRY(tmap(&S.a0, w.w_down, static_cast<uint64_t>(E) * H, I, decode ? 128 : 256));
-    MV_TRY(tmap(&S.b, ws.a_perm, ws.n_pos, I, bbox));
+    MV_TRY(map(&S.a0, w.w_down, static_cast<uint64_t>(E) * H, I, decode ? 128 : 256));
+    MV_TRY(map(&S.b, ws.a_perm, ws.n_pos, I, bbox));
     S.a1 = S.a0;
     S.out = ws.y_perm;
     S.ld_out = H;
@@ -1060,9 +1089,9 @@ mv_status draft_gemm_impl(const uint16_t* u, int B, int H, const mv_draft_weight
   P.epi = mv::EPI_STORE_BF16;
   P.m_tile = 128;
   P.dep_set = -1;
-  MV_TRY(tmap(&P.a0, d.w_proj, H, 2 * static_cast<uint64_t>(H), 128));
+  MV_TRY(tmap3(&P.a0, d.w_proj, H, 2 * static_cast<uint64_t>(H), 128));
   P.a1 = P.a0;
-  MV_TRY(tmap(&P.b, u, B, 2 * static_cast<uint64_t>(H), bbox));
+  MV_TRY(tmap3(&P.b, u, B, 2 * static_cast<uint64_t>(H), bbox));
   P.out = z;
   P.ld_out = H;
   P.K = 2 * H;
@@ -1075,9 +1104,9 @@ mv_status draft_gemm_impl(const uint16_t* u, int B, int H, const mv_draft_weight
   G.epi = mv::EPI_SWIGLU;
   G.m_tile = 128;
   G.dep_set = 0;
-  MV_TRY(tmap(&G.a0, d.w_gate, Id, H, 128));
-  MV_TRY(tmap(&G.a1, d.w_up, Id, H, 128));
-  MV_TRY(tmap(&G.b, z, B, H, bbox));
+  MV_TRY(tmap3(&G.a0, d.w_gate, Id, H, 128));
+  MV_TRY(tmap3(&G.a1, d.w_up, Id, H, 128));
+  MV_TRY(tmap3(&G.b, z, B, H, bbox));
   G.out = a;
   G.ld_out = Id;
   G.K = H;
@@ -1090,9 +1119,9 @@ mv_status draft_gemm_impl(const uint16_t* u, int B, int H, const mv_draft_weight
   D.epi = mv::EPI_STORE_BF16;
   D.m_tile = 128;
   D.dep_set = 1;
-  MV_TRY(tmap(&D.a0, d.w_down, H, Id, 128));
+  MV_TRY(tmap3(&D.a0, d.w_down, H, Id, 128));
   D.a1 = D.a0;
-  MV_TRY(tmap(&D.b, a, B, Id, bbox));
+  MV_TRY(tmap3(&D.b, a, B, Id, bbox));
   D.out = hout;
   D.res = z;
   D.ld_out = H;

@@ -22,7 +22,7 @@ enum { GEMM_MOE_DECODE = 0, GEMM_MOE_PREFILL = 1, GEMM_LM = 2, GEMM_LM_WIDE = 3 
 #ifndef MV_PREFILL_BBOX
 #define MV_PREFILL_BBOX 128
 #endif
-constexpr int kDecodeBBox = 16;
+constexpr int kDecodeBBox = 32;  // GEMM_MOE_DECODE: one 3D box of 32 token rows x two k-blocks
 constexpr int kPrefillBBox = MV_PREFILL_BBOX;
 constexpr int kLmBBox = 16;       // GEMM_LM: few token rows
 constexpr int kLmWideBBox = 128;  // GEMM_LM_WIDE: 128 or more token rows

@@ -83,7 +83,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   constexpr int kBBox = BBOX;  // B rows per TMA box (the B tensor maps are built with this box height)
   static_assert(BBOX % 8 == 0 && BBOX <= BN, "BBOX");
   constexpr int B_TILE_BYTES = BN * 128;
-  constexpr int STAGE_BYTES = 2 * kATileBytes + NB * B_TILE_BYTES;
+  // Weights-on-M tiles (BN = 32) take two k-blocks per stage through 3D tensor
+  // maps: one TMA instruction brings both k-blocks of a 128-row weight tile
+  // (or of the token rows).  A TMA instruction costs about 0.25 us of the SM's
+  // copy engine whatever its size, which bounds one SM's stream when only a
+  // few SMs have work (batch 1, the draft block).  Stage layout: A0 [kb0][kb1],
+  // A1 (the up weights) [kb0][kb1], B [kb0][kb1].
+  constexpr bool kKB2 = !LM && BN == 32;
+  static_assert(!kKB2 || NB == 2, "two B slots per stage");
+  constexpr int STAGE_BYTES = (kKB2 ? 4 : 2) * kATileBytes + NB * B_TILE_BYTES;
   constexpr int ACC_COLS = 2 * BN;  // two accumulators (D0, D1) per slot
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 128, "BN");
   static_assert(2 * ACC_COLS <= 512, "TMEM");
@@ -104,7 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   __shared__ int g_begin[kMaxGroups + 1];  // first unit of each group
   __shared__ int g_rows[kMaxGroups];
   __shared__ int g_row0[kMaxGroups];
-  __shared__ int g_nt[kMaxGroups];
+  __shared__ short g_nt[kMaxGroups];
   __shared__ unsigned char g_set[kMaxGroups];
   __shared__ short g_gi[kMaxGroups];
   __shared__ int set_base[5];
@@ -170,7 +178,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const int nchunk = (ui.nvalid + kBBox - 1) / kBBox;
     const uint32_t b_bytes = nchunk * kBBox * 128;
     const int kblocks = S.K / 64;
-    if (S.mode == MODE_KPAIR) {
+    if (kKB2) {
+      const int kb0 = 2 * ks;
+      const bool gu = (S.mode == MODE_GATEUP);
+      if (wts) {
+        mbar_arrive_expect_tx(&full_bar[stg], (gu ? 4u : 2u) * kATileBytes + 2u * B_TILE_BYTES);
+        tma_load_3d(st, &S.a0, 0, a_row0, kb0, &full_bar[stg], pol_w);
+        if (gu) tma_load_3d(st + 2 * kATileBytes, &S.a1, 0, a_row0, kb0, &full_bar[stg], pol_w);
+      }
+      if (toks) tma_load_3d(st + 4 * kATileBytes, &S.b, 0, ui.b_row0, kb0, &full_bar[stg], pol_x);
+      (void)nchunk;
+      (void)b_bytes;
+    } else if (S.mode == MODE_KPAIR) {
       const int kb0 = 2 * ks;
       const bool two = kb0 + 1 < kblocks;
       uint8_t* b1 = b0 + (NB > 1 ? B_TILE_BYTES : 0);
@@ -206,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   };
   auto unit_stages = [](const GemmSet& S) {
     const int kblocks = S.K / 64;
-    return (S.mode == MODE_KPAIR) ? (kblocks + 1) / 2 : kblocks;
+    return (kKB2 || S.mode == MODE_KPAIR) ? (kblocks + 1) / 2 : kblocks;
   };
 
   // The first set, when its rows are static and it depends on nothing, gives
@@ -269,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     g_gi[g] = static_cast<short>(gi);
     const int mt = (S.M + S.m_tile - 1) / S.m_tile;
     const int nt = rows > 0 ? (rows + BN - 1) / BN : 0;
-    g_nt[g] = nt;
+    g_nt[g] = static_cast<short>(nt);
     g_begin[g + 1] = mt * nt;  // unit count, scanned below
   }
   if (tid == 0) g_begin[0] = 0;
@@ -395,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         const uint32_t idesc = tok_m ? idesc_bf16_f32(128, n_tok) : idesc_bf16_f32(128, n_mma);
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(slot * ACC_COLS);
         const int kblocks = S.K / 64;
-        const int nstage = (S.mode == MODE_KPAIR) ? (kblocks + 1) / 2 : kblocks;
+        const int nstage = unit_stages(S);
         bool ok = true;
         for (int ks = 0; ks < nstage; ++ks) {
           if (!mbar_wait(&full_bar[stage], phase, &abort_s, p.err, deadline)) {
@@ -406,7 +425,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
           const uint32_t a1 = st + kATileBytes;
           const uint32_t b0 = st + 2 * kATileBytes;
-          if (tok_m) {
+          if (kKB2) {
+            // two k-blocks: D0 += A0[h] B[h] (and D1 += A1[h] B[h] for gate/up)
+            const bool gu = (S.mode == MODE_GATEUP);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (h == 1 && 2 * ks + 1 >= kblocks) break;
+              const uint32_t ah = st + h * kATileBytes;
+              const uint32_t uh = st + (2 + h) * kATileBytes;
+              const uint32_t bh = st + 4 * kATileBytes + h * B_TILE_BYTES;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                tc_mma_bf16(d0, smem_desc_k128(ah + kk * 32), smem_desc_k128(bh + kk * 32), idesc,
+                            (ks | h | kk) != 0 ? 1u : 0u);
+              if (gu) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  tc_mma_bf16(d0 + BN, smem_desc_k128(uh + kk * 32), smem_desc_k128(bh + kk * 32), idesc,
+                              (ks | h | kk) != 0 ? 1u : 0u);
+              }
+            }
+          } else if (tok_m) {
             // A = the token rows (B slot), B = the 256 weight rows of slots 0-1
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
@@ -713,10 +752,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 // ---------------------------------------------------------------------------
 template <int BN, int STAGES, int NB, bool LM, int BBOX>
 static cudaError_t launch_gemm_impl(const GemmParams& p, int grid, cudaStream_t stream) {
-  constexpr int STAGE_BYTES = 2 * kATileBytes + NB * BN * 128;
+  constexpr int STAGE_BYTES = ((!LM && BN == 32) ? 4 : 2) * kATileBytes + NB * BN * 128;  // as in the kernel
   constexpr int EXTRA = LM ? 4 * 32 * 33 * 4 : 0;  // argmax epilogue transpose buffers
   constexpr int SMEM = STAGES * STAGE_BYTES + EXTRA + 1024;
-  static_assert(SMEM + 12 * 1024 <= 227 * 1024, "shared memory (dynamic + static)");
+  // the kernel's static shared memory is 9,216 bytes (ptxas); the opt-in limit is 227 KB
+  static_assert(SMEM + 9216 <= 227 * 1024, "shared memory (dynamic + static)");
   auto kern = gemm_tc_kernel<BN, STAGES, NB, LM, BBOX>;
   static thread_local int configured_dev = -1;
   int dev = 0;
@@ -736,7 +776,7 @@ static cudaError_t launch_gemm_impl(const GemmParams& p, int grid, cudaStream_t 
 //   GEMM_LM_WIDE      the same with 128-row token boxes, for 128 or more tokens
 cudaError_t launch_gemm(int config, const GemmParams& p, int grid, cudaStream_t stream) {
   switch (config) {
-    case GEMM_MOE_DECODE: return launch_gemm_impl<32, 5, 2, false, kDecodeBBox>(p, grid, stream);
+    case GEMM_MOE_DECODE: return launch_gemm_impl<32, 3, 2, false, kDecodeBBox>(p, grid, stream);
     case GEMM_MOE_PREFILL: return launch_gemm_impl<128, 4, 1, false, kPrefillBBox>(p, grid, stream);
     case GEMM_LM: return launch_gemm_impl<128, 4, 1, true, kLmBBox>(p, grid, stream);
     case GEMM_LM_WIDE: return launch_gemm_impl<128, 4, 1, true, kLmWideBBox>(p, grid, stream);
