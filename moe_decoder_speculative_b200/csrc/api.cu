@@ -583,6 +583,7 @@ mv_status route_impl(const uint16_t* x, int T, const mv_moe_shape& s, const uint
       a.idx = idx;
       a.w = tw;
       a.err = err;
+      a.timeout_ns = timeout_ns();
       a.pf = pf;
       return mv::launch_combine_route(a, st);
     }
@@ -939,6 +940,7 @@ static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts,
       a.idx = idx_buf;
       a.w = tw_buf;
       a.err = err;
+      a.timeout_ns = timeout_ns();
       a.pf = moe_first_wave(*shape, layers[0], kPrefetchBudget);
       a.slab_counts = slab_counts(0);
       a.inv_out = slab_inv(0);
@@ -990,6 +992,7 @@ static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts,
           a.idx = idx_n;
           a.w = tw_n;
           a.err = err;
+          a.timeout_ns = timeout_ns();
           a.pf = moe_first_wave(*shape, wn, kPrefetchBudget);
           a.slab_counts = slab_counts(l + 1);
           a.inv_out = slab_inv(l + 1);

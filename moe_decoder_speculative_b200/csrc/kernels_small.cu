@@ -54,61 +54,65 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
-// Top-k of one row's E logits (held in shared memory) by one warp: k rounds
-// of a warp argmax (larger logit wins, equal logits -> lower expert id), then
-// the renormalised softmax weights exp(l_j - l_max) / sum_selected.
-__device__ __forceinline__ void topk_select_row(const float* lrow, int E, int k, int lane,
-                                                int32_t* idx_out, float* w_out, int32_t* sel_s = nullptr) {
-  constexpr int kMaxPer = 8;  // E <= 256
-  float v[kMaxPer];
-  const int per = (E + 31) / 32;
-#pragma unroll
-  for (int q = 0; q < kMaxPer; ++q) {
-    const int e = lane + 32 * q;
-    v[q] = (q < per && e < E) ? lrow[e] : -__int_as_float(0x7f800000);
-  }
-  float selv[8];
-  int sele[8];
-  for (int j = 0; j < k; ++j) {
-    float bv = -__int_as_float(0x7f800000);
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int q = 0; q < kMaxPer; ++q) {
-      const int e = lane + 32 * q;
-      if (q < per && e < E && better(v[q], e, bv, bi)) {
-        bv = v[q];
-        bi = e;
+// Order key of a logit: larger logits give larger keys, -0 and +0 the same
+// key, and NaN the smallest key of all (below -inf), so that a NaN is only
+// ever selected when a row has fewer than k numbers.
+__device__ __forceinline__ uint32_t logit_key(float v) {
+  uint32_t u = __float_as_uint(v);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return 0u;  // NaN
+  if ((u << 1) == 0u) u = 0u;                       // -0 -> +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Top-k of `nrows` rows of E logits (shared memory, row r at ls + r * E) by
+// the whole block; every thread must call it, as it synchronises the block.
+// Selection by rank: the rank of an element is the number of elements of its
+// row that come before it in the order "larger logit first, equal logits ->
+// lower expert id first" (NaN last), and the element of rank j < k takes
+// slot j, so the slots are in descending logit order.  Eight consecutive
+// threads share one element, each comparing it with an eighth of the row,
+// and add their counts with shuffles.  Then warp r writes row r's slots: ids,
+// and the renormalised softmax weights exp(l_j - l_0) / sum_{i<k}
+// exp(l_i - l_0), the sum taken in slot order.  slot_s holds 8 entries per
+// row (k <= 8) and keeps the selected ids for the caller.
+__device__ void topk_rows_block(const float* ls, int E, int k, int nrows, int32_t* slot_s,
+                                int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int chunk = (E + 7) >> 3;
+  const int items = nrows * E * 8;
+  for (int base = 0; base < items; base += blockDim.x) {  // uniform trip count: shuffles see full warps
+    const int it = base + tid;
+    const int q = it >> 3, sub = it & 7;
+    int cnt = 0, e = 0;
+    const float* lr = ls;
+    if (it < items) {
+      const int r = q / E;
+      e = q - r * E;
+      lr = ls + r * E;
+      const uint32_t ke = logit_key(lr[e]);
+      const int i1 = min(E, (sub + 1) * chunk);
+      for (int i = sub * chunk; i < i1; ++i) {
+        const uint32_t ki = logit_key(lr[i]);
+        cnt += (ki > ke || (ki == ke && i < e)) ? 1 : 0;
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (better(ov, oi, bv, bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    selv[j] = bv;
-    sele[j] = bi;
-#pragma unroll
-    for (int q = 0; q < kMaxPer; ++q)
-      if (lane + 32 * q == bi) v[q] = -__int_as_float(0x7f800000);
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, 1);
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, 2);
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, 4);
+    if (it < items && sub == 0 && cnt < k) slot_s[(q / E) * 8 + cnt] = e;
   }
-  const float mx = selv[0];
-  float s = 0.f;
-  for (int j = 0; j < k; ++j) s += expf(selv[j] - mx);
-  if (lane < k) {
-    float my_v = selv[0];
-    int my_e = sele[0];
-    for (int j = 1; j < k; ++j)
-      if (j == lane) {
-        my_v = selv[j];
-        my_e = sele[j];
-      }
-    idx_out[lane] = my_e;
-    w_out[lane] = expf(my_v - mx) / s;
-    if (sel_s) sel_s[lane] = my_e;
+  __syncthreads();
+  for (int r = tid >> 5; r < nrows; r += blockDim.x >> 5) {
+    if (lane < k) {
+      const float* lr = ls + r * E;
+      const int32_t* sl = slot_s + r * 8;
+      const float mx = lr[sl[0]];
+      float s = 0.f;
+      for (int j = 0; j < k; ++j) s += expf(lr[sl[j]] - mx);
+      const int e = sl[lane];
+      idx_out[r * k + lane] = e;
+      w_out[r * k + lane] = expf(lr[e] - mx) / s;
+    }
   }
 }
 
@@ -121,7 +125,7 @@ __device__ __forceinline__ void topk_select_row(const float* lrow, int E, int k,
 // over all E restricted to the kept experts and renormalised.
 // A CTA of 8 warps owns R rows: the rows sit in shared memory, warp w computes
 // experts w, w+8, ... for all R rows (each router weight row is read once per
-// CTA, 16-byte loads), then warp r < R selects the top-k of row r.
+// CTA, 16-byte loads), then the block selects the top-k of its rows by rank.
 // ---------------------------------------------------------------------------
 template <int R>
 __global__ void __launch_bounds__(256) router_topk_kernel(const uint16_t* __restrict__ x, int T,
@@ -133,6 +137,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const uint16_t* __rest
   extern __shared__ __align__(128) uint8_t sm[];
   uint16_t* xs = reinterpret_cast<uint16_t*>(sm);                        // [R][H]
   float* ls = reinterpret_cast<float*>(sm + static_cast<size_t>(R) * H * 2);  // [R][E]
+  __shared__ int32_t slot_s[R * 8];
   pdl_trigger();
   pdl_wait();
   const int row0 = blockIdx.x * R;
@@ -174,9 +179,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const uint16_t* __rest
   }
   __syncthreads();
 
-  if (warp < nrows)
-    topk_select_row(ls + warp * E, E, k, lane, idx + static_cast<size_t>(row0 + warp) * k,
-                    wout + static_cast<size_t>(row0 + warp) * k);
+  topk_rows_block(ls, E, k, nrows, slot_s, idx + static_cast<size_t>(row0) * k, wout + static_cast<size_t>(row0) * k);
 }
 
 // Router with the whole router weight matrix staged in shared memory
@@ -198,6 +201,7 @@ __global__ void __launch_bounds__(256, 1) router_smem_kernel(const uint16_t* __r
   float* ls = reinterpret_cast<float*>(xs + static_cast<size_t>(R) * H);      // [R][E]
   __shared__ __align__(8) uint64_t bar;
   __shared__ int ok_s;
+  __shared__ int32_t slot_s[R * 8];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int hv = H / 8;
   const uint32_t total = static_cast<uint32_t>(E) * H * 2;
@@ -270,8 +274,8 @@ __global__ void __launch_bounds__(256, 1) router_smem_kernel(const uint16_t* __r
       }
     }
     __syncthreads();
-    if (warp < nrows) topk_select_row(ls + warp * E, E, k, lane, idx + static_cast<size_t>(row0 + warp) * k,
-                                      wout + static_cast<size_t>(row0 + warp) * k);
+    topk_rows_block(ls, E, k, nrows, slot_s, idx + static_cast<size_t>(row0) * k,
+                    wout + static_cast<size_t>(row0) * k);
     __syncthreads();
   }
 }
@@ -336,10 +340,13 @@ cudaError_t launch_router(const uint16_t* x, int T, int H, int E, int k, const u
 //      rounded separately, in slot order, shared last), written to `out` and
 //      kept in shared memory; without them, the rows of `x` are loaded as is;
 //  (2) the router of the next layer on those rows: logits h[r] . W_r[e]
-//      (+ bias) in fp32, warp w owning experts w, w+8, ...; the router rows
-//      stream from L2 four experts at a time, all loads of a batch issued
-//      before any is used (NV 16-byte vectors per lane per expert row);
-//  (3) top-k with renormalised softmax weights, one warp per row;
+//      (+ bias) in fp32, warp w owning experts w, w+16, ... (NV 16-byte
+//      vectors per lane per expert row).  With STAGE the whole router matrix
+//      is copied into shared memory by bulk copies issued at the CTA's start,
+//      before it waits for its predecessor (the weights depend on nothing),
+//      so the copy overlaps that wait and the combine; otherwise the router
+//      rows stream from L2 four experts at a time;
+//  (3) top-k with renormalised softmax weights (topk_rows_block);
 //  (4) with slab_counts: the grouping by expert of the next layer, done here
 //      instead of by a separate permute launch.  Each routed entry claims the
 //      next free row of its expert's slab (an atomic counter per expert) and
@@ -347,7 +354,7 @@ cudaError_t launch_router(const uint16_t* x, int T, int H, int E, int k, const u
 //      slab's capacity (only possible for rows whose logits are all -inf or
 //      NaN) is undone, reported as an internal error and its entry skipped.
 // ---------------------------------------------------------------------------
-template <int R, int NV>
+template <int R, int NV, bool STAGE>
 __global__ void __launch_bounds__(512) combine_route_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ y_perm, const float* __restrict__ y_sh,
     const int32_t* __restrict__ inv, const float* __restrict__ w_prev, int k_prev, int n_pos,
@@ -355,19 +362,40 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
     const float* __restrict__ bias, int32_t* __restrict__ idx, float* __restrict__ wout, int* err,
     const L2Prefetch pf, int32_t* __restrict__ slab_counts, int32_t* __restrict__ inv_out,
     uint16_t* __restrict__ x_slab, int slab_rows, const uint16_t* __restrict__ norm_gain,
-    uint16_t* __restrict__ xn_out) {
+    uint16_t* __restrict__ xn_out, uint64_t timeout_ns) {
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ int32_t sel_s[R * 8];  // the experts each row selected
+  __shared__ int32_t sel_s[R * 8];  // the experts each row selected, by slot
   __shared__ int32_t pos_s[R * 8];  // their slab rows (-1: skipped)
   __shared__ float nred[R][16];     // RMSNorm partial sums, one per warp
-  uint16_t* hs = reinterpret_cast<uint16_t*>(sm);                         // [R][H]
+  __shared__ __align__(8) uint64_t wbar;  // STAGE: the router matrix has landed
+  __shared__ int wok_s;
+  const uint32_t wbytes = STAGE ? static_cast<uint32_t>(E) * H * 2 : 0u;
+  const uint16_t* wsm = reinterpret_cast<const uint16_t*>(sm);           // STAGE: [E][H]
+  uint16_t* hs = reinterpret_cast<uint16_t*>(sm + wbytes);                // [R][H]
   float* ls = reinterpret_cast<float*>(hs + static_cast<size_t>(R) * H);  // [R][E]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int hv = H / 8;
   const int row0 = blockIdx.x * R;
   const int nrows = min(R, T - row0);
   pdl_trigger();
-  if (blockIdx.x == 0 && tid == 0) prefetch_l2_bulk(wr, static_cast<uint32_t>(E) * H * 2);  // weights: no dependency
+  if (STAGE) {
+    if (row0 < T && tid == 0) {
+      mbar_init(&wbar, 1);
+      fence_barrier_init();
+      mbar_arrive_expect_tx(&wbar, wbytes);
+      constexpr uint32_t kChunk = 32768;
+      for (uint32_t off = 0; off < wbytes; off += kChunk) {
+        const uint32_t sz = min(kChunk, wbytes - off);
+        asm volatile(
+            "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                smem_u32(sm + off)),
+            "l"(reinterpret_cast<const uint8_t*>(wr) + off), "r"(sz), "r"(smem_u32(&wbar))
+            : "memory");
+      }
+    }
+  } else if (blockIdx.x == 0 && tid == 0) {
+    prefetch_l2_bulk(wr, static_cast<uint32_t>(E) * H * 2);  // weights: no dependency
+  }
   prefetch_share(pf);  // the next GEMM's first weights, while HBM is otherwise idle
   if (row0 >= T) return;  // a prefetch-only CTA (uniform across the CTA)
   pdl_wait();  // expert outputs / rows come from the previous kernel
@@ -481,6 +509,25 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
     __syncthreads();
   }
 
+  if (STAGE) {  // bounded wait for the router matrix; on a timeout the rows are reported, not routed
+    if (tid == 0) {
+      int dummy = 0;
+      wok_s = mbar_wait(&wbar, 0, &dummy, err, globaltimer_ns() + timeout_ns) ? 1 : 0;
+      // whatever the outcome, the copies must land before this CTA may exit
+      if (!wok_s) mbar_wait(&wbar, 0, &dummy, nullptr, globaltimer_ns() + kDrainNs);
+    }
+    __syncthreads();
+    if (!wok_s) {
+      if (tid < nrows * k) {
+        const size_t i = static_cast<size_t>(row0) * k + tid;
+        idx[i] = -1;
+        wout[i] = 0.f;
+        if (slab_counts) inv_out[i] = -1;
+      }
+      return;
+    }
+  }
+
   // (2) router logits: warp w owns experts w, w+16, w+32, w+48 (one batch of
   //     loads for E <= 64); each x vector is converted once and reused.
   constexpr int EB = 4;
@@ -493,8 +540,12 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
         const int c = lane + 32 * v;
-        wv[b][v] = (e < E && c < hv) ? __ldg(reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e) * H) + c)
-                                     : make_uint4(0, 0, 0, 0);
+        if (STAGE)
+          wv[b][v] = (e < E && c < hv) ? reinterpret_cast<const uint4*>(wsm + static_cast<size_t>(e) * H)[c]
+                                       : make_uint4(0, 0, 0, 0);
+        else
+          wv[b][v] = (e < E && c < hv) ? __ldg(reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e) * H) + c)
+                                       : make_uint4(0, 0, 0, 0);
       }
     }
     float acc[EB][R];
@@ -535,9 +586,7 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
   __syncthreads();
 
   // (3) top-k
-  if (warp < nrows)
-    topk_select_row(ls + warp * E, E, k, lane, idx + static_cast<size_t>(row0 + warp) * k,
-                    wout + static_cast<size_t>(row0 + warp) * k, slab_counts ? sel_s + warp * 8 : nullptr);
+  topk_rows_block(ls, E, k, nrows, sel_s, idx + static_cast<size_t>(row0) * k, wout + static_cast<size_t>(row0) * k);
   if (!slab_counts) return;  // uniform across the CTA
 
   // (4) slab placement of the routed rows
@@ -569,15 +618,42 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
   }
 }
 
-template <int R, int NV>
-static cudaError_t launch_combine_route_rv(const CombineRouteArgs& a, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(R) * a.H * 2 + static_cast<size_t>(R) * a.E * 4;
+// Shared memory of one combine-route CTA: the rows and their logits, plus
+// the router matrix when it is staged.
+static size_t combine_route_smem(int R, int H, int E, bool stage) {
+  return (stage ? static_cast<size_t>(E) * H * 2 : 0) + static_cast<size_t>(R) * H * 2 +
+         static_cast<size_t>(R) * E * 4;
+}
+
+template <int R, int NV, bool STAGE>
+static cudaError_t launch_combine_route_rvs(const CombineRouteArgs& a, cudaStream_t s) {
+  const size_t smem = combine_route_smem(R, a.H, a.E, STAGE);
+  if (STAGE) {
+    static thread_local int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+      cudaError_t e = cudaFuncSetAttribute(combine_route_kernel<R, NV, STAGE>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
+      if (e != cudaSuccess) return e;
+      configured_dev = dev;
+    }
+  }
   const int rows_ctas = (a.T + R - 1) / R;
   const int grid = rows_ctas > prefetch_ctas(a.pf) ? rows_ctas : prefetch_ctas(a.pf);  // extra CTAs only prefetch
-  return launch_pdl(combine_route_kernel<R, NV>, dim3(grid), dim3(512), smem, s, a.x, a.y_perm, a.y_sh, a.inv,
-                    a.w_prev, a.k_prev, a.n_pos > 0 ? a.n_pos : a.T * a.k_prev, a.out, a.T, a.H, a.E, a.k, a.wr,
-                    a.bias, a.idx, a.w, a.err, a.pf, a.slab_counts, a.inv_out, a.x_slab, a.slab_rows, a.norm_gain,
-                    a.xn_out);
+  return launch_pdl(combine_route_kernel<R, NV, STAGE>, dim3(grid), dim3(512), smem, s, a.x, a.y_perm, a.y_sh,
+                    a.inv, a.w_prev, a.k_prev, a.n_pos > 0 ? a.n_pos : a.T * a.k_prev, a.out, a.T, a.H, a.E, a.k,
+                    a.wr, a.bias, a.idx, a.w, a.err, a.pf, a.slab_counts, a.inv_out, a.x_slab, a.slab_rows,
+                    a.norm_gain, a.xn_out, a.timeout_ns > 0 ? a.timeout_ns : kDrainNs);
+}
+
+// The router matrix is staged when it fits beside the rows (E * H * 2 bytes,
+// 160 KB at the model shape) and its address suits the bulk copy.
+template <int R, int NV>
+static cudaError_t launch_combine_route_rv(const CombineRouteArgs& a, cudaStream_t s) {
+  const bool stage = combine_route_smem(R, a.H, a.E, true) <= 200 * 1024 &&
+                     (reinterpret_cast<uintptr_t>(a.wr) & 15) == 0;
+  return stage ? launch_combine_route_rvs<R, NV, true>(a, s) : launch_combine_route_rvs<R, NV, false>(a, s);
 }
 
 // Larger batches route with the shared-memory-staged router instead (each of

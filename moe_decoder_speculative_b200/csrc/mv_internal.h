@@ -81,6 +81,8 @@ struct CombineRouteArgs {
   // bf16(RMSNorm(row) * norm_gain), also written to xn_out [T][H].
   const uint16_t* norm_gain;
   uint16_t* xn_out;
+  // Bound on the wait for the staged router matrix (0: the drain bound).
+  uint64_t timeout_ns;
 };
 constexpr float kRmsNormEps = 1e-6f;
 cudaError_t launch_rmsnorm(const uint16_t* x, int T, int H, const uint16_t* gain, uint16_t* out, cudaStream_t s);
