@@ -294,6 +294,7 @@ struct Carve {
 struct FfnWs {
   int32_t *counts, *offsets, *perm, *inv, *sort;
   int32_t* inv_alt;  // slab layout: the other layer's inverse map (layers alternate)
+  int32_t* ent;      // slab layout: the routing entry (r * k + j) of each slab row
   uint16_t *x_perm, *a_perm, *a_sh;
   float *y_perm, *y_sh;
   int64_t n_pos;     // rows of x_perm / a_perm / y_perm
@@ -321,6 +322,7 @@ FfnWs carve_ffn(Carve& c, int64_t T, const mv_moe_shape& s, bool slabs = false) 
   w.perm = c.take<int32_t>(n);
   w.inv = c.take<int32_t>(n);
   w.inv_alt = slabs ? c.take<int32_t>(n) : nullptr;
+  w.ent = slabs ? c.take<int32_t>(rows) : nullptr;
   w.sort = c.take<int32_t>(mv::permute_uses_sort(static_cast<int>(T), s.k) ? mv::sort_scratch_ints(static_cast<int>(T), s.E, s.k) : 1);
   w.x_perm = c.take<uint16_t>(rows * s.H);
   w.a_perm = c.take<uint16_t>(rows * s.I);
@@ -482,6 +484,8 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
     MV_TRY(map(&S.b, ws.a_perm, ws.n_pos, I, bbox));
     S.a1 = S.a0;
     S.out = ws.y_perm;
+    // slab layout: rows are stored by routing entry, so the combine needs no gather map
+    S.row_map = slab_counts ? ws.ent : nullptr;
     S.ld_out = H;
     S.K = I;
     S.M = H;
@@ -524,7 +528,7 @@ mv_status ffn_forward_impl(const uint16_t* x, int T, const mv_moe_shape& s, cons
   const int32_t* inv = slab_counts ? slab_inv : ws.inv;
   e = run_kernel(KIND_COMBINE, st, [&] {
     return mv::launch_combine(ws.y_perm, s.I_shared > 0 ? ws.y_sh : nullptr, inv, tw, res, out, T, s.H, s.k,
-                              static_cast<int>(ws.n_pos), err, combine_pf, st);
+                              static_cast<int>(ws.n_pos), err, combine_pf, st, slab_counts != nullptr);
   });
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   return MV_OK;
@@ -944,6 +948,7 @@ static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts,
       a.pf = moe_first_wave(*shape, layers[0], kPrefetchBudget);
       a.slab_counts = slab_counts(0);
       a.inv_out = slab_inv(0);
+      a.ent_out = fw.ent;
       a.x_slab = fw.x_perm;
       a.slab_rows = static_cast<int>(T);
       a.norm_gain = layers[0].norm_gain;
@@ -996,6 +1001,8 @@ static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts,
           a.pf = moe_first_wave(*shape, wn, kPrefetchBudget);
           a.slab_counts = slab_counts(l + 1);
           a.inv_out = slab_inv(l + 1);
+          a.ent_out = fw.ent;
+          a.y_by_entry = slabs ? 1 : 0;
           a.x_slab = fw.x_perm;
           a.slab_rows = static_cast<int>(T);
           a.norm_gain = wn.norm_gain;

@@ -66,6 +66,7 @@ struct GemmSet {
   const float* bias;       // EPI_TOPK: fp32 [M] added to the logits, or nullptr
   int32_t topk;            // EPI_TOPK: k
   const uint16_t* res;     // EPI_STORE_BF16: bf16 [rows][ld_out] added before rounding, or nullptr
+  const int32_t* row_map;  // EPI_STORE_F32 (swap-AB): output row of B row b is row_map[b], or nullptr: b
 };
 
 struct GemmParams {

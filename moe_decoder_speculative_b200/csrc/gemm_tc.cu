@@ -653,6 +653,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           const int m = ui.m0 + h * 128 + row;
           const bool mvalid = m < S.M;
           for (int c0 = 0; c0 < n_mma; c0 += 32) {
+            // output rows of these 32 B rows: lane j holds row j's (row_map, or b itself)
+            const int bj = ui.b_row0 + c0 + lane;
+            const int orow = (S.row_map && c0 + lane < ui.nvalid) ? __ldg(S.row_map + bj) : bj;
             uint32_t d[32];
             tmem_ld32(tl + h * BN + c0, d);
             tmem_ld_wait();
@@ -660,8 +663,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int n = c0 + j;
-              if (mvalid && n < ui.nvalid)
-                out[static_cast<size_t>(ui.b_row0 + n) * S.ld_out + m] = __uint_as_float(d[j]);
+              const int o = __shfl_sync(0xffffffffu, orow, j);
+              if (mvalid && n < ui.nvalid) out[static_cast<size_t>(o) * S.ld_out + m] = __uint_as_float(d[j]);
             }
           }
         }

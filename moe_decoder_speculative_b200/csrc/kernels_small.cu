@@ -91,6 +91,7 @@ __device__ void topk_rows_block(const float* ls, int E, int k, int nrows, int32_
       lr = ls + r * E;
       const uint32_t ke = logit_key(lr[e]);
       const int i1 = min(E, (sub + 1) * chunk);
+#pragma unroll 8
       for (int i = sub * chunk; i < i1; ++i) {
         const uint32_t ki = logit_key(lr[i]);
         cnt += (ki > ke || (ki == ke && i < e)) ? 1 : 0;
@@ -102,16 +103,19 @@ __device__ void topk_rows_block(const float* ls, int E, int k, int nrows, int32_
     if (it < items && sub == 0 && cnt < k) slot_s[(q / E) * 8 + cnt] = e;
   }
   __syncthreads();
-  for (int r = tid >> 5; r < nrows; r += blockDim.x >> 5) {
+  // lane j computes slot j's exponential; the sum adds them in slot order
+  for (int r = tid >> 5; r < nrows; r += blockDim.x >> 5) {  // whole warps: the shuffles see every lane
+    const float* lr = ls + r * E;
+    const int32_t* sl = slot_s + r * 8;
+    const int e = lane < k ? sl[lane] : 0;
+    const float mx = lr[sl[0]];
+    const float ex = lane < k ? expf(lr[e] - mx) : 0.f;
+    float s = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < k; ++j) s += __shfl_sync(0xffffffffu, ex, j);
     if (lane < k) {
-      const float* lr = ls + r * E;
-      const int32_t* sl = slot_s + r * 8;
-      const float mx = lr[sl[0]];
-      float s = 0.f;
-      for (int j = 0; j < k; ++j) s += expf(lr[sl[j]] - mx);
-      const int e = sl[lane];
       idx_out[r * k + lane] = e;
-      w_out[r * k + lane] = expf(lr[e] - mx) / s;
+      w_out[r * k + lane] = ex / s;
     }
   }
 }
@@ -362,7 +366,7 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
     const float* __restrict__ bias, int32_t* __restrict__ idx, float* __restrict__ wout, int* err,
     const L2Prefetch pf, int32_t* __restrict__ slab_counts, int32_t* __restrict__ inv_out,
     uint16_t* __restrict__ x_slab, int slab_rows, const uint16_t* __restrict__ norm_gain,
-    uint16_t* __restrict__ xn_out, uint64_t timeout_ns) {
+    uint16_t* __restrict__ xn_out, uint64_t timeout_ns, int32_t* __restrict__ ent_out, int y_by_entry) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ int32_t sel_s[R * 8];  // the experts each row selected, by slot
   __shared__ int32_t pos_s[R * 8];  // their slab rows (-1: skipped)
@@ -417,8 +421,11 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
         float4 ya[8], yb[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          if (pos[j] >= 0 && pos[j] < n_pos) {
-            const float4* yp = reinterpret_cast<const float4*>(y_perm + static_cast<size_t>(pos[j]) * H) + 2 * c;
+          // by entry, the row address needs no routing data: the loads issue with those of inv
+          const bool ok = y_by_entry ? (j < k_prev) : (pos[j] >= 0 && pos[j] < n_pos);
+          const size_t yrow = y_by_entry ? row * k_prev + j : static_cast<size_t>(pos[j]);
+          if (ok) {
+            const float4* yp = reinterpret_cast<const float4*>(y_perm + yrow * H) + 2 * c;
             ya[j] = yp[0];
             yb[j] = yp[1];
           } else {
@@ -606,6 +613,7 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
     if (p < 0 && err) atomicOr(err, kErrInternal);
     pos_s[r * 8 + j] = p;
     inv_out[static_cast<size_t>(row0 + r) * k + j] = p;
+    if (ent_out && p >= 0) ent_out[p] = (row0 + r) * k + j;
   }
   __syncthreads();
   for (int i = tid; i < nrows * k * hv; i += blockDim.x) {
@@ -644,7 +652,8 @@ static cudaError_t launch_combine_route_rvs(const CombineRouteArgs& a, cudaStrea
   return launch_pdl(combine_route_kernel<R, NV, STAGE>, dim3(grid), dim3(512), smem, s, a.x, a.y_perm, a.y_sh,
                     a.inv, a.w_prev, a.k_prev, a.n_pos > 0 ? a.n_pos : a.T * a.k_prev, a.out, a.T, a.H, a.E, a.k,
                     a.wr, a.bias, a.idx, a.w, a.err, a.pf, a.slab_counts, a.inv_out, a.x_slab, a.slab_rows,
-                    a.norm_gain, a.xn_out, a.timeout_ns > 0 ? a.timeout_ns : kDrainNs);
+                    a.norm_gain, a.xn_out, a.timeout_ns > 0 ? a.timeout_ns : kDrainNs, a.ent_out,
+                    a.y_by_entry ? 1 : 0);
 }
 
 // The router matrix is staged when it fits beside the rows (E * H * 2 bytes,
@@ -963,7 +972,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
                                                       const int32_t* __restrict__ inv,
                                                       const float* __restrict__ w,
                                                       const uint16_t* res, uint16_t* out, int T,
-                                                      int H, int k, int n_pos, int* err, const L2Prefetch pf) {
+                                                      int H, int k, int n_pos, int* err, const L2Prefetch pf,
+                                                      int by_entry) {
   pdl_trigger();
   prefetch_share(pf);
   pdl_wait();
@@ -983,8 +993,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     float4 ya[8], yb[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      if (pos[j] >= 0 && pos[j] < n_pos) {
-        const float4* yp = reinterpret_cast<const float4*>(y_perm + static_cast<size_t>(pos[j]) * H) + 2 * c;
+      // by entry, the row address needs no routing data: the loads issue with those of inv
+      const bool ok = by_entry ? (j < k) : (pos[j] >= 0 && pos[j] < n_pos);
+      const size_t yrow = by_entry ? static_cast<size_t>(r) * k + j : static_cast<size_t>(pos[j]);
+      if (ok) {
+        const float4* yp = reinterpret_cast<const float4*>(y_perm + yrow * H) + 2 * c;
         ya[j] = yp[0];
         yb[j] = yp[1];
       } else {
@@ -1029,14 +1042,14 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t* inv,
                            const float* w, const uint16_t* res, uint16_t* out, int T, int H,
-                           int k, int n_pos, int* err, const L2Prefetch& pf, cudaStream_t s) {
+                           int k, int n_pos, int* err, const L2Prefetch& pf, cudaStream_t s, bool y_by_entry) {
   if (T <= 0) return cudaSuccess;
   const long long total = static_cast<long long>(T) * (H / 8);
   const long long blocks = (total + 255) / 256;
   int grid = static_cast<int>(blocks < 148LL * 8 ? blocks : 148LL * 8);
   if (grid < prefetch_ctas(pf)) grid = prefetch_ctas(pf);  // the grid-stride loop leaves the extra CTAs idle
   return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, s, y_perm, y_sh, inv, w, res, out, T, H, k, n_pos, err,
-                    pf);
+                    pf, y_by_entry ? 1 : 0);
 }
 
 // ---------------------------------------------------------------------------

@@ -77,6 +77,10 @@ struct CombineRouteArgs {
   int32_t* inv_out;
   uint16_t* x_slab;
   int slab_rows;
+  int32_t* ent_out;         // with slab_counts, or nullptr: ent_out[p] = r * k + j (the entry of slab row p)
+  // y_perm holds the combined layer's expert outputs by entry (row r * k_prev
+  // + j) instead of by grouped position; inv then only tells valid entries.
+  int y_by_entry;
   // Pre-RMSNorm variant, or nullptr: the rows are routed (and placed) as
   // bf16(RMSNorm(row) * norm_gain), also written to xn_out [T][H].
   const uint16_t* norm_gain;
@@ -100,9 +104,11 @@ cudaError_t launch_permute_sorted(const int32_t* idx, int T, int E, int k, int32
                                   int32_t* perm, int32_t* inv, const uint16_t* x, int H, uint16_t* x_perm,
                                   int32_t* scratch, cudaStream_t s);
 // n_pos: the number of y_perm rows (positions in inv are checked against it).
+// y_by_entry: y_perm rows are entries r * k + j (inv only marks valid ones).
 cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t* inv,
                            const float* w, const uint16_t* res, uint16_t* out, int T, int H,
-                           int k, int n_pos, int* err, const L2Prefetch& pf, cudaStream_t s);
+                           int k, int n_pos, int* err, const L2Prefetch& pf, cudaStream_t s,
+                           bool y_by_entry = false);
 // The FastMTP draft block's per-sequence step (kernels_small.cu, mtp_step_kernel).
 struct MtpStepArgs {
   const uint64_t* keys;   // previous step's LM keys [B][ld] (nparts used), or nullptr: take t0
