@@ -302,10 +302,12 @@ struct FfnWs {
 
 // Decode-sized verify steps group the routed rows by expert inside the
 // routing kernel (combine_route) instead of a permute launch: expert e owns
-// rows [e*T, (e+1)*T) of x_perm, a_perm and y_perm (a row selects an expert
-// at most once, so T rows always suffice) and its row count is an atomic
-// counter in the layer's scheduling block.  Larger batches keep the compact
-// stable permutation.
+// rows [e*T, (e+1)*T) of x_perm and a_perm (a row selects an expert at most
+// once, so T rows always suffice) and its row count is an atomic counter in
+// the layer's scheduling block; the down projection stores its outputs in
+// y_perm by routing entry (row * k + slot, through the `ent` map the routing
+// kernel writes), so the combine reads them without a gather map.  Larger
+// batches keep the compact stable permutation.
 bool use_slabs(int64_t T, const mv_moe_shape& s) {
   return T * s.k <= 16LL * s.E && mv::combine_route_supported(static_cast<int>(T), s.H, s.E);
 }
