@@ -82,6 +82,57 @@ def test_router_topk_large_batch(T, bias):
     np.testing.assert_allclose(tw[same], w_ref[same], rtol=2e-5, atol=2e-6)
 
 
+def _router_case(T, seed):
+    rng = np.random.default_rng(seed)
+    H, E, k = 1280, 64, 6
+    x = wl.f32_to_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    wr = wl.f32_to_bf16_bits(rng.standard_normal((E, H)).astype(np.float32) * 0.02)
+    return x, wr, bd.MoeShape(H, E, 896, 0, k), k
+
+
+@pytest.mark.parametrize("T", [4, 128, 700])
+def test_router_rows_with_fewer_than_k_finite_logits(T):
+    """Only 4 experts have finite logits (bias -inf elsewhere) under top-6: every
+    row still gets 6 distinct experts, the 4 finite ones in descending order and
+    then the -inf ones by id (0 and 1), with weight 0, as the oracle's stable
+    ordering gives.  1 and 2 rows per routing CTA (T <= 512, T > 512)."""
+    x, wr, shape, k = _router_case(T, 100 + T)
+    finite = np.array([5, 17, 40, 63])
+    b = np.full(shape.E, -np.inf, np.float32)
+    b[finite] = 0.0
+    idx_ref, w_ref, _, _ = oracle.router(x, wr, k, bias=b)
+    idx, tw = bd.moe_router_topk(bd.bf16_to_device(x), shape, bd.bf16_to_device(wr), torch.from_numpy(b).cuda())
+    idx, tw = to_np(idx), to_np(tw)
+    np.testing.assert_array_equal(idx_ref[:, 4:], np.tile([0, 1], (T, 1)))    # the oracle's own reading
+    np.testing.assert_array_equal(idx[:, 4:], idx_ref[:, 4:])
+    assert np.all(np.sort(idx[:, :4], axis=1) == finite)
+    assert np.all(tw[:, 4:] == 0.0)
+    same = np.all(idx == idx_ref, axis=1)
+    assert same.mean() > 0.95
+    np.testing.assert_allclose(tw[same], w_ref[same], rtol=2e-5, atol=2e-6)
+
+
+@pytest.mark.parametrize("T", [128, 700])
+def test_router_nan_logits_are_never_chosen_over_numbers(T):
+    """A NaN logit (bias NaN on experts 0-9) ranks below every number: with 54
+    numbers per row the routing equals the oracle's with those experts at -inf."""
+    x, wr, shape, k = _router_case(T, 200 + T)
+    b = np.zeros(shape.E, np.float32)
+    b[:10] = np.nan
+    b_ref = b.copy()
+    b_ref[:10] = -np.inf
+    idx_ref, w_ref, _, gap = oracle.router(x, wr, k, bias=b_ref)
+    idx, tw = bd.moe_router_topk(bd.bf16_to_device(x), shape, bd.bf16_to_device(wr), torch.from_numpy(b).cuda())
+    idx, tw = to_np(idx), to_np(tw)
+    assert idx.min() >= 10 and idx.max() < shape.E
+    assert np.all(np.isfinite(tw))
+    ok = gap >= GATE_GAP
+    assert same_routing(idx, idx_ref)[ok].all()
+    same = np.all(idx == idx_ref, axis=1)
+    assert same.mean() > 0.95
+    np.testing.assert_allclose(tw[same], w_ref[same], rtol=2e-5, atol=2e-6)
+
+
 @pytest.mark.parametrize("T,E,k", [(16, 8, 2), (128, 64, 6), (37, 64, 6), (1, 8, 8), (1000, 256, 8)])
 def test_expert_permute(T, E, k):
     rng = np.random.default_rng(T * 7 + E)
