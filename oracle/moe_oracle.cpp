@@ -94,10 +94,17 @@ void router_row(const uint16_t* x, int H, int E, int k, const uint16_t* w_router
     if (bias) v += static_cast<Acc>(bias[e]);
     l[e] = v;
   }
-  // Order experts by logit, largest first; equal logits keep the lower id first.
+  // Order experts by logit, largest first; equal logits keep the lower id
+  // first (stable sort).  A NaN logit comes after every number, so a row with
+  // fewer than k numbers still selects k distinct experts: the -inf ones next
+  // by id, then the NaN ones by id.
   std::vector<int> order(E);
   std::iota(order.begin(), order.end(), 0);
-  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return l[a] > l[b]; });
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+    const bool na = std::isnan(l[a]), nb = std::isnan(l[b]);
+    if (na || nb) return !na && nb;
+    return l[a] > l[b];
+  });
   for (int j = 0; j < k; ++j) idx[j] = order[j];
 
   if (gap_out)

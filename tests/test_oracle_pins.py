@@ -90,6 +90,54 @@ def test_router_selection_brute_force(oracle_mod, E, k):
         assert gap[0] == np.float32(want_gap)
 
 
+def test_router_fewer_than_k_numbers_takes_the_rest_by_id(oracle_mod):
+    """Reading of the selection rule on degenerate rows: numbers first (largest
+    first), then -inf logits by id, then NaN logits by id; k distinct experts.
+    Logits are set through the bias on a zero row, so the expected ids follow
+    from the rule alone.  Weights: 0 on -inf experts when the row has numbers
+    and no NaN (a NaN logit anywhere makes the softmax over all E NaN)."""
+    H, E, k = 8, 8, 6
+    x = np.zeros((1, H), np.float32)
+    wr = np.zeros((E, H), np.float32)
+    nan, inf = np.float32(np.nan), np.float32(np.inf)
+    cases = [
+        # bias per expert                                    expected slots
+        ([-inf, 0.5, -inf, 2.0, -inf, -inf, 1.0, -inf], [3, 6, 1, 0, 2, 4]),
+        ([nan, 0.5, -inf, 2.0, nan, -inf, 1.0, nan], [3, 6, 1, 2, 5, 0]),
+        ([nan, nan, nan, 1.0, nan, nan, nan, nan], [3, 0, 1, 2, 4, 5]),
+        ([-inf] * 8, [0, 1, 2, 3, 4, 5]),
+    ]
+    for b, want in cases:
+        b = np.array(b, np.float32)
+        idx, w, _, _ = oracle_mod.router(bf16(x), bf16(wr), k, bias=b)
+        assert idx[0].tolist() == want, (b, idx[0])
+        fin = np.isfinite(b[want])
+        if fin.any() and not np.isnan(b).any():
+            assert np.all(w[0][~fin] == 0)
+            np.testing.assert_allclose(w[0][fin].sum(), 1.0, rtol=1e-6)
+        elif np.isnan(b).any():
+            assert np.all(np.isnan(w[0]))
+
+
+def test_router_nan_logits_do_not_displace_numbers(oracle_mod):
+    """With at least k numbers, NaN logits change no selection: it equals the
+    one with those experts at -inf.  The weights then follow the form over the
+    selected experts (the softmax over all E would be NaN)."""
+    rng = np.random.default_rng(41)
+    T, H, E, k = 32, 64, 16, 4
+    x, wr = rand_bf16(rng, (T, H), 1.0), rand_bf16(rng, (E, H), 0.3)
+    b_nan = np.zeros(E, np.float32)
+    b_nan[[0, 3, 9]] = np.nan
+    b_inf = b_nan.copy()
+    b_inf[[0, 3, 9]] = -np.inf
+    a = oracle_mod.router(x, wr, k, bias=b_nan, weight_form=1)
+    c = oracle_mod.router(x, wr, k, bias=b_inf, weight_form=1)
+    np.testing.assert_array_equal(a[0], c[0])
+    np.testing.assert_array_equal(a[1], c[1])
+    assert np.all(np.isfinite(a[1]))
+    assert not np.isin(a[0], [0, 3, 9]).any()
+
+
 def test_gate_weights_invariants_and_forms(oracle_mod):
     """w >= 0, sum w = 1, and the literal softmax-then-renormalise form equals
     the short form exp(l - l_max_sel) / sum_sel."""
