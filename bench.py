@@ -30,6 +30,7 @@ import os
 import re
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -130,7 +131,7 @@ class ClockSampler:
     def __init__(self, gpu_id: str | None):
         self.gpu_id = gpu_id
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"moe_verify_clocks_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
