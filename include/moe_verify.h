@@ -72,7 +72,7 @@ typedef enum {
 } mv_status;
 
 /* Shape of one MoE layer.  I_shared = 0 means no shared expert.  The model
- * card's "2 shared" experts are passed as one always-on SwiGLU of
+ * card's two shared experts are passed as one always-on SwiGLU of
  * I_shared = 2*I whose gate/up rows and down columns are the two concatenated;
  * that is exactly the sum of the two experts' outputs. */
 typedef struct {
@@ -106,7 +106,7 @@ typedef struct {
 
 /* ---------------------------------------------------------------------------
  * moe_router_topk - router of one MoE layer (model card, architecture
- * paragraph: "64 routed experts ... under top-6 routing").
+ * paragraph: each token is routed to 6 of the 64 routed experts).
  * For every row r: logits l[e] = x[r] . w_router[e] (+ router_bias[e]) in
  * fp32; the k largest logits are kept (equal logits: lower expert id first),
  * slot j holding the j-th largest; topk_w[r][j] = softmax over all E logits
