@@ -233,3 +233,68 @@ def test_speculative_loop_with_the_draft_block_is_lossless(oracle_mod):
             assert drafts.shape == (B, K) and np.all((drafts >= 0) & (drafts < Vt))
         for b in range(B):
             assert seqs[b][:2 + n] == greedy[b][:2 + n]
+
+
+# ------------------------------------------- where the loop step starts drafting
+
+def _start_case(rng, half):
+    """A verify step with no MoE layers (h_L = the input rows) whose rows are
+    one-hot, row r = e_r, and an LM head that sends e_r to token pi(r), so the
+    verifier's choice at row r is pi(r).  Each sequence's drafts are built to
+    keep a chosen number of them.  The draft block has a zero FFN and reads
+    only one half of its input: the hidden half (projection [I | 0]) or the
+    embedding half ([0 | I], with one-hot embeddings E[v] = e_{sigma(v)})."""
+    B, K = 4, 3
+    T = B * (K + 1)
+    pi = rng.permutation(V)
+    sigma = rng.permutation(V)
+    hidden = bf(np.eye(T, H))
+    w_lm = bf(perm_matrix(pi))              # W_lm[pi[r]] = e_r
+    g = pi[np.arange(T)]
+    keep = np.array([2, 0, 3, 1])
+    drafts = np.zeros((B, K), np.int32)
+    for b in range(B):
+        for i in range(K):
+            d = g[b * (K + 1) + i]
+            drafts[b, i] = d if i < keep[b] else (d + 1) % V
+    blk = base_block(rng)
+    proj = np.zeros((H, 2 * H), np.float32)
+    if half == "hidden":
+        proj[:, :H] = np.eye(H)
+    else:
+        proj[:, H:] = np.eye(H)
+        blk["w_emb"] = bf(perm_matrix(sigma).T)   # E[v] = e_{sigma[v]}
+    blk["w_proj"] = bf(proj)
+    return B, K, pi, sigma, hidden, w_lm, drafts, keep, blk
+
+
+def test_loop_step_drafts_from_the_last_kept_row(oracle_mod):
+    """The draft block starts from the verifier's final hidden state at each
+    sequence's last kept row, b*(K+1) + accepted[b].  With a block that reads
+    only the hidden half, that row r = e_r normalises to 8 e_r, and every
+    step's choice is pi(r): a start at row b*(K+1), or one past the kept row,
+    gives another token."""
+    rng = np.random.default_rng(31)
+    B, K, pi, _, hidden, w_lm, drafts, keep, blk = _start_case(rng, "hidden")
+    st = oracle_mod.speculative_step(hidden, drafts, B, K, [], 2, w_lm, blk)
+    np.testing.assert_array_equal(st["accepted"], keep)
+    r = np.arange(B) * (K + 1) + keep
+    np.testing.assert_array_equal(st["next_drafts"], np.repeat(pi[r][:, None], K, axis=1))
+    for wrong in (np.arange(B) * (K + 1), r + 1):
+        assert np.any(pi[wrong] != pi[r])
+
+
+def test_loop_step_drafts_from_the_verifiers_next_token(oracle_mod):
+    """The first draft step embeds the verifier's next token, g at the last
+    kept row: with a block that reads only the embedding half, t0 = pi(r)
+    embeds to e_{sigma(pi(r))}, so the first draft is pi(sigma(pi(r))) and
+    every later step walks pi o sigma once more."""
+    rng = np.random.default_rng(32)
+    B, K, pi, sigma, hidden, w_lm, drafts, keep, blk = _start_case(rng, "embed")
+    st = oracle_mod.speculative_step(hidden, drafts, B, K, [], 2, w_lm, blk)
+    r = np.arange(B) * (K + 1) + keep
+    np.testing.assert_array_equal(st["next_token"], pi[r])
+    t = pi[r]
+    for j in range(K):
+        t = pi[sigma[t]]
+        np.testing.assert_array_equal(st["next_drafts"][:, j], t)
