@@ -41,8 +41,10 @@ sys.path.insert(0, ROOT)
 
 from moe_decoder_speculative_b200 import workloads as wl  # noqa: E402
 
-METRIC = "verified tokens/s per MoE verify step at 32x(K+1) rows"
-UNIT = "tokens/s"
+# The workload's metric name; `value` counts committed tokens (accepted + 1 per
+# sequence, the tokens a verify step emits), and `rows_per_s` the verified rows.
+METRIC = "verified tokens/s per MoE verify step at 32x(K+1) rows, counted as committed tokens (accepted+1 per sequence)"
+UNIT = "committed tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -54,6 +56,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=2, help="workload id (default: concurrency-32 verify)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="leave out the prefill-layer figures the default line carries")
     ap.add_argument("--layers", type=int, default=None,
                     help="run only the first N MoE layers (a smaller case for profiling; not a bench line)")
     ap.add_argument("--graph", action="store_true",
@@ -347,18 +351,30 @@ def run_ours(args):
     plan = bd.VerifyPlan(shape, layers, w_lm, w.B, w.K, dev)
     T = w.T
 
-    # drafts: the verifier's own argmax (one untimed pass) copied with p = 0.576
+    # drafts: the verifier's own argmax (one untimed pass) copied with probability p_agree
     zero = torch.zeros((w.B, w.K), dtype=torch.int32, device=dev)
     _, _, _, am = plan(hidden, zero)
+    tie_rows = 0
+    if w.tie_frac > 0:
+        # near-tied LM-head rows built from this first pass's choices, then a second pass
+        w_lm_np, rows_t, _ = wl.make_tied_lm_head(w, inp["w_lm"], am.cpu().numpy())
+        tie_rows = len(rows_t)
+        w_lm = bd.bf16_to_device(w_lm_np, dev)
+        plan = bd.VerifyPlan(shape, layers, w_lm, w.B, w.K, dev)
+        _, _, _, am = plan(hidden, zero)
     drafts_np = wl.make_drafts(w, am.cpu().numpy())
     drafts = torch.from_numpy(drafts_np).to(dev)
 
-    # touched experts per layer (for the algorithmic byte count), via the public per-step calls
-    touched = []
+    # touched experts per layer (for the algorithmic byte count) and the hot
+    # experts' share of the routing slots, via the public per-step calls
+    touched, hot_share = [], []
+    hot = torch.from_numpy(wl.hot_experts(w)).to(dev) if w.n_hot else None
     h = hidden
     for lw in layers:
         idx, tw = bd.moe_router_topk(h, shape, lw.t["w_router"], lw.t["router_bias"])
         touched.append(int(torch.unique(idx).numel()))
+        if hot is not None:
+            hot_share.append(round(float(torch.isin(idx, hot).float().mean().item()), 4))
         h = bd.moe_ffn_forward(h, shape, lw, idx, tw, residual=h)
     plan.sync_status()
 
@@ -466,14 +482,14 @@ def run_ours(args):
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic (seeded bf16 weights N(0,0.02^2), hidden N(0,1); drafts copy the "
-                                  "verifier argmax w.p. 0.576)",
+        "dtype": "bf16", "data": f"synthetic (seeded bf16 weights N(0,0.02^2), hidden N(0,1); drafts copy the "
+                                  f"verifier argmax w.p. {w.p_agree})",
         "config": {"workload": w.name, "B": w.B, "K": w.K, "rows": T, "layers": len(layers), "H": w.H, "E": w.E,
                    "top_k": w.k, "I": w.I, "I_shared": w.I_sh, "V": w.V,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "launch": "CUDA graph replay (verify_graph_launch)" if args.graph else "eager (verify_step)",
                    "layer": "pre-RMSNorm variant" if args.norm else "residual, no norm",
-                   "l2": "weights (5.8 GB) far larger than L2: no flush needed"},
+                   "l2": f"weights ({step_bytes / 1e9:.2f} GB per step) larger than L2: no flush needed"},
         "rows_per_s": world * T * K / (ms / 1e3),
         "committed_per_step": committed_all,
         "step_roofline": {"alg_bytes": int(step_bytes), "achieved_gbs": round(step_bytes / (ms / K / 1e3) / 1e9, 1),
@@ -491,7 +507,14 @@ def run_ours(args):
         "clocks": clk,
         "touched_experts": touched,
     }
+    if w.n_hot:
+        out["skew"] = {"hot_experts": wl.hot_experts(w).tolist(), "router_bias": w.hot_bias,
+                       "hot_share_of_slots": hot_share, "tied_lm_rows": tie_rows}
 
+    if rank == 0 and world == 1 and args.workload == 2 and not args.no_prefill and args.layers is None:
+        # the prefill-sized MoE layer (8 pages x 1,156 visual tokens), tensor-bound:
+        # reported beside the decode step, not part of its value
+        out["prefill_layer"] = measure_prefill(3, min(args.steps, 50), args.warmup)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
@@ -691,15 +714,16 @@ def run_spec(args):
     return 0
 
 
-def run_prefill(args):
-    """A MoE layer over prefill-sized batches (routing + grouped SwiGLU experts +
-    combine), tensor-bound: reports rows/s and the grouped GEMM's TFLOP/s."""
+def measure_prefill(wid, steps, warmup):
+    """The prefill-sized MoE layer (routing + grouped SwiGLU experts + combine
+    over 8 pages x 1,156 visual tokens), device-timed with CUDA events: the
+    layer's time and rows/s, and the grouped GEMM's TFLOP/s against the bf16
+    tensor peak (burst: a sub-millisecond kernel timed alone by events)."""
     import torch
 
     from moe_decoder_speculative_b200 import binding as bd
 
-    torch.cuda.set_device(0)
-    w = wl.workload(args.workload)
+    w = wl.workload(wid)
     inp = wl.make_inputs(w, layers=1)
     shape = bd.shape_of(w)
     lw = bd.LayerWeights(inp["layers"][0])
@@ -714,51 +738,69 @@ def run_prefill(args):
         bd.moe_router_topk(x, shape, lw.t["w_router"], lw.t["router_bias"], idx, tw)
         bd.moe_ffn_forward(x, shape, lw, idx, tw, residual=x, out=out, ws=ws)
 
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, warmup)):
         step()
     torch.cuda.synchronize()
     bd.sync_status(ws)
     touched = int(torch.unique(idx).numel())
     stream = torch.cuda.current_stream()
-    with ClockSampler(gpu_uuid(torch, torch.device("cuda", 0))) as clocks:
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n0 = bd.launch_count()
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        launches = bd.launch_count() - n0
-        ms = e0.elapsed_time(e1)
-        bd.profile_enable(True)
-        for _ in range(args.steps):
-            step()
-        torch.cuda.synchronize()
-        bd.profile_enable(False)
-        kern = bd.profile_collect()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = bd.launch_count()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = bd.launch_count() - n0
+    ms = e0.elapsed_time(e1)
+    bd.profile_enable(True)
+    for _ in range(steps):
+        step()
+    torch.cuda.synchronize()
+    bd.profile_enable(False)
+    kern = bd.profile_collect()
     bd.sync_status(ws)
-    clk = clocks.summary()
     gemm_flops = T * (w.k * 3 * 2 * w.H * w.I + 3 * 2 * w.H * w.I_sh)
     layer_flops = gemm_flops + T * 2 * w.H * w.E
     g = kern.get("grouped_moe_gemm", {"launches": 0, "ms": 0.0})
     gemm_s = g["ms"] / max(1, g["launches"]) / 1e3
     burst, sustained, src = measured_tensor_peaks()
     achieved = gemm_flops / gemm_s / 1e12 if gemm_s > 0 else None
-    K = args.steps
-    print(json.dumps({
-        "metric": "prefill MoE layer rows/s (8 pages x 1,156 visual tokens)", "value": T * K / (ms / 1e3),
-        "unit": "rows/s", "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": ms / K,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "rows": T, "H": w.H, "E": w.E, "top_k": w.k, "I": w.I, "I_shared": w.I_sh,
-                   "touched_experts": touched,
-                   "l2": "weights + activations (0.5 GB) larger than L2: no flush needed"},
-        "layer_tflops": layer_flops / (ms / K / 1e3) / 1e12,
-        "roofline": {"kernel": "grouped_moe_gemm", "bound": "tensor", "achieved": achieved,
-                     "peak": sustained, "peak_burst": burst, "peak_source": src, "unit": "TFLOP/s",
-                     "frac": (achieved / sustained) if achieved else None, "alg_flops_per_launch": gemm_flops},
+    layer_s = ms / steps / 1e3
+    return {
+        "workload": w.name, "rows": T, "touched_experts": touched, "ms_per_layer": ms / steps,
+        "rows_per_s": T / layer_s, "launches": int(launches),
+        "layer_tflops": round(layer_flops / layer_s / 1e12, 1),
+        "layer_frac_of_burst": round(layer_flops / layer_s / 1e12 / burst, 4),
+        "gemm": {"kernel": "grouped_moe_gemm", "bound": "tensor", "avg_us": round(gemm_s * 1e6, 2),
+                 "achieved": round(achieved, 1) if achieved else None, "unit": "TFLOP/s",
+                 "peak": burst, "frac": round(achieved / burst, 4) if achieved else None,
+                 "peak_sustained": sustained, "frac_of_sustained": round(achieved / sustained, 4) if achieved else None,
+                 "peak_source": src, "alg_flops_per_launch": gemm_flops},
         "kernels": {k: {"launches": v["launches"], "avg_us": round(1e3 * v["ms"] / max(1, v["launches"]), 2)}
                     for k, v in kern.items() if v["launches"]},
-        "gpu_launches": int(launches), "clocks": clk,
+    }
+
+
+def run_prefill(args):
+    """The prefill layer as its own bench line (rows/s)."""
+    import torch
+
+    torch.cuda.set_device(0)
+    w = wl.workload(args.workload)
+    with ClockSampler(gpu_uuid(torch, torch.device("cuda", 0))) as clocks:
+        r = measure_prefill(args.workload, args.steps, args.warmup)
+    K = args.steps
+    print(json.dumps({
+        "metric": "prefill MoE layer rows/s (8 pages x 1,156 visual tokens)", "value": r["rows_per_s"],
+        "unit": "rows/s", "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": r["ms_per_layer"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "rows": w.T, "H": w.H, "E": w.E, "top_k": w.k, "I": w.I, "I_shared": w.I_sh,
+                   "touched_experts": r["touched_experts"],
+                   "l2": "weights + activations (0.5 GB) larger than L2: no flush needed"},
+        "layer_tflops": r["layer_tflops"], "layer_frac_of_burst": r["layer_frac_of_burst"],
+        "roofline": r["gemm"], "kernels": r["kernels"],
+        "gpu_launches": r["launches"], "clocks": clocks.summary(),
     }))
     return 0
 

@@ -33,7 +33,8 @@ import numpy as np
 __all__ = [
     "Workload", "WORKLOADS", "workload", "f32_to_bf16_bits", "bf16_bits_to_f32",
     "normal_bf16", "make_layer", "make_hidden", "make_lm_head", "make_inputs",
-    "make_drafts", "hot_experts", "router_bias", "make_draft_block",
+    "make_drafts", "hot_experts", "router_bias", "make_draft_block", "layer_seeds",
+    "make_tied_lm_head",
 ]
 
 
@@ -57,6 +58,7 @@ class Workload:
     p_agree: float = 0.576
     n_hot: int = 0        # skewed routing: number of hot experts
     hot_share: float = 0.0
+    hot_bias: float = 0.0  # fp32 router-logit bias on the hot experts (the value the skew script stores)
     tie_frac: float = 0.0  # fraction of rows given near-tied LM logits
 
     @property
@@ -70,6 +72,12 @@ class Workload:
 
 MODEL = dict(H=1280, E=64, k=6, I=896, I_sh=1792, V=129280)
 
+# Router-logit bias on the 4 hot experts of the skewed-routing workload: the
+# value stored in tests/golden/skew_router_bias.json by the script beside it,
+# which bisects it on the CPU oracle so that the hot experts take 50% of the
+# top-6 slots (a CPU test re-runs that bisection and compares).
+HOT_BIAS_W4 = 1.625
+
 # The five workloads: a tiny one the oracle finishes in well under a second,
 # the batch-1 interactive case, the concurrency-32 decode verify (the headline),
 # the 8-page x 1,156-visual-token prefill layer, and the skewed-routing stress.
@@ -81,7 +89,7 @@ WORKLOADS = {
     3: Workload(3, "prefill_moe_t9248_l1", H=1280, E=64, k=6, I=896, I_sh=1792, V=0,
                 B=8, K=-1, L=1, T_override=8 * 1156),
     4: Workload(4, "skew_verify_b256_k1_l1", **MODEL, B=256, K=1, L=1, p_agree=0.9,
-                n_hot=4, hot_share=0.5, tie_frac=0.05),
+                n_hot=4, hot_share=0.5, hot_bias=HOT_BIAS_W4, tie_frac=0.05),
 }
 
 
@@ -203,23 +211,32 @@ def make_lm_head(w: Workload) -> np.ndarray | None:
     return normal_bf16(_tree(w.id)[2], (w.V, w.H), w.w_std)
 
 
+def layer_seeds(w: Workload) -> list:
+    """The seed sequence of each of the workload's L layers."""
+    return _tree(w.id)[1].spawn(w.L)
+
+
 def make_inputs(w: Workload, layers: int | None = None, norm: bool = False) -> dict:
-    """All tensors of a workload except the drafts (which need the verifier's argmax).
+    """All tensors of a workload except the drafts (which need the verifier's
+    argmax) and, for the skewed-routing workload, the near-tied LM-head rows
+    (which need the verifier's argmax too: make_tied_lm_head).
 
     ``layers`` limits how many of the L layers are drawn (for partial tests); the
-    layers that are drawn are the same bytes as in the full workload.
+    layers that are drawn are the same bytes as in the full workload.  With hot
+    experts, every layer's router carries the fp32 bias ``w.hot_bias`` on them.
     """
-    t = _tree(w.id)
     L = w.L if layers is None else min(layers, w.L)
-    layer_ss = t[1].spawn(w.L)
+    layer_ss = layer_seeds(w)
     out = {
         "hidden": make_hidden(w),
         "layers": [make_layer(w, layer_ss[l], norm) for l in range(L)],
         "w_lm": make_lm_head(w),
     }
     if w.n_hot:
-        hot = hot_experts(w)
-        out["hot_experts"] = hot
+        out["hot_experts"] = hot_experts(w)
+        out["beta"] = w.hot_bias
+        for lay in out["layers"]:
+            lay["router_bias"] = router_bias(w, w.hot_bias)
     return out
 
 
@@ -258,3 +275,33 @@ def router_bias(w: Workload, beta: float) -> np.ndarray:
 def tie_rng(w: Workload) -> np.random.Generator:
     """Random stream used to choose the rows that get near-tied LM logits."""
     return np.random.Generator(np.random.PCG64(_tree(w.id)[5]))
+
+
+def make_tied_lm_head(w: Workload, w_lm: np.ndarray, verifier_argmax: np.ndarray):
+    """Near-tied LM-head rows for ``w.tie_frac`` of the rows (seeded).
+
+    For each chosen row r, a token v2 that no row chose is given the LM-head
+    row of r's choice g: W_lm[v2] := W_lm[g] (an exact tie of the two logits);
+    for every other such row one element of W_lm[v2] is then moved by 1-4 bf16
+    codes (a gap of ~1e-4).  ``verifier_argmax`` (the choices before the ties)
+    is supplied by the caller; this function only copies rows and moves bit
+    patterns.  Returns (the new W_lm, the chosen rows, their v2 tokens).
+    """
+    rng = tie_rng(w)
+    g_first = np.asarray(verifier_argmax, dtype=np.int64)
+    T = len(g_first)
+    n = max(1, int(round(w.tie_frac * T)))
+    rows = np.sort(rng.choice(T, size=n, replace=False))
+    unused = np.setdiff1d(np.arange(w.V), np.unique(g_first))
+    v2s = rng.choice(unused, size=n, replace=False)
+    w2 = w_lm.copy()
+    for i, (r, v2) in enumerate(zip(rows, v2s)):
+        w2[v2] = w_lm[g_first[r]]
+        if i % 2:
+            while True:   # a normal, finite element: nearby codes stay same-signed and finite
+                col = int(rng.integers(0, w.H))
+                if 0x0100 <= (int(w2[v2, col]) & 0x7FFF) < 0x7F00:
+                    break
+            codes = int(rng.integers(1, 5)) * (1 if rng.random() < 0.5 else -1)
+            w2[v2, col] = np.uint16(int(w2[v2, col]) + codes)
+    return w2, rows, v2s

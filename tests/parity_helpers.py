@@ -20,63 +20,16 @@ LM_GAP = 1e-2
 MOE_TOL = 2e-2
 
 
-def bisect_router_bias(w: wl.Workload, x, layer, share=0.5, tol=0.01):
-    """Smallest-magnitude bias beta on the hot experts giving them `share` of
-    the top-k slots (within tol), found on the oracle's router."""
-    hot = wl.hot_experts(w)
-    lo, hi = 0.0, 8.0
-    beta = hi
-    for _ in range(40):
-        beta = 0.5 * (lo + hi)
-        idx, _, _, _ = oracle.router(x, layer["w_router"], w.k, bias=wl.router_bias(w, beta))
-        s = np.isin(idx, hot).mean()
-        if abs(s - share) <= tol / 4:
-            break
-        if s < share:
-            lo = beta
-        else:
-            hi = beta
-    return float(np.float32(beta))
-
-
-def add_near_ties(w: wl.Workload, w_lm, g_first):
-    """Give tie_frac of the rows an exactly tied or nearly tied LM-head row:
-    W_lm[v2] := W_lm[g] for a token v2 no row chose; half of them get one
-    element nudged by 1-4 bf16 ulps."""
-    rng = wl.tie_rng(w)
-    T = len(g_first)
-    n = max(1, int(round(w.tie_frac * T)))
-    rows = np.sort(rng.choice(T, size=n, replace=False))
-    unused = np.setdiff1d(np.arange(w.V), np.unique(g_first))
-    v2s = rng.choice(unused, size=n, replace=False)
-    w2 = w_lm.copy()
-    for i, (r, v2) in enumerate(zip(rows, v2s)):
-        w2[v2] = w_lm[g_first[r]]
-        if i % 2:
-            while True:   # a normal, finite element: nearby codes stay same-signed and finite
-                col = int(rng.integers(0, w.H))
-                if 0x0100 <= (int(w2[v2, col]) & 0x7FFF) < 0x7F00:
-                    break
-            ulps = int(rng.integers(1, 5)) * (1 if rng.random() < 0.5 else -1)
-            w2[v2, col] = np.uint16(int(w2[v2, col]) + ulps)
-    return w2, rows, v2s
-
-
 @functools.lru_cache(maxsize=4)
 def reference(wid: int, layers: int | None = None):
     """Inputs and the oracle's verify step for a workload (cached)."""
     w = wl.workload(wid)
-    inp = wl.make_inputs(w, layers)
-    if w.n_hot:
-        beta = bisect_router_bias(w, inp["hidden"], inp["layers"][0], w.hot_share)
-        for lay in inp["layers"]:
-            lay["router_bias"] = wl.router_bias(w, beta)
-        inp["beta"] = beta
+    inp = wl.make_inputs(w, layers)   # the skewed workload's router bias is part of the inputs
     st = oracle.moe_stack(inp["hidden"], inp["layers"], w.k, keep=True)
     if w.has_verify:
         am, zmax, lm_gap = oracle.lm_head_argmax(st["h"], inp["w_lm"])
-        if w.tie_frac > 0:
-            inp["w_lm"], inp["tie_rows"], inp["tie_tokens"] = add_near_ties(w, inp["w_lm"], am)
+        if w.tie_frac > 0:   # near-tied LM rows, built from the oracle's first choices
+            inp["w_lm"], inp["tie_rows"], inp["tie_tokens"] = wl.make_tied_lm_head(w, inp["w_lm"], am)
             am, zmax, lm_gap = oracle.lm_head_argmax(st["h"], inp["w_lm"])
         drafts = wl.make_drafts(w, am)
         acc, nxt, em = oracle.greedy_accept(am, drafts, w.B, w.K)
