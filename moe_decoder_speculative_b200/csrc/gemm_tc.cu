@@ -520,18 +520,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       };
       if (kTokM && S.epi == EPI_TOPK) {
         // tokens on M: this thread holds all router logits of token `row`;
-        // top-k on the logits (ties to the lower id, slots in descending
-        // order), weights exp(l_j - l_max) / sum over the kept experts.  The
-        // TMEM loads are warp-collective, so every lane issues them; only the
-        // selection and the stores depend on the row being valid.
+        // top-k on the logits, slots in descending order, weights
+        // exp(l_j - l_0) / sum over the kept experts in slot order.  The order
+        // is the one every router of this library uses: a larger logit first,
+        // equal logits (-0 equal to +0) by the lower id, a NaN after every
+        // number (-inf included), so a row with fewer than k numbers still
+        // keeps k distinct experts.  Each logit becomes one 64-bit key (its
+        // order key above the inverted expert id), so all keys differ and an
+        // empty slot (key 0) sorts below every expert.  The TMEM loads are
+        // warp-collective, so every lane issues them; only the selection and
+        // the stores depend on the row being valid.
         const bool tvalid = row < ui.nvalid;
         constexpr int kMaxK = 8;
+        uint64_t sk[kMaxK];
         float sv[kMaxK];
-        int si[kMaxK];
 #pragma unroll
         for (int j = 0; j < kMaxK; ++j) {
-          sv[j] = -__int_as_float(0x7f800000);
-          si[j] = 0x7fffffff;
+          sk[j] = 0;
+          sv[j] = 0.f;
         }
         for (int c0 = 0; c0 < S.M; c0 += 32) {
           uint32_t d[32];
@@ -541,41 +547,54 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int e = c0 + j;
+              if (e >= S.M) continue;
               float v = __uint_as_float(d[j]);
-              if (e < S.M && S.bias) v += S.bias[e];
-              if (e < S.M && v > sv[kMaxK - 1]) {  // insert, larger first; equal values keep the earlier id
+              if (S.bias) v += S.bias[e];
+              uint32_t u = __float_as_uint(v);
+              uint32_t okey;
+              if ((u & 0x7fffffffu) > 0x7f800000u) {
+                okey = 0u;  // NaN: below every number
+              } else {
+                if ((u << 1) == 0u) u = 0u;  // -0 -> +0
+                okey = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+              }
+              const uint64_t ck = (static_cast<uint64_t>(okey) << 32) | static_cast<uint64_t>(0xFFFFFFFFu - e);
+              if (ck > sk[kMaxK - 1]) {  // insert, larger key first
                 int pos = kMaxK - 1;
 #pragma unroll
                 for (int q = kMaxK - 1; q > 0; --q)
-                  if (v > sv[q - 1]) pos = q - 1;
+                  if (ck > sk[q - 1]) pos = q - 1;
 #pragma unroll
                 for (int q = kMaxK - 1; q > 0; --q)
                   if (q > pos) {
+                    sk[q] = sk[q - 1];
                     sv[q] = sv[q - 1];
-                    si[q] = si[q - 1];
                   }
 #pragma unroll
                 for (int q = 0; q < kMaxK; ++q)
                   if (q == pos) {
+                    sk[q] = ck;
                     sv[q] = v;
-                    si[q] = e;
                   }
               }
             }
           }
         }
         if (tvalid) {
+          float ex[kMaxK];
           float s = 0.f;
 #pragma unroll
-          for (int j = 0; j < kMaxK; ++j)
-            if (j < S.topk) s += expf(sv[j] - sv[0]);
+          for (int j = 0; j < kMaxK; ++j) {
+            ex[j] = (j < S.topk) ? expf(sv[j] - sv[0]) : 0.f;
+            if (j < S.topk) s += ex[j];
+          }
           int32_t* oi = static_cast<int32_t*>(S.out) + static_cast<size_t>(ui.b_row0 + row) * S.topk;
           float* ow = static_cast<float*>(S.out2) + static_cast<size_t>(ui.b_row0 + row) * S.topk;
 #pragma unroll
           for (int j = 0; j < kMaxK; ++j)
             if (j < S.topk) {
-              oi[j] = si[j];
-              ow[j] = expf(sv[j] - sv[0]) / s;
+              oi[j] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(sk[j] & 0xFFFFFFFFull));
+              ow[j] = ex[j] / s;
             }
         }
       } else if (kTokM && (S.epi == EPI_SWIGLU_ROWS || S.epi == EPI_STORE_ROWS)) {
