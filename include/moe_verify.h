@@ -121,7 +121,9 @@ MV_API mv_status moe_router_topk(const uint16_t* x, int32_t T, const mv_moe_shap
                           int32_t* topk_idx, float* topk_w, mv_stream_t stream);
 
 /* ---------------------------------------------------------------------------
- * moe_expert_permute - group the (row, slot) routing entries by expert.
+ * moe_expert_permute - group the (row, slot) routing entries by expert (model
+ * card, architecture paragraph: each token goes to 6 of 64 routed experts, so
+ * an expert's FFN runs on the rows routed to it, gathered together).
  * Entry id i = r*k + j.  counts[e] = number of entries routed to e;
  * offsets[e] = sum of counts[e'] for e' < e, offsets[E] = T*k; perm lists the
  * entry ids grouped by expert, ascending within each expert; inv[i] is the
@@ -146,7 +148,10 @@ MV_API mv_status moe_rmsnorm(const uint16_t* x, int32_t T, int32_t H, const uint
 MV_API size_t moe_ffn_workspace_size(int32_t T, const mv_moe_shape* shape);
 
 /* ---------------------------------------------------------------------------
- * moe_ffn_forward - one MoE FFN layer given its routing.
+ * moe_ffn_forward - one MoE FFN layer given its routing (model card,
+ * architecture paragraph: 64 routed experts plus 2 always-on shared experts,
+ * each row's output mixing its 6 routed experts; model card, mixture-of-
+ * experts paragraph: about 570M of the 3.4B parameters are active per token).
  * For every row r: m[r] = sum_j topk_w[r][j] * SwiGLU_{topk_idx[r][j]}(x[r])
  *                        + SwiGLU_shared(x[r]),
  * SwiGLU_e(x) = W_down[e] . bf16(silu(W_gate[e] . x) * (W_up[e] . x)),
@@ -208,7 +213,9 @@ MV_API mv_status greedy_accept(const int32_t* argmax, const int32_t* drafts, int
  *   nothing.
  *   The first call on a device looks up the array's device address (this
  *   may load the library's device code); make that first call before any
- *   stream capture.  Every call on a device shares the one array and clears
+ *   stream capture.  Later calls reuse the address while the device keeps
+ *   the same CUDA context; after cudaDeviceReset the next call looks it up
+ *   again.  Every call on a device shares the one array and clears
  *   its counter and error word on the stream, so calls that overlap on the
  *   GPU (other streams, other threads) race: serialise them.  If a bounded
  *   device-side wait ever runs out, every argmax of that call is -1.

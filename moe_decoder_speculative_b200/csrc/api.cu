@@ -1400,24 +1400,57 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+struct NoAllocAddr {
+  void* ptr = nullptr;
+  unsigned long long ctx_id = 0;  // the CUDA context the address belongs to
+};
+NoAllocAddr g_noalloc_addr[kNoAllocMaxDevices];
+
+// Unique id of the calling thread's current CUDA context (driver entry points
+// through the runtime, which the library links statically); 0 if unknown.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // Device address of the scratch array on the current device.  The array's name
-// is only a host-side stand-in, so the address is looked up once per device
-// (with that device current) and cached.
+// is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress, with the device current, once per device and context:
+// the first call on a device does it (this may load the library's device
+// code), later calls reuse it, and a call after the device's context was
+// destroyed and re-created (cudaDeviceReset) looks it up again.
 mv_status noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(MV_ERR_UNSUPPORTED_SHAPE, "device %d out of range", dev);
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
+  NoAllocAddr& a = g_noalloc_addr[dev];
+  const unsigned long long id = current_context_id();
+  if (!a.ptr || id == 0 || id != a.ctx_id) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress of the no-alloc scratch");
-    g_noalloc_addr[dev] = p;
+    a.ptr = p;
+    a.ctx_id = current_context_id();  // the lookup made the device's primary context current
   }
-  *out = g_noalloc_addr[dev];
+  *out = a.ptr;
   return MV_OK;
 }
 
