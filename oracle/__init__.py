@@ -57,9 +57,11 @@ def _load():
             f32 = ctypes.c_float
             lib.oracle_rmsnorm.argtypes = [P, i, i, P, f32, P, i]
             lib.oracle_fastmtp_draft.argtypes = [P, P, i, i, i, i, i, P, P, P, P, P, P, P, P, f32, P, P, P, i, i]
+            lib.oracle_rope.argtypes = [P, i, i, i, P, ctypes.c_double, P]
+            lib.oracle_decode_attention.argtypes = [P, P, P, P, i, i, i, i, i, P, i]
             for f in ("oracle_router", "oracle_moe_ffn", "oracle_swiglu",
                       "oracle_lm_head_argmax", "oracle_greedy_accept", "oracle_num_threads",
-                      "oracle_rmsnorm", "oracle_fastmtp_draft"):
+                      "oracle_rmsnorm", "oracle_fastmtp_draft", "oracle_rope", "oracle_decode_attention"):
                 getattr(lib, f).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -262,3 +264,40 @@ def speculative_step(hidden, drafts, B, K, layers, k, w_lm, draft, eps=RMS_EPS, 
                         n_threads=n_threads)
     st.update(draft_h0=h0, next_drafts=nxt["drafts"], draft_h_steps=nxt["h_steps"], draft_gaps=nxt["gaps"])
     return st
+
+
+ROPE_THETA = 10000.0   # rotary base of the decoder's positions (a reading; the pages give none)
+
+
+def rope(x, pos, n_heads, theta=ROPE_THETA):
+    """Rotary position embedding of every row of x [T][n_heads*d] (bf16 bits),
+    row r at position pos[r]: pairs (i, i+d/2) of each head turn by
+    pos * theta^(-2i/d).  Returns bf16 bits of the same shape."""
+    x = _u16(np.atleast_2d(x))
+    T, n = x.shape
+    d = n // n_heads
+    pos = np.ascontiguousarray(pos, np.int32)
+    y = np.zeros_like(x)
+    rc = _load().oracle_rope(_p(x), T, int(n_heads), d, _p(pos), float(theta), _p(y))
+    if rc:
+        raise ValueError("oracle_rope: invalid arguments")
+    return y
+
+
+def decode_attention(q, k_cache, v_cache, ctx_len, K, n_threads=0):
+    """Causal self-attention of the verify rows over the key/value cache.
+
+    q [B*(K+1)][nh*d] bf16 bits (row r = b*(K+1)+j, position ctx_len[b]+j);
+    k_cache, v_cache [B][nh][L_max][d] bf16 bits, holding each sequence's
+    earlier positions and this step's K+1 rows; ctx_len [B] int32.
+    Returns the outputs [B*(K+1)][nh*d] in float64 (not rounded)."""
+    k_cache, v_cache = _u16(k_cache), _u16(v_cache)
+    B, nh, L_max, d = k_cache.shape
+    q = _u16(q).reshape(B * (K + 1), nh * d)
+    ctx = np.ascontiguousarray(ctx_len, np.int32)
+    out = np.zeros((B * (K + 1), nh * d), np.float64)
+    rc = _load().oracle_decode_attention(_p(q), _p(k_cache), _p(_u16(v_cache)), _p(ctx), B, int(K), nh, d, L_max,
+                                         _p(out), int(n_threads))
+    if rc:
+        raise ValueError("oracle_decode_attention: invalid arguments")
+    return out

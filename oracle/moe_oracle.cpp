@@ -20,6 +20,9 @@
 //     paragraph: the drafts come from FastMTP, one dense draft block applied
 //     recursively for K steps (not K separate heads).  The pages give the
 //     block no shape; the reading taken is in fastmtp_draft_row below.
+//   * model card, architecture paragraph: a 32,768-position limit, the only
+//     fact the pages give about the decoder's self-attention.  The reading
+//     taken is in decode_attention_row below.
 // The pages give no formulas; the readings taken where they are silent are:
 //   gating = softmax over the E routed logits, keep the top k (selected on the
 //   logits, ties to the lower expert id, slots in descending-logit order), then
@@ -241,6 +244,52 @@ void draft_step_row(const uint16_t* h, int32_t t, int H, int Id, const uint16_t*
     h_out[i] = float_to_bf16(static_cast<float>(static_cast<Acc>(bf16_to_float(z[i])) + y[i]));
 }
 
+// Rotary position embedding of one head vector x[d] at position pos (the
+// reading of the decoder's positions): pairs (i, i + d/2) for i < d/2 turn by
+// the angle pos * theta^(-2i/d):
+//   y_i       = x_i cos(a) - x_{i+d/2} sin(a)
+//   y_{i+d/2} = x_{i+d/2} cos(a) + x_i sin(a)
+// computed in double and rounded to bf16 once.
+void rope_head(const uint16_t* x, int d, int32_t pos, double theta, uint16_t* y) {
+  const int half = d / 2;
+  for (int i = 0; i < half; ++i) {
+    const double a = static_cast<double>(pos) * std::pow(theta, -2.0 * i / d);
+    const double c = std::cos(a), s = std::sin(a);
+    const double x0 = bf16_to_float(x[i]), x1 = bf16_to_float(x[i + half]);
+    y[i] = float_to_bf16(static_cast<float>(x0 * c - x1 * s));
+    y[i + half] = float_to_bf16(static_cast<float>(x1 * c + x0 * s));
+  }
+}
+
+// Causal self-attention of one query row of one head over a sequence's key /
+// value cache (the reading of the decoder's attention on the verify rows):
+// the query at position p sees the cached positions 0..p, scores
+// s_j = (q . k_j) / sqrt(d), weights softmax(s) over those positions, output
+// o = sum_j softmax_j * v_j.  Everything in double, in ascending position and
+// index order; k_j, v_j are rows of the cache (stride d between positions).
+void decode_attention_row(const uint16_t* q, const uint16_t* k, const uint16_t* v, int d, int p, double* o) {
+  const double scale = 1.0 / std::sqrt(static_cast<double>(d));
+  std::vector<double> s(static_cast<size_t>(p) + 1);
+  double mx = -std::numeric_limits<double>::infinity();
+  for (int j = 0; j <= p; ++j) {
+    double acc = 0.0;
+    for (int i = 0; i < d; ++i)
+      acc += static_cast<double>(bf16_to_float(q[i])) * bf16_to_float(k[static_cast<size_t>(j) * d + i]);
+    s[j] = acc * scale;
+    mx = std::max(mx, s[j]);
+  }
+  double z = 0.0;
+  for (int j = 0; j <= p; ++j) {
+    s[j] = std::exp(s[j] - mx);
+    z += s[j];
+  }
+  for (int i = 0; i < d; ++i) o[i] = 0.0;
+  for (int j = 0; j <= p; ++j) {
+    const double w = s[j] / z;
+    for (int i = 0; i < d; ++i) o[i] += w * bf16_to_float(v[static_cast<size_t>(j) * d + i]);
+  }
+}
+
 void set_threads(int n_threads) {
 #ifdef _OPENMP
   if (n_threads > 0) omp_set_num_threads(n_threads);
@@ -409,6 +458,43 @@ int oracle_fastmtp_draft(const uint16_t* h0, const int32_t* t0, int B, int K, in
       t = d;
     }
   }
+  return 0;
+}
+
+// RoPE of T rows of nh heads of d values (row r at position pos[r]); x and y
+// are [T][nh*d] bf16.  d must be even.
+int oracle_rope(const uint16_t* x, int T, int nh, int d, const int32_t* pos, double theta, uint16_t* y) {
+  if (!x || !pos || !y || T < 0 || nh <= 0 || d <= 0 || (d & 1) || !(theta > 0.0)) return 1;
+  for (int r = 0; r < T; ++r)
+    for (int h = 0; h < nh; ++h) {
+      const size_t o = (static_cast<size_t>(r) * nh + h) * d;
+      rope_head(x + o, d, pos[r], theta, y + o);
+    }
+  return 0;
+}
+
+// Self-attention of the verify rows over the key/value cache.  B sequences of
+// K+1 query rows each (row r = b*(K+1) + j); sequence b holds ctx_len[b]
+// earlier positions and this step's K+1 rows at positions ctx_len[b] + j, so
+// query row j sees positions 0..ctx_len[b]+j.  q [B*(K+1)][nh][d] bf16;
+// k_cache, v_cache [B][nh][L_max][d] bf16; out [B*(K+1)][nh][d] double.
+int oracle_decode_attention(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                            const int32_t* ctx_len, int B, int K, int nh, int d, int L_max, double* out,
+                            int n_threads) {
+  if (!q || !k_cache || !v_cache || !ctx_len || !out || B < 0 || K < 0 || nh <= 0 || d <= 0 || L_max <= 0)
+    return 1;
+  for (int b = 0; b < B; ++b)
+    if (ctx_len[b] < 0 || ctx_len[b] + K + 1 > L_max) return 1;
+  set_threads(n_threads);
+  const int T = B * (K + 1);
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+  for (int r = 0; r < T; ++r)
+    for (int h = 0; h < nh; ++h) {
+      const int b = r / (K + 1), j = r % (K + 1);
+      const size_t head = (static_cast<size_t>(b) * nh + h) * static_cast<size_t>(L_max) * d;
+      decode_attention_row(q + (static_cast<size_t>(r) * nh + h) * d, k_cache + head, v_cache + head, d,
+                           ctx_len[b] + j, out + (static_cast<size_t>(r) * nh + h) * d);
+    }
   return 0;
 }
 
