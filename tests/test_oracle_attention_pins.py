@@ -164,15 +164,18 @@ def test_rope_at_position_zero_is_the_identity(oracle_mod):
 
 
 def test_rope_turns_pairs_i_and_i_plus_half(oracle_mod):
-    """d = 4: e_0 at position p becomes (cos p, 0, sin p, 0) (pairs (0, 2) and
-    (1, 3), the first pair at angle p), and e_1 turns by p / sqrt(10000) = p / 100
-    into (0, cos, 0, sin).  Interleaved pairs (0, 1) or the opposite sense fail."""
+    """d = 4: e_0 at position p becomes (cos p, 0, sin p, 0) and e_2 becomes
+    (-sin p, 0, cos p, 0) (pairs (0, 2) and (1, 3), the first pair at angle p),
+    and e_1 turns by p / sqrt(10000) = p / 100 into (0, cos, 0, sin).
+    Interleaved pairs (0, 1) or the opposite sense fail."""
     for p in (1, 3, 17):
         y0 = f(oracle_mod.rope(bf([[1, 0, 0, 0]]), np.array([p], np.int32), 1)[0])
         np.testing.assert_array_equal(y0, f(bf([np.cos(p), 0, np.sin(p), 0])))
         y1 = f(oracle_mod.rope(bf([[0, 1, 0, 0]]), np.array([p], np.int32), 1)[0])
         a = p * 10000.0 ** (-2 * 1 / 4)
         np.testing.assert_array_equal(y1, f(bf([0, np.cos(a), 0, np.sin(a)])))
+        y2 = f(oracle_mod.rope(bf([[0, 0, 1, 0]]), np.array([p], np.int32), 1)[0])
+        np.testing.assert_array_equal(y2, f(bf([-np.sin(p), 0, np.cos(p), 0])))   # the same turn, e_2 -> (-sin, cos)
 
 
 def test_rope_scores_depend_on_the_relative_position(oracle_mod):
