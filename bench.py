@@ -66,6 +66,8 @@ def parse_args():
                     help="per-step latency of one sequence (batch 1) for K = 0, 1, 3, eager and graph")
     ap.add_argument("--norm", action="store_true",
                     help="the pre-RMSNorm variant of every layer (seeded norm gains)")
+    ap.add_argument("--attention", action="store_true",
+                    help="the decoder self-attention over the key/value cache alone (decode_attention)")
     ap.add_argument("--spec", action="store_true",
                     help="the draft-and-verify loop step (speculative_step) and the FastMTP draft block alone")
     return ap.parse_args()
@@ -515,6 +517,8 @@ def run_ours(args):
         # the prefill-sized MoE layer (8 pages x 1,156 visual tokens), tensor-bound:
         # reported beside the decode step, not part of its value
         out["prefill_layer"] = measure_prefill(3, min(args.steps, 50), args.warmup)
+        # the decoder's self-attention over a 4,096-position cache (decode_attention), HBM-bound
+        out["attention"] = measure_attention(min(args.steps, 50), args.warmup)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
@@ -782,6 +786,52 @@ def measure_prefill(wid, steps, warmup):
     }
 
 
+def measure_attention(steps, warmup, B=32, K=3, n_heads=10, max_ctx=4096):
+    """The decoder's self-attention on the verify rows (decode_attention):
+    32 sequences x (K+1 = 4) rows, 10 heads of 128, each sequence with 4,096
+    cached positions (about 2 pages of 1,156 visual tokens plus their output
+    tokens).  HBM-bound: the algorithmic bytes are the visible keys and values
+    once, the queries in and the outputs out; inputs (0.67 GB) exceed L2."""
+    import torch
+
+    from moe_decoder_speculative_b200 import binding as bd
+
+    HD = 128
+    L_max = max_ctx + K + 1
+    g = torch.Generator(device="cuda").manual_seed(7)
+    q = torch.randn((B * (K + 1), n_heads * HD), device="cuda", generator=g).to(torch.bfloat16)
+    kc = torch.randn((B, n_heads, L_max, HD), device="cuda", generator=g).to(torch.bfloat16)
+    vc = torch.randn((B, n_heads, L_max, HD), device="cuda", generator=g).to(torch.bfloat16)
+    ctx = torch.full((B,), max_ctx, dtype=torch.int32, device="cuda")
+    ws = bd.workspace(bd.decode_attention_workspace_size(B, K, n_heads, max_ctx))
+    out = torch.empty_like(q)
+    for _ in range(max(3, warmup)):
+        bd.decode_attention(q, kc, vc, ctx, K, max_ctx, out=out, ws=ws)
+    torch.cuda.synchronize()
+    bd.sync_status(ws)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    bd.profile_enable(True)
+    e0.record(stream)
+    for _ in range(steps):
+        bd.decode_attention(q, kc, vc, ctx, K, max_ctx, out=out, ws=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    bd.profile_enable(False)
+    kern = bd.profile_collect().get("decode_attention", {"launches": 0, "ms": 0.0})
+    bd.sync_status(ws)
+    alg = B * n_heads * (max_ctx + K + 1) * HD * 2 * 2 + 2 * q.numel() * 2
+    avg_s = kern["ms"] / max(1, kern["launches"]) / 1e3
+    peak, src = measured_peaks()
+    gbs = alg / avg_s / 1e9 if avg_s > 0 else None
+    del q, kc, vc, out, ws
+    torch.cuda.empty_cache()
+    return {"kernel": "decode_attention", "B": B, "K": K, "n_heads": n_heads, "head_dim": HD,
+            "cached_positions": max_ctx, "avg_us": round(avg_s * 1e6, 2), "ms_per_call": e0.elapsed_time(e1) / steps,
+            "alg_bytes_per_launch": int(alg), "bound": "hbm", "achieved": round(gbs, 1) if gbs else None,
+            "unit": "GB/s", "peak": peak, "peak_source": src, "frac": round(gbs / peak, 4) if gbs else None}
+
+
 def run_prefill(args):
     """The prefill layer as its own bench line (rows/s)."""
     import torch
@@ -805,10 +855,33 @@ def run_prefill(args):
     return 0
 
 
+def run_attention(args):
+    """The decoder's self-attention on the verify rows as its own bench line."""
+    import torch
+
+    torch.cuda.set_device(0)
+    with ClockSampler(gpu_uuid(torch, torch.device("cuda", 0))) as clocks:
+        r = measure_attention(args.steps, args.warmup)
+    print(json.dumps({
+        "metric": "decode self-attention of the verify rows over the key/value cache, GB/s", "value": r["achieved"],
+        "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_call"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "attention_b32_k3_h10x128_ctx4096", "B": r["B"], "K": r["K"], "n_heads": r["n_heads"],
+                   "head_dim": r["head_dim"], "cached_positions": r["cached_positions"],
+                   "l2": "cache (0.67 GB) larger than L2: no flush needed"},
+        "roofline": {k: r[k] for k in ("kernel", "bound", "achieved", "peak", "unit", "frac", "peak_source",
+                                       "alg_bytes_per_launch")},
+        "clocks": clocks.summary(),
+    }))
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.attention:
+        return run_attention(args)
     if args.latency:
         return run_latency(args)
     if args.spec:

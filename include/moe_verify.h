@@ -342,6 +342,39 @@ MV_API mv_status verify_graph_launch(mv_verify_graph* graph, mv_stream_t stream)
 MV_API int32_t verify_graph_kernels(const mv_verify_graph* graph);
 MV_API mv_status verify_graph_destroy(mv_verify_graph* graph);
 
+/* ---------------------------------------------------------------------------
+ * decode_attention - the decoder's self-attention on the verify rows, over a
+ * key/value cache.  The jina-ocr-v1 model card (architecture paragraph) gives
+ * the decoder's attention only a 32,768-position limit; the reading this call
+ * follows is causal multi-head attention with as many key/value heads as query
+ * heads (Q, K, V, O each H x H, which keeps the card's ~570M active
+ * parameters per token) and head dim 128 (10 heads at H = 1280), keys
+ * rotated before they enter the cache.
+ * Sequence b holds ctx_len[b] earlier positions; this step's K+1 rows sit at
+ * positions ctx_len[b] + j (their keys and values already written into the
+ * cache).  For query row r = b*(K+1) + j and head h:
+ *   s_p = (q[r][h] . k_cache[b][h][p]) / sqrt(128)   for p = 0..ctx_len[b]+j
+ *   out[r][h] = sum_p softmax(s)_p * v_cache[b][h][p]
+ * in fp32 (products of bf16 values, online softmax), rounded to bf16 once.
+ *   q, out   [B*(K+1)][n_heads*128] bf16 (heads concatenated per row)
+ *   k_cache, v_cache [B][n_heads][L_max][128] bf16 (head-major, each
+ *            sequence's positions contiguous per head); positions past
+ *            ctx_len[b]+K are never read into a result
+ *   ctx_len  [B] int32, DEVICE memory; every value must satisfy
+ *            0 <= ctx_len[b] <= max_ctx and ctx_len[b] + K + 1 <= L_max.  A
+ *            value outside that range is not read past: the sequence's rows
+ *            are left unwritten and mv_sync_status reports MV_ERR_INTERNAL.
+ *   max_ctx  host-side bound on ctx_len (sizes the work split and workspace)
+ * head_dim must be 128 and K <= 7 (MV_ERR_UNSUPPORTED_SHAPE otherwise).
+ * The workspace holds the split results; calls on one workspace must not
+ * overlap in time.
+ * ------------------------------------------------------------------------- */
+MV_API size_t decode_attention_workspace_size(int32_t B, int32_t K, int32_t n_heads, int32_t max_ctx);
+MV_API mv_status decode_attention(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                                  const int32_t* ctx_len, int32_t B, int32_t K, int32_t n_heads, int32_t head_dim,
+                                  int32_t L_max, int32_t max_ctx, uint16_t* out, void* ws, size_t ws_bytes,
+                                  mv_stream_t stream);
+
 /* Clears the workspace's header (its sticky error word) on the stream.  Call
  * once on a freshly allocated workspace before its first use (a workspace
  * allocated zero-filled needs no call). */

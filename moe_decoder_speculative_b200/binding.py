@@ -26,7 +26,8 @@ EXPORTED = ["moe_router_topk", "moe_expert_permute", "moe_ffn_workspace_size", "
             "mv_launch_count", "mv_profile_enable", "mv_profile_collect", "mv_kernel_name",
             "mv_set_wait_timeout_ns", "lm_head_argmax_noalloc", "verify_graph_create", "verify_graph_launch",
             "verify_graph_kernels", "verify_graph_destroy", "fastmtp_draft_workspace_size", "fastmtp_draft",
-            "speculative_step_workspace_size", "speculative_step", "moe_rmsnorm"]
+            "speculative_step_workspace_size", "speculative_step", "moe_rmsnorm",
+            "decode_attention_workspace_size", "decode_attention"]
 
 
 class MVError(RuntimeError):
@@ -94,6 +95,8 @@ def lib():
             "fastmtp_draft_workspace_size": (sz, [i32, i32, i32, i32, i32]),
             "fastmtp_draft": (i32, [P, P, i32, i32, i32, ctypes.POINTER(DraftWeightsC), P, i32, P, P, P, sz, P]),
             "speculative_step_workspace_size": (sz, [i32, i32, S, i32, i32]),
+            "decode_attention_workspace_size": (sz, [i32, i32, i32, i32]),
+            "decode_attention": (i32, [P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, sz, P]),
             "speculative_step": (i32, [P, P, i32, i32, S, W, i32, P, i32, ctypes.POINTER(DraftWeightsC), P, P, P, P,
                                        P, P, sz, P]),
         }
@@ -248,6 +251,25 @@ def greedy_accept(argmax, drafts, B: int, K: int, emitted=True, stream=None):
     _check(lib().greedy_accept(_p(argmax), _p(drafts) if K > 0 else None, B, K, _p(acc), _p(nxt), _p(em),
                                _stream(stream)))
     return acc, nxt, em
+
+
+def decode_attention_workspace_size(B: int, K: int, n_heads: int, max_ctx: int) -> int:
+    return int(lib().decode_attention_workspace_size(B, K, n_heads, max_ctx))
+
+
+def decode_attention(q, k_cache, v_cache, ctx_len, K: int, max_ctx: int, out=None, ws=None, stream=None):
+    """Causal self-attention of the B*(K+1) verify rows q [T][n_heads*128]
+    over the cache k_cache / v_cache [B][n_heads][L_max][128] (bf16), with
+    ctx_len [B] int32 earlier positions per sequence (device tensor, every
+    value <= max_ctx).  Returns out [T][n_heads*128] bf16."""
+    B, n_heads, L_max, head_dim = k_cache.shape
+    if out is None:
+        out = torch.empty((B * (K + 1), n_heads * head_dim), dtype=torch.bfloat16, device=q.device)
+    if ws is None:
+        ws = workspace(decode_attention_workspace_size(B, K, n_heads, max_ctx), q.device)
+    _check(lib().decode_attention(_p(q), _p(k_cache), _p(v_cache), _p(ctx_len), B, K, n_heads, head_dim, L_max,
+                                  max_ctx, _p(out), _p(ws), ws.numel(), _stream(stream)))
+    return out
 
 
 def verify_step_workspace_size(B: int, K: int, shape: MoeShape, V: int) -> int:

@@ -72,12 +72,13 @@ enum Kind {
   KIND_DRAFT_LM,
   KIND_DRAFT_STEP,
   KIND_RMSNORM,
+  KIND_ATTENTION,
   KIND_COUNT
 };
 const char* kKindNames[KIND_COUNT] = {"router_topk",       "expert_permute",     "grouped_moe_gemm",
                                       "combine_unpermute", "combine_route",      "lm_head_gemm_argmax",
                                       "lm_argmax_finalize", "greedy_accept",     "draft_block_gemm",
-                                      "draft_lm_head_argmax", "draft_step", "rmsnorm"};
+                                      "draft_lm_head_argmax", "draft_step", "rmsnorm", "decode_attention"};
 
 struct ProfRec {
   int kind;
@@ -665,6 +666,46 @@ mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, in
   cudaError_t e = run_kernel(kind, st, [&] { return mv::launch_gemm(wide ? mv::GEMM_LM_WIDE : mv::GEMM_LM, p, gemm_grid(units), st); });
   if (e != cudaSuccess) return cuda_fail(e, "lm_head_gemm_argmax launch");
   return MV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// decoder self-attention over the key/value cache
+// ---------------------------------------------------------------------------
+constexpr int kAttnHeadDim = 128;
+constexpr int kAttnMaxHeads = 256;
+
+// Positions per split of one (sequence, head): a fixed 512, so the split
+// boundaries (and with them the fp32 summation order of every row) depend on
+// nothing but the position: a sequence gives the same bits whatever B, K or
+// max_ctx the call has (batch invariance).  At 128 rows and 4,096 cached
+// positions that is 9 splits per pair, 2,880 CTAs: several waves of the GPU.
+constexpr int kAttnSplit = 512;
+struct AttnPlan {
+  int split_len, n_split, nq;
+};
+AttnPlan attn_plan(int64_t B, int K, int n_heads, int max_ctx) {
+  (void)B;
+  (void)n_heads;
+  AttnPlan pl{};
+  pl.nq = mv::attention_nq(K);
+  const int64_t n_keys = static_cast<int64_t>(max_ctx) + K + 1;
+  pl.split_len = kAttnSplit;
+  pl.n_split = static_cast<int>((n_keys + kAttnSplit - 1) / kAttnSplit);
+  return pl;
+}
+
+struct AttnWs {
+  int* counters;
+  float* part_ml;
+  float* part_o;
+};
+AttnWs carve_attn(Carve& c, int64_t B, int n_heads, const AttnPlan& pl) {
+  AttnWs w;
+  const size_t pairs = static_cast<size_t>(B) * n_heads;
+  w.counters = c.take<int>(pairs);
+  w.part_ml = c.take<float>(pairs * pl.n_split * pl.nq * 2);
+  w.part_o = c.take<float>(pairs * pl.n_split * pl.nq * kAttnHeadDim);
+  return w;
 }
 
 }  // namespace
@@ -1358,6 +1399,68 @@ int32_t verify_graph_kernels(const mv_verify_graph* graph) { return graph ? grap
 mv_status verify_graph_destroy(mv_verify_graph* graph) {
   free_graph(graph);
   return MV_OK;
+}
+
+size_t decode_attention_workspace_size(int32_t B, int32_t K, int32_t n_heads, int32_t max_ctx) {
+  if (B < 0 || K < 0 || n_heads <= 0 || max_ctx < 0 || mv::attention_nq(K) == 0) return 0;
+  Carve c{nullptr};
+  c.off = kHeader;
+  carve_attn(c, B, n_heads, attn_plan(B, K, n_heads, max_ctx));
+  return c.off;
+}
+
+mv_status decode_attention(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                           const int32_t* ctx_len, int32_t B, int32_t K, int32_t n_heads, int32_t head_dim,
+                           int32_t L_max, int32_t max_ctx, uint16_t* out, void* ws, size_t ws_bytes,
+                           mv_stream_t stream) {
+  if (B < 0 || K < 0 || n_heads <= 0 || L_max <= 0 || max_ctx < 0)
+    return fail(MV_ERR_INVALID_ARG, "bad sizes B=%d K=%d n_heads=%d L_max=%d max_ctx=%d", B, K, n_heads, L_max,
+                max_ctx);
+  if (head_dim != kAttnHeadDim) return fail(MV_ERR_UNSUPPORTED_SHAPE, "head_dim=%d (only 128)", head_dim);
+  if (mv::attention_nq(K) == 0) return fail(MV_ERR_UNSUPPORTED_SHAPE, "K=%d (at most 7 drafts)", K);
+  if (n_heads > kAttnMaxHeads) return fail(MV_ERR_UNSUPPORTED_SHAPE, "n_heads=%d (at most %d)", n_heads, kAttnMaxHeads);
+  if (static_cast<int64_t>(max_ctx) + K + 1 > L_max)
+    return fail(MV_ERR_INVALID_ARG, "max_ctx + K + 1 = %lld exceeds the cache length L_max=%d",
+                static_cast<long long>(max_ctx) + K + 1, L_max);
+  if (static_cast<int64_t>(B) * n_heads * L_max >= (1LL << 31))
+    return fail(MV_ERR_UNSUPPORTED_SHAPE, "B * n_heads * L_max must stay below 2^31 cache rows");
+  MV_TRY(check_ptr(q, "q", B == 0));
+  MV_TRY(check_ptr(k_cache, "k_cache"));
+  MV_TRY(check_ptr(v_cache, "v_cache"));
+  MV_TRY(check_ptr(ctx_len, "ctx_len", B == 0));
+  MV_TRY(check_ptr(out, "out", B == 0));
+  MV_TRY(check_ptr(ws, "workspace"));
+  const size_t need = decode_attention_workspace_size(B, K, n_heads, max_ctx);
+  if (ws_bytes < need) return fail(MV_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+  if (B == 0) return MV_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const AttnPlan pl = attn_plan(B, K, n_heads, max_ctx);
+  Carve c{static_cast<char*>(ws) + kHeader};
+  const AttnWs aw = carve_attn(c, B, n_heads, pl);
+  mv::AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  const uint64_t rows = static_cast<uint64_t>(B) * n_heads * L_max;
+  MV_TRY(tmap3(&p.k_map, k_cache, rows, kAttnHeadDim, 64));
+  MV_TRY(tmap3(&p.v_map, v_cache, rows, kAttnHeadDim, 64));
+  p.q = q;
+  p.ctx_len = ctx_len;
+  p.out = out;
+  p.part_o = aw.part_o;
+  p.part_ml = aw.part_ml;
+  p.counters = aw.counters;
+  p.err = static_cast<int*>(ws);
+  p.K = K;
+  p.n_heads = n_heads;
+  p.L_max = L_max;
+  p.max_ctx = max_ctx;
+  p.split_len = pl.split_len;
+  p.n_split = pl.n_split;
+  p.scale = 1.0f / sqrtf(static_cast<float>(kAttnHeadDim));
+  p.timeout_ns = timeout_ns();
+  cudaError_t e = cudaMemsetAsync(aw.counters, 0, static_cast<size_t>(B) * n_heads * sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the attention split counters");
+  e = run_kernel(KIND_ATTENTION, st, [&] { return mv::launch_decode_attention(p, B, st); });
+  return e == cudaSuccess ? MV_OK : cuda_fail(e, "decode_attention launch");
 }
 
 mv_status mv_workspace_init(void* ws, size_t ws_bytes, mv_stream_t stream) {

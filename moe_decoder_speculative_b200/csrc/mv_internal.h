@@ -138,4 +138,26 @@ cudaError_t launch_accept_from_keys(const uint64_t* keys, int nparts, int ld, co
                                     int B, int K, int32_t* accepted, int32_t* next_token,
                                     int32_t* emitted, int32_t* argmax, cudaStream_t s);
 
+// Decoder self-attention of the verify rows over the key/value cache
+// (attention.cu).  Head dim 128; cache [B][n_heads][L_max][128] bf16 read
+// through 3D tensor maps ([k-half][row][64] view, 64-row boxes).
+struct AttnParams {
+  CUtensorMap k_map;
+  CUtensorMap v_map;
+  const uint16_t* q;        // [B*(K+1)][n_heads*128] bf16
+  const int32_t* ctx_len;   // [B]
+  uint16_t* out;            // [B*(K+1)][n_heads*128] bf16
+  float* part_o;            // [B*n_heads][n_split][NQ][128]
+  float* part_ml;           // [B*n_heads][n_split][NQ][2]: running max, sum of weights
+  int* counters;            // [B*n_heads], zero at launch
+  int* err;
+  int K, n_heads, L_max, max_ctx;
+  int split_len;            // positions per split, a multiple of 64
+  int n_split;              // grid.x: splits of the longest sequence
+  float scale;              // 1 / sqrt(128)
+  uint64_t timeout_ns;
+};
+int attention_nq(int K);  // query rows per (sequence, head) the kernel is compiled for: 1, 2, 4, 8 (0: K too large)
+cudaError_t launch_decode_attention(const AttnParams& p, int B, cudaStream_t s);
+
 }  // namespace mv

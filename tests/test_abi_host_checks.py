@@ -127,3 +127,30 @@ def test_graph_handle_calls(L):
         L.mv_profile_enable(0)
     bad = args[:14] + (need - 1,)
     assert L.verify_graph_create(*bad, ctypes.byref(g)) == WS_SMALL
+
+
+def test_decode_attention_checks(L):
+    B, K, nh, L_max, max_ctx = 2, 3, 4, 600, 512
+    need = L.decode_attention_workspace_size(B, K, nh, max_ctx)
+    assert need > 0
+    assert L.decode_attention_workspace_size(B, K, nh, 4 * max_ctx) > need
+    assert L.decode_attention_workspace_size(B, 8, nh, max_ctx) == 0          # K + 1 > 8 rows
+    ok = dict(q=A, k=A, v=A, ctx=A, B=B, K=K, nh=nh, hd=128, L=L_max, mc=max_ctx, out=A, ws=A, wsb=need)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return L.decode_attention(a["q"], a["k"], a["v"], a["ctx"], a["B"], a["K"], a["nh"], a["hd"], a["L"],
+                                  a["mc"], a["out"], a["ws"], a["wsb"], None)
+
+    assert call(B=-1) == INVALID
+    assert call(nh=0) == INVALID
+    assert call(hd=64) == SHAPE                               # head dim 128 only
+    assert call(K=8) == SHAPE                                 # at most 7 drafts
+    assert call(L=max_ctx + K) == INVALID                     # max_ctx + K + 1 > L_max
+    assert b"L_max" in L.mv_last_error()
+    assert call(q=None) == INVALID
+    assert call(v=None) == INVALID
+    assert call(ctx=A + 4) == MISALIGNED
+    assert call(out=A + 2) == MISALIGNED
+    assert call(wsb=need - 1) == WS_SMALL
+    assert call(B=0, q=None, ctx=None, out=None) == OK        # nothing to do, nothing launched
