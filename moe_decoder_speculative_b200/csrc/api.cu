@@ -417,8 +417,13 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
     S.dep_set = -1;
   };
   const bool tokm = !decode;  // large groups: tokens on the MMA's M side
+  // Large groups run on CTA pairs (cta_group::2) when pairs can be resident:
+  // 256-token units, every operand through 3D maps with 128-row boxes.
+  const int pair_clusters = tokm ? mv::gemm_pair_max_clusters() : 0;
+  const bool pair = pair_clusters > 0;
   const int bbox = decode ? mv::kDecodeBBox : mv::kPrefillBBox;
-  auto map = [decode](CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box) {
+  auto map = [decode, pair](CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box) {
+    if (pair) return tmap3(m, ptr, rows, cols, 128);
     return decode ? tmap3(m, ptr, rows, cols, box) : tmap(m, ptr, rows, cols, box);
   };
   if (Ish > 0) {  // shared expert, gate/up
@@ -502,6 +507,7 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
   }
   p.nsets = ns;
   cudaError_t e = run_kernel(KIND_GEMM_MOE, st, [&] {
+    if (pair) return mv::launch_gemm_pair(p, pair_clusters, st);
     return mv::launch_gemm(decode ? mv::GEMM_MOE_DECODE : mv::GEMM_MOE_PREFILL, p, gemm_grid(units), st);
   });
   return e == cudaSuccess ? MV_OK : cuda_fail(e, "grouped_moe_gemm launch");

@@ -30,6 +30,12 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 }
 
 cudaError_t launch_gemm(int config, const GemmParams& p, int grid, cudaStream_t stream);
+// CTA-pair (cta_group::2) form of the tokens-on-M modes (MODE_TGATEUP with
+// EPI_SWIGLU_ROWS, MODE_TPAIR with EPI_STORE_ROWS) for prefill-sized groups:
+// 256-token units, 3D tensor maps with 128-row boxes for every operand.
+// gemm_pair_max_clusters(): pairs that can be resident at once (0: unavailable).
+int gemm_pair_max_clusters();
+cudaError_t launch_gemm_pair(const GemmParams& p, int clusters, cudaStream_t stream);
 
 // Up to four device ranges a kernel prefetches into L2 before it waits for its
 // predecessor (the first weights the next GEMM will stream), split evenly over
