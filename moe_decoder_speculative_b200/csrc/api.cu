@@ -423,7 +423,7 @@ mv_status moe_gemm_impl(const uint16_t* x, int T, const mv_moe_shape& s, const m
   const bool pair = pair_clusters > 0;
   const int bbox = decode ? mv::kDecodeBBox : mv::kPrefillBBox;
   auto map = [decode, pair](CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box) {
-    if (pair) return tmap3(m, ptr, rows, cols, 128);
+    if (pair) return mv::kPairKB == 2 ? tmap3(m, ptr, rows, cols, 128) : tmap(m, ptr, rows, cols, 128);
     return decode ? tmap3(m, ptr, rows, cols, box) : tmap(m, ptr, rows, cols, box);
   };
   if (Ish > 0) {  // shared expert, gate/up

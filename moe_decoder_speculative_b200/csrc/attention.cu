@@ -38,7 +38,7 @@ constexpr int kHd = 128;          // head dim
 constexpr int kTile = 64;         // cache positions per tile
 constexpr int kTileBytes = kTile * kHd * 2;  // 16 KB per K or V tile
 constexpr int kAttnThreads = 128;
-constexpr int kQPad = 68;         // floats per query half in shared memory (64 + 4: no bank conflict between halves)
+constexpr int kQRows = 16;        // the queries padded to the MMA's N (16)
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -56,10 +56,14 @@ template <int NQ, int STAGES>
 __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* q_s = reinterpret_cast<float*>(smem + STAGES * 2 * kTileBytes);  // [NQ][2][kQPad]
-  float* p_s = q_s + NQ * 2 * kQPad;                                        // [kTile][NQ]
+  // the queries as the MMA's B operand: bf16 [2 k-blocks][16 rows][64], 128-byte swizzle
+  uint8_t* q_mma = smem + STAGES * 2 * kTileBytes;
+  float* p_s = reinterpret_cast<float*>(q_mma + 2 * kQRows * 128);  // [kTile][NQ]
   __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t s_bar;  // the tile's scores are in TMEM
+  __shared__ __align__(8) uint64_t done_bar;  // every MMA of this CTA has completed (before TMEM is freed)
   __shared__ float red_s[4][NQ];
+  __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
   __shared__ int last_s;
 
@@ -87,11 +91,20 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
   if (tid == 0) {
     abort_s = 0;
     for (int i = 0; i < STAGES; ++i) mbar_init(&full_bar[i], 1);
+    mbar_init(&s_bar, 1);
+    mbar_init(&done_bar, 1);
     fence_barrier_init();
     tma_prefetch_desc(&p.k_map);
     tma_prefetch_desc(&p.v_map);
   }
+  if (warp == 0) {  // 32 TMEM columns: the 16 score columns of one tile
+    tmem_alloc(&tmem_s, 32);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
   const uint64_t pol = policy_evict_first();
   auto issue = [&](int t) {  // tile t of this split into stage t % STAGES
     const int st = t % STAGES;
@@ -105,18 +118,26 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
   if (tid == 0)
     for (; issued < STAGES && issued < ntiles; ++issued) issue(issued);
 
-  // queries of this (sequence, head) in fp32; rows past K+1 are zero padding
-  for (int i = tid; i < NQ * kHd; i += kAttnThreads) {
-    const int j = i / kHd, c = i % kHd;
-    float v = 0.f;
-    if (j < nq) v = bf16_bits_to_f32(p.q[(static_cast<size_t>(b) * nq + j) * (p.n_heads * kHd) + h * kHd + c]);
-    q_s[(j * 2 + (c >> 6)) * kQPad + (c & 63)] = v;
+  // queries of this (sequence, head) into the swizzled B tile: row j = query
+  // j (rows past K+1 zero), 16-byte chunk c of k-block kb at
+  // kb * 2 KB + j * 128 + ((c ^ (j % 8)) * 16)
+  for (int i = tid; i < kQRows * 16; i += kAttnThreads) {
+    const int j = i >> 4, c = i & 15;  // 16 chunks of 8 dims per row
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (j < nq)
+      v = *reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * nq + j) * (p.n_heads * kHd) + h * kHd + c * 8);
+    const int kb = c >> 3, cc = c & 7;
+    *reinterpret_cast<uint4*>(q_mma + kb * (kQRows * 128) + j * 128 + ((cc ^ (j & 7)) << 4)) = v;
   }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the MMA reads the queries through the async proxy
   __syncthreads();
 
-  const int key = tid >> 1, half = tid & 1;  // QK: position `key` of the tile, dims [64 half, +64)
-  const int g = tid & 31, kg = tid >> 5;      // PV: dims [4g, 4g+4), positions kg, kg+4, ...
+  const int g = tid & 31, kg = tid >> 5;  // PV: dims [4g, 4g+4), positions kg, kg+4, ...
   const float scale = p.scale;
+  // QK on the tensor core: S[128 x 16] = K_tile[128 x 128] . Q[16 x 128]^T with
+  // the tile's 64 positions in rows 0-63 (rows 64-127 read the next 8 KB of
+  // the stage and are ignored), fp32 in TMEM lanes = positions.
+  const uint32_t idesc = idesc_bf16_f32(128, kQRows);
   float m[NQ], l_part[NQ], o[4][NQ];
 #pragma unroll
   for (int j = 0; j < NQ; ++j) {
@@ -132,66 +153,59 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
     const uint8_t* kt = smem + st * 2 * kTileBytes;
     const uint8_t* vt = kt + kTileBytes;
     if (!mbar_wait(&full_bar[st], static_cast<uint32_t>((t / STAGES) & 1), &abort_s, p.err, deadline)) ok = false;
+    tc_fence_before();
     __syncthreads();
     if (abort_s) break;  // uniform after the barrier
     const int tk0 = k0 + t * kTile;
     const int nk = min(kTile, k1 - tk0);  // valid positions in this tile
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t ka = smem_u32(kt), qb = smem_u32(q_mma);
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_bf16(tmem, smem_desc_k128(ka + kb * (kTile * 128) + kk * 32),
+                      smem_desc_k128(qb + kb * (kQRows * 128) + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+      tc_commit(&s_bar);
+    }
 
     // ---- scores: s_j = (q_j . k) * scale, -inf where position > ctx + j ----
+    const int key = tid;  // warps 0-1: position `key` of the tile (TMEM lane)
     float s[NQ];
-#pragma unroll
-    for (int j = 0; j < NQ; ++j) s[j] = 0.f;
-#pragma unroll 2
-    for (int c = 0; c < 8; ++c) {
-      const uint4 kv = *reinterpret_cast<const uint4*>(tile_chunk(kt, key, half, c));
-      float kf[8];
-      const uint32_t w4[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        kf[2 * i] = __uint_as_float(w4[i] << 16);
-        kf[2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
-      }
+    if (warp < 2) {
+      if (!mbar_wait(&s_bar, static_cast<uint32_t>(t & 1), &abort_s, p.err, deadline)) ok = false;
+      tc_fence_after();
+      uint32_t r[kQRows];
+      tmem_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16), r);
+      tmem_ld_wait();
+      const int pos = tk0 + key;
 #pragma unroll
       for (int j = 0; j < NQ; ++j) {
-        const float4* qp = reinterpret_cast<const float4*>(q_s + (j * 2 + half) * kQPad + c * 8);
-        const float4 qa = qp[0], qb = qp[1];
-        s[j] = fmaf(qa.x, kf[0], s[j]);
-        s[j] = fmaf(qa.y, kf[1], s[j]);
-        s[j] = fmaf(qa.z, kf[2], s[j]);
-        s[j] = fmaf(qa.w, kf[3], s[j]);
-        s[j] = fmaf(qb.x, kf[4], s[j]);
-        s[j] = fmaf(qb.y, kf[5], s[j]);
-        s[j] = fmaf(qb.z, kf[6], s[j]);
-        s[j] = fmaf(qb.w, kf[7], s[j]);
+        const bool vis = key < nk && j < nq && pos <= ctx + j;
+        s[j] = vis ? __uint_as_float(r[j]) * scale : -__int_as_float(0x7f800000);
+        float v = s[j];
+#pragma unroll
+        for (int o2 = 1; o2 < 32; o2 <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o2));
+        if (lane == 0) red_s[warp][j] = v;
       }
     }
-    const int pos = tk0 + key;
-    float tmax[NQ];
-#pragma unroll
-    for (int j = 0; j < NQ; ++j) {
-      s[j] += __shfl_xor_sync(0xffffffffu, s[j], 1);  // the two halves of the position
-      const bool vis = key < nk && j < nq && pos <= ctx + j;
-      s[j] = vis ? s[j] * scale : -__int_as_float(0x7f800000);
-      float v = s[j];
-#pragma unroll
-      for (int o2 = 2; o2 < 32; o2 <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o2));
-      tmax[j] = v;
-    }
-    if (lane == 0)
-#pragma unroll
-      for (int j = 0; j < NQ; ++j) red_s[warp][j] = tmax[j];
+    tc_fence_before();
     __syncthreads();
+    if (abort_s) break;
     float alpha[NQ];
 #pragma unroll
     for (int j = 0; j < NQ; ++j) {
-      const float tm = fmaxf(fmaxf(red_s[0][j], red_s[1][j]), fmaxf(red_s[2][j], red_s[3][j]));
+      const float tm = fmaxf(red_s[0][j], red_s[1][j]);
       const float mn = fmaxf(m[j], tm);
       const bool none = (mn == -__int_as_float(0x7f800000));  // nothing visible yet for this query
       alpha[j] = none ? 1.f : expf(m[j] - mn);
-      const float pj = (none || s[j] == -__int_as_float(0x7f800000)) ? 0.f : expf(s[j] - mn);
+      if (warp < 2) {
+        const float pj = (none || s[j] == -__int_as_float(0x7f800000)) ? 0.f : expf(s[j] - mn);
+        l_part[j] = l_part[j] * alpha[j] + pj;
+        p_s[key * NQ + j] = pj;
+      }
       m[j] = mn;
-      l_part[j] = l_part[j] * alpha[j] + (half == 0 ? pj : 0.f);
-      if (half == 0) p_s[key * NQ + j] = pj;
     }
     __syncthreads();
 
@@ -200,7 +214,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
     for (int d = 0; d < 4; ++d)
 #pragma unroll
       for (int j = 0; j < NQ; ++j) o[d][j] *= alpha[j];
-    const int vhalf = g >> 4, vchunk = (g & 15) >> 1, vsub = (g & 1) * 8;
+  const int vhalf = g >> 4, vchunk = (g & 15) >> 1, vsub = (g & 1) * 8;
     for (int kk = kg; kk < nk; kk += 4) {
       const uint2 vv = *reinterpret_cast<const uint2*>(tile_chunk(vt, kk, vhalf, vchunk) + vsub);
       const float vf[4] = {__uint_as_float(vv.x << 16), __uint_as_float(vv.x & 0xFFFF0000u),
@@ -231,6 +245,17 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
       ++issued;
     }
   }
+
+  // No MMA is issued after the loop: wait for the last ones, then free TMEM.
+  if (tid == 0) {
+    tc_commit(&done_bar);
+    int dummy = 0;
+    mbar_wait(&done_bar, 0, &dummy, p.err, globaltimer_ns() + kDrainNs);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 32);
 
   if (!ok || abort_s) {
     // Drain: every issued copy must land before the CTA exits.
@@ -316,7 +341,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
 
 // Dynamic shared memory of one CTA: the tile ring, the queries, the weights.
 static size_t attention_smem(int nq_t, int stages) {
-  return static_cast<size_t>(stages) * 2 * kTileBytes + static_cast<size_t>(nq_t) * 2 * kQPad * 4 +
+  return static_cast<size_t>(stages) * 2 * kTileBytes + static_cast<size_t>(2) * kQRows * 128 +
          static_cast<size_t>(kTile) * nq_t * 4 + 1024;
 }
 

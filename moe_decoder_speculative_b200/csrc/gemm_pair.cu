@@ -40,8 +40,9 @@ namespace {
 
 constexpr int kPairThreads = 192;
 constexpr int kHalfTile = 128 * 128;           // 128 rows x 64 bf16 (one k-block)
-constexpr int kPairStageBytes = 4 * kHalfTile;  // A: 2 k-blocks x 128 rows, B: 2 k-blocks x 128 rows = 64 KB
-constexpr int kPairStages = 3;
+constexpr int kKB = kPairKB;                   // k-blocks per stage
+constexpr int kPairStageBytes = 2 * kKB * kHalfTile;  // A: kKB k-blocks x 128 rows, B: the same
+constexpr int kPairStages = 6 / kKB;           // 192 KB of stages
 constexpr int kPairTok = 256;                  // token rows per unit (128 per CTA)
 constexpr int kAccCols = 256;                  // one accumulator: 256 columns; two of them
 
@@ -64,6 +65,17 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
 
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// 2D tiled TMA load into this CTA's shared memory whose completion counts on
+// the barrier at `bar_cluster` (the even CTA's), for a CTA-pair MMA.
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* m, int32_t x, int32_t y,
+                                                 uint32_t bar_cluster, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(bar_cluster), "l"(policy)
+      : "memory");
 }
 
 // 3D tiled TMA load into this CTA's shared memory whose completion counts on
@@ -250,7 +262,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     return ui;
   };
   const int my_units = total_units > cluster ? (total_units - cluster + nclusters - 1) / nclusters : 0;
-  auto unit_stages = [&](const GemmSet& S) { return (S.K / 64 + 1) / 2; };
+  auto unit_stages = [&](const GemmSet& S) { return (S.K / 64 + kKB - 1) / kKB; };
 
   if (warp == 0) {
     // ========================= TMA producer ==================================
@@ -296,9 +308,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           }
           uint8_t* st = smem + stage * kPairStageBytes;
           // both CTAs' A and B boxes (a box past the last k-block is zero-filled and still counts)
-          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 8u * kHalfTile);
-          tma_load_3d_pair(st, &S.b, 0, t_row, 2 * ks, full0 + stage * 8, pol_x);
-          tma_load_3d_pair(st + 2 * kHalfTile, wmap, 0, w_row, 2 * ks, full0 + stage * 8, pol_w);
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2u * kPairStageBytes);
+          if (kKB == 2) {  // one 3D box brings two k-blocks
+            tma_load_3d_pair(st, &S.b, 0, t_row, 2 * ks, full0 + stage * 8, pol_x);
+            tma_load_3d_pair(st + kKB * kHalfTile, wmap, 0, w_row, 2 * ks, full0 + stage * 8, pol_w);
+          } else {
+            tma_load_2d_pair(st, &S.b, ks * 64, t_row, full0 + stage * 8, pol_x);
+            tma_load_2d_pair(st + kKB * kHalfTile, wmap, ks * 64, w_row, full0 + stage * 8, pol_w);
+          }
           fills[stage]++;
           if (++stage == kPairStages) {
             stage = 0;
@@ -343,10 +360,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           tc_fence_after();
           const uint32_t st = smem_u32(smem + stage * kPairStageBytes);
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (h == 1 && 2 * ks + 1 >= kblocks) break;
+          for (int h = 0; h < kKB; ++h) {
+            if (h > 0 && kKB * ks + h >= kblocks) break;
             const uint32_t a = st + h * kHalfTile;            // token rows, k-block h
-            const uint32_t b = st + (2 + h) * kHalfTile;      // weight rows, k-block h
+            const uint32_t b = st + (kKB + h) * kHalfTile;    // weight rows, k-block h
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               tc_mma_pair(d0, smem_desc_k128(a + kk * 32), smem_desc_k128(b + kk * 32), idesc,
@@ -396,7 +413,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
               for (int q = 0; q < 2; ++q) {
                 const float gf = __uint_as_float(g[2 * j + q]);
                 const float uf = __uint_as_float(v[2 * j + q]);
-                a2[q] = (gf / (1.0f + expf(-gf))) * uf;
+                // silu(g) * u = g u / (1 + e^-g) with the fast exponential and
+                // division (a few ulp of fp32, far below the bf16 rounding of a);
+                // the IEEE forms made this epilogue the kernel's bottleneck
+                a2[q] = __fdividef(gf * uf, 1.0f + __expf(-gf));
               }
               packed[j] = static_cast<uint32_t>(f32_to_bf16_bits(a2[0])) |
                           (static_cast<uint32_t>(f32_to_bf16_bits(a2[1])) << 16);

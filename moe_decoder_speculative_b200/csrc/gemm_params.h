@@ -25,6 +25,12 @@ enum { GEMM_MOE_DECODE = 0, GEMM_MOE_PREFILL = 1, GEMM_LM = 2, GEMM_LM_WIDE = 3 
 constexpr int kDecodeBBox = 32;  // GEMM_MOE_DECODE: one 3D box of 32 token rows x two k-blocks
 constexpr int kPrefillBBox = MV_PREFILL_BBOX;
 constexpr int kLmBBox = 16;       // GEMM_LM: few token rows
+// CTA-pair prefill GEMM: 64-wide k-blocks per stage (1: 2D boxes, six 32 KB
+// stages; 2: 3D boxes, three 64 KB stages).
+#ifndef MV_PAIR_KB
+#define MV_PAIR_KB 2
+#endif
+constexpr int kPairKB = MV_PAIR_KB;
 constexpr int kLmWideBBox = 128;  // GEMM_LM_WIDE: 128 or more token rows
 
 // Sticky device error bits, OR-ed into the workspace's error word.
