@@ -39,7 +39,11 @@
  *               this interface.
  *   Determinism Every result is a deterministic function of the inputs: no
  *               floating-point atomics, and the same row gives the same bits
- *               whatever other rows share its batch.
+ *               whatever other rows share its batch, among batches of one
+ *               size class: decode-sized batches (T*k <= 16*E routed entries,
+ *               T <= 1024) run one set of tile forms, larger ones another
+ *               (tokens on the MMA's M side, CTA pairs, the tensor-core
+ *               router), whose fp32 sums differ in the last bits.
  */
 #ifndef MOE_VERIFY_H
 #define MOE_VERIFY_H
