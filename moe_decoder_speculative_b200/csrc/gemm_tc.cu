@@ -532,13 +532,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         // the stores depend on the row being valid.
         const bool tvalid = row < ui.nvalid;
         constexpr int kMaxK = 8;
-        uint64_t sk[kMaxK];
-        float sv[kMaxK];
+        // Two independent sorted lists (even and odd experts of each chunk of
+        // 32), so consecutive insertions do not wait on each other, merged at
+        // the end.  An insertion keeps a list sorted, larger key first.
+        uint64_t ka[kMaxK], kb[kMaxK];
+        float va[kMaxK], vb[kMaxK];
 #pragma unroll
         for (int j = 0; j < kMaxK; ++j) {
-          sk[j] = 0;
-          sv[j] = 0.f;
+          ka[j] = kb[j] = 0;
+          va[j] = vb[j] = 0.f;
         }
+        auto insert = [](uint64_t (&sk)[kMaxK], float (&sv)[kMaxK], uint64_t ck, float v) {
+          if (ck > sk[kMaxK - 1]) {
+#pragma unroll
+            for (int q = 0; q < kMaxK; ++q) {  // carry the smaller of (slot, candidate) down the list
+              const bool gt = ck > sk[q];
+              const uint64_t tk = gt ? sk[q] : ck;
+              const float tv = gt ? sv[q] : v;
+              sk[q] = gt ? ck : sk[q];
+              sv[q] = gt ? v : sv[q];
+              ck = tk;
+              v = tv;
+            }
+          }
+        };
         for (int c0 = 0; c0 < S.M; c0 += 32) {
           uint32_t d[32];
           tmem_ld32(tl + c0, d);
@@ -559,27 +576,38 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 okey = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
               }
               const uint64_t ck = (static_cast<uint64_t>(okey) << 32) | static_cast<uint64_t>(0xFFFFFFFFu - e);
-              if (ck > sk[kMaxK - 1]) {  // insert, larger key first
-                int pos = kMaxK - 1;
-#pragma unroll
-                for (int q = kMaxK - 1; q > 0; --q)
-                  if (ck > sk[q - 1]) pos = q - 1;
-#pragma unroll
-                for (int q = kMaxK - 1; q > 0; --q)
-                  if (q > pos) {
-                    sk[q] = sk[q - 1];
-                    sv[q] = sv[q - 1];
-                  }
-#pragma unroll
-                for (int q = 0; q < kMaxK; ++q)
-                  if (q == pos) {
-                    sk[q] = ck;
-                    sv[q] = v;
-                  }
-              }
+              if (j & 1)
+                insert(kb, vb, ck, v);
+              else
+                insert(ka, va, ck, v);
             }
           }
         }
+        // merge: the k largest of the two lists are max(ka[i], kb[7 - i])
+        // (a bitonic sequence), sorted by a bitonic network of 3 x 4 steps
+        uint64_t sk[kMaxK];
+        float sv[kMaxK];
+#pragma unroll
+        for (int i = 0; i < kMaxK; ++i) {
+          const bool ga = ka[i] > kb[kMaxK - 1 - i];
+          sk[i] = ga ? ka[i] : kb[kMaxK - 1 - i];
+          sv[i] = ga ? va[i] : vb[kMaxK - 1 - i];
+        }
+#pragma unroll
+        for (int step = kMaxK / 2; step > 0; step >>= 1)
+#pragma unroll
+          for (int i = 0; i < kMaxK; ++i)
+            if ((i & step) == 0) {
+              const int jx = i + step;
+              if (sk[jx] > sk[i]) {  // larger key first
+                const uint64_t tk = sk[i];
+                const float tv = sv[i];
+                sk[i] = sk[jx];
+                sv[i] = sv[jx];
+                sk[jx] = tk;
+                sv[jx] = tv;
+              }
+            }
         if (tvalid) {
           float ex[kMaxK];
           float s = 0.f;

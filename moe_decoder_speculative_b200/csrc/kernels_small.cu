@@ -967,6 +967,11 @@ cudaError_t launch_permute_sorted(const int32_t* idx, int T, int E, int k, int32
 // Each product and sum is rounded separately (no fused multiply-add), in the
 // order written.  One thread owns 8 consecutive hidden features of a row.
 // ---------------------------------------------------------------------------
+// Combine: out[r] = bf16(res[r] + (sum_j w[r][j] * y[pos(r, j)] + y_sh[r])), the
+// products and sums singly rounded, in slot order with the shared expert last.
+// One warp per row: lanes 0..k-1 load the row's routing once and broadcast it,
+// then each lane combines 8-column chunks lane, lane + 32, ...; all the loads
+// of a chunk (k expert rows, the shared row, the residual) issue together.
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y_perm,
                                                       const float* __restrict__ y_sh,
                                                       const int32_t* __restrict__ inv,
@@ -978,65 +983,75 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   prefetch_share(pf);
   pdl_wait();
   const int hv = H / 8;
-  const long long total = static_cast<long long>(T) * hv;
-  for (long long t = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; t < total;
-       t += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int r = static_cast<int>(t / hv);
-    const int c = static_cast<int>(t % hv);
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < T; r += nwarps) {  // uniform per warp
+    const int pl = (lane < k) ? inv[static_cast<size_t>(r) * k + lane] : -1;
+    const float wl = (lane < k) ? w[static_cast<size_t>(r) * k + lane] : 0.f;
     int pos[8];
     float wj[8];
+    bool okj[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      pos[j] = (j < k) ? inv[static_cast<size_t>(r) * k + j] : -1;
-      wj[j] = (j < k) ? w[static_cast<size_t>(r) * k + j] : 0.f;
+      pos[j] = __shfl_sync(0xffffffffu, pl, j);
+      wj[j] = __shfl_sync(0xffffffffu, wl, j);
+      okj[j] = (j < k) && pos[j] >= 0 && pos[j] < n_pos;
     }
-    float4 ya[8], yb[8];
+    bool bad = false;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      // by entry, the row address needs no routing data: the loads issue with those of inv
-      const bool ok = by_entry ? (j < k) : (pos[j] >= 0 && pos[j] < n_pos);
-      const size_t yrow = by_entry ? static_cast<size_t>(r) * k + j : static_cast<size_t>(pos[j]);
-      if (ok) {
-        const float4* yp = reinterpret_cast<const float4*>(y_perm + yrow * H) + 2 * c;
-        ya[j] = yp[0];
-        yb[j] = yp[1];
-      } else {
-        ya[j] = yb[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < 8; ++j) bad |= (j < k) && !okj[j];
+    if (lane == 0 && err && bad) atomicOr(err, kErrInternal);  // an entry routed to no valid expert
+    for (int c = lane; c < hv; c += 32) {
+      float4 ya[8], yb[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        // by entry, the row address needs no routing data
+        const bool ld = by_entry ? (j < k) : okj[j];
+        const size_t yrow = by_entry ? static_cast<size_t>(r) * k + j : static_cast<size_t>(pos[j]);
+        if (ld) {
+          const float4* yp = reinterpret_cast<const float4*>(y_perm + yrow * H) + 2 * c;
+          ya[j] = yp[0];
+          yb[j] = yp[1];
+        } else {
+          ya[j] = yb[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
-    }
-    float m[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m[i] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j >= k) continue;
-      if (pos[j] < 0 || pos[j] >= n_pos) {  // entry routed to no valid expert
-        if (err && c == 0) atomicOr(err, kErrInternal);
-        continue;
+      float4 sa = make_float4(0.f, 0.f, 0.f, 0.f), sb = sa;
+      if (y_sh) {
+        const float4* ys = reinterpret_cast<const float4*>(y_sh + static_cast<size_t>(r) * H) + 2 * c;
+        sa = ys[0];
+        sb = ys[1];
       }
-      const float yv[8] = {ya[j].x, ya[j].y, ya[j].z, ya[j].w, yb[j].x, yb[j].y, yb[j].z, yb[j].w};
+      uint4 rv = make_uint4(0, 0, 0, 0);
+      if (res) rv = reinterpret_cast<const uint4*>(res + static_cast<size_t>(r) * H)[c];
+      float m[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(m[i], __fmul_rn(wj[j], yv[i]));
+      for (int i = 0; i < 8; ++i) m[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (!okj[j]) continue;
+        const float yv[8] = {ya[j].x, ya[j].y, ya[j].z, ya[j].w, yb[j].x, yb[j].y, yb[j].z, yb[j].w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(m[i], __fmul_rn(wj[j], yv[i]));
+      }
+      if (y_sh) {
+        const float yv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(m[i], yv[i]);
+      }
+      if (res) {
+        float rf[8];
+        bf16x8_to_f32(rv, rf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(rf[i], m[i]);
+      }
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        o[i] = static_cast<uint32_t>(f32_to_bf16_bits(m[2 * i])) |
+               (static_cast<uint32_t>(f32_to_bf16_bits(m[2 * i + 1])) << 16);
+      reinterpret_cast<uint4*>(out + static_cast<size_t>(r) * H)[c] = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    if (y_sh) {
-      const float4* ys = reinterpret_cast<const float4*>(y_sh + static_cast<size_t>(r) * H) + 2 * c;
-      const float4 a = ys[0], b = ys[1];
-      const float yv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(m[i], yv[i]);
-    }
-    if (res) {
-      float rf[8];
-      bf16x8_to_f32(reinterpret_cast<const uint4*>(res + static_cast<size_t>(r) * H)[c], rf);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m[i] = __fadd_rn(rf[i], m[i]);
-    }
-    uint32_t o[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      o[i] = static_cast<uint32_t>(f32_to_bf16_bits(m[2 * i])) |
-             (static_cast<uint32_t>(f32_to_bf16_bits(m[2 * i + 1])) << 16);
-    reinterpret_cast<uint4*>(out + static_cast<size_t>(r) * H)[c] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -1044,8 +1059,7 @@ cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t
                            const float* w, const uint16_t* res, uint16_t* out, int T, int H,
                            int k, int n_pos, int* err, const L2Prefetch& pf, cudaStream_t s, bool y_by_entry) {
   if (T <= 0) return cudaSuccess;
-  const long long total = static_cast<long long>(T) * (H / 8);
-  const long long blocks = (total + 255) / 256;
+  const long long blocks = (static_cast<long long>(T) + 7) / 8;  // 8 rows (warps) per CTA
   int grid = static_cast<int>(blocks < 148LL * 8 ? blocks : 148LL * 8);
   if (grid < prefetch_ctas(pf)) grid = prefetch_ctas(pf);  // the grid-stride loop leaves the extra CTAs idle
   return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, s, y_perm, y_sh, inv, w, res, out, T, H, k, n_pos, err,
