@@ -63,3 +63,31 @@ def test_out_of_range_expert_ids_are_reported():
         bd.sync_status(ws)
     assert exc.value.status == 7  # MV_ERR_INTERNAL
     bd.sync_status(ws)
+
+
+def test_wait_bound_runs_out_in_the_verify_step_and_context_survives():
+    """The whole verify step with a 1 ns bound: the waits of its routing, GEMM
+    and LM-head launches run out; the kernels drain their copies, exit and the
+    step reports MV_ERR_TIMEOUT.  With the default bound restored the same
+    step gives the same tokens as before."""
+    w, inp, st = reference(0)
+    shape = bd.shape_of(w)
+    plan = bd.VerifyPlan(shape, [bd.LayerWeights(l) for l in inp["layers"]], bd.bf16_to_device(inp["w_lm"]),
+                         w.B, w.K)
+    hidden = bd.bf16_to_device(inp["hidden"])
+    d = torch.from_numpy(st["drafts"]).cuda()
+    good = [t.cpu().numpy().copy() for t in plan(hidden, d)]
+    plan.sync_status()
+    try:
+        bd.set_wait_timeout_ns(1)
+        plan(hidden, d)
+        with pytest.raises(bd.MVError) as exc:
+            plan.sync_status()
+        assert exc.value.status == 6  # MV_ERR_TIMEOUT
+    finally:
+        bd.set_wait_timeout_ns(0)
+    plan.sync_status()
+    again = [t.cpu().numpy() for t in plan(hidden, d)]
+    plan.sync_status()
+    for a, b in zip(good, again):
+        np.testing.assert_array_equal(a, b)

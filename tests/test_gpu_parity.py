@@ -480,3 +480,55 @@ def test_prefill_groups_of_every_size():
     m_ref, _ = oracle.moe_ffn(x[rows], lay, idx[rows], tw[rows])
     m_gpu = wl.bf16_bits_to_f32(bd.bf16_from_device(out))[rows]
     assert moe_error(m_gpu, m_ref) <= MOE_TOL
+
+
+def _biased_reference(wid, layers, dead):
+    """Oracle reference of a workload whose router bias is -30 on the `dead`
+    experts in every layer, so that no row chooses them."""
+    w = wl.workload(wid)
+    inp = wl.make_inputs(w, layers)
+    for lay in inp["layers"]:
+        b = np.zeros(w.E, np.float32) if lay.get("router_bias") is None else lay["router_bias"].copy()
+        b[dead] = -30.0
+        lay["router_bias"] = b
+    st = oracle.moe_stack(inp["hidden"], inp["layers"], w.k, keep=True)
+    am, _, lm_gap = oracle.lm_head_argmax(st["h"], inp["w_lm"])
+    drafts = wl.make_drafts(w, am)
+    acc, nxt, em = oracle.greedy_accept(am, drafts, w.B, w.K)
+    st.update(argmax=am, lm_gap=lm_gap, drafts=drafts, accepted=acc, next_token=nxt, emitted=em)
+    for lay in st["layers"]:
+        assert not np.isin(lay["idx"], dead).any()
+    return w, inp, st
+
+
+def test_verify_step_with_experts_no_row_chooses_tiny():
+    """Tiny workload (16 rows, top-2 of 8 experts) with experts 0 and 5 chosen
+    by no row: their groups are empty in every layer (no units, no outputs
+    read by the combine).  Every row equals the oracle."""
+    w, inp, st = _biased_reference(0, None, [0, 5])
+    _, _, _, acc, nxt, em, am = run_verify(w, inp, st["drafts"])
+    check_verify(w, st, acc, nxt, em, am, exact_all=True)
+
+
+def test_verify_step_with_experts_no_row_chooses_conc32():
+    """The concurrency-32 batch (128 rows, top-6 of 64) through 2 layers with
+    experts 3, 17, 40 and 63 chosen by no row (empty slabs in both layers, the
+    second layer's routing fused with the first layer's combine).  Unflagged
+    rows equal the oracle, and the step's argmax equals the public per-layer
+    calls' (router, grouped FFN, LM head) bit for bit."""
+    w, inp, st = _biased_reference(2, 2, [3, 17, 40, 63])
+    plan, hidden, d, acc, nxt, em, am = run_verify(w, inp, st["drafts"])
+    check_verify(w, st, acc, nxt, em, am)
+    _, _, am_chain = gpu_layer_chain(w, inp, plan, hidden)
+    np.testing.assert_array_equal(am_chain, am)
+
+
+def test_verify_step_two_layers_equals_the_per_layer_calls():
+    """Concurrency-32 batch, 2 layers, no bias: the step (slab grouping inside
+    the fused combine-route kernel) and the public per-layer calls give the
+    same argmax bit for bit, and unflagged rows equal the oracle."""
+    w, inp, st = reference(2, 2)
+    plan, hidden, d, acc, nxt, em, am = run_verify(w, inp, st["drafts"])
+    check_verify(w, st, acc, nxt, em, am)
+    _, _, am_chain = gpu_layer_chain(w, inp, plan, hidden)
+    np.testing.assert_array_equal(am_chain, am)
