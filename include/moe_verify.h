@@ -43,7 +43,9 @@
  *               size class: decode-sized batches (T*k <= 16*E routed entries,
  *               T <= 1024) run one set of tile forms, larger ones another
  *               (tokens on the MMA's M side, CTA pairs, the tensor-core
- *               router), whose fp32 sums differ in the last bits.
+ *               router), whose fp32 sums differ in the last bits.  The LM
+ *               head has its own two classes: below 256 rows and from 256
+ *               rows (CTA pairs).
  */
 #ifndef MOE_VERIFY_H
 #define MOE_VERIFY_H

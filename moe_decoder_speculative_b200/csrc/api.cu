@@ -339,6 +339,10 @@ constexpr int kMaxLayers = 64;  // decoder layers one verify_step call may run
 
 int lm_parts(int V) { return (V + 255) / 256 * 4; }  // (256-row vocabulary tile, lane quarter)
 int lm_parts_alloc(int V) { return (V + 127) / 128 * 4; }  // any split into 256- and 128-row tiles
+#ifndef MV_LM_PAIR_MIN_ROWS
+#define MV_LM_PAIR_MIN_ROWS 256
+#endif
+constexpr int kLmPairMinRows = MV_LM_PAIR_MIN_ROWS;  // LM heads of this many rows or more run on CTA pairs
 
 uint64_t timeout_ns() {
   const int64_t t = g_timeout_ns.load();
@@ -619,6 +623,39 @@ mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, in
   p.err = err;
   p.sched = sched;
   p.timeout_ns = timeout_ns();
+  // From 256 rows the contraction is tensor-bound (each vocabulary tile is
+  // reused by several token tiles) and runs on CTA pairs: 256 tokens x 256
+  // vocabulary rows per unit, each SM loading half of both, so a k-block
+  // costs an SM 32 KB of shared-memory fill instead of 48 KB.
+  const int pair_clusters = T >= kLmPairMinRows ? mv::gemm_pair_max_clusters() : 0;
+  if (pair_clusters > 0) {
+    mv::GemmSet& S = p.set[0];
+    S.mode = mv::MODE_TLM;
+    S.epi = mv::EPI_ARGMAX_ROWS;
+    S.m_tile = 256;
+    S.dep_set = -1;
+    const auto pmap = [](CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
+      return mv::kPairKB == 2 ? tmap3(m, ptr, rows, cols, 128) : tmap(m, ptr, rows, cols, 128);
+    };
+    MV_TRY(pmap(&S.a0, w_lm, V, H));
+    MV_TRY(pmap(&S.b, h, T, H));
+    S.a1 = S.a0;
+    S.out = parts;
+    S.ld_out = ld;
+    S.K = H;
+    S.M = V;
+    S.groups = 1;
+    S.static_rows = T;
+    p.nsets = 1;
+    const int used = (V + 255) / 256;  // one key per token and 256-row vocabulary tile
+    if (used > ld) return fail(MV_ERR_INTERNAL, "LM key slots %d exceed the row stride %d", used, ld);
+    *nparts_used = used;
+    const int64_t units = int64_t(used) * ((T + 255) / 256);
+    const int clusters = static_cast<int>(std::min<int64_t>(pair_clusters, units));
+    cudaError_t e = run_kernel(kind, st, [&] { return mv::launch_gemm_pair(p, clusters, st); });
+    if (e != cudaSuccess) return cuda_fail(e, "lm_head_gemm_argmax launch");
+    return MV_OK;
+  }
   const int nt = (T + 127) / 128;
   const bool wide = T >= 128;  // whole 128-row token tiles: one TMA box per stage
   const int bbox = wide ? mv::kLmWideBBox : mv::kLmBBox;
@@ -1567,14 +1604,14 @@ mv_status noalloc_scratch(void** out) {
 // if a bounded device-side wait of the GEMM ran out (the callers of this path
 // have no workspace through which to read the error word).
 __global__ void __launch_bounds__(128) noalloc_finalize_kernel(const uint64_t* __restrict__ keys, int nparts,
-                                                               int T, int32_t* __restrict__ argmax,
+                                                               int ld, int T, int32_t* __restrict__ argmax,
                                                                const int* __restrict__ err) {
   __shared__ uint64_t red[4];
   mv::pdl_trigger();
   mv::pdl_wait();
   const int t = blockIdx.x;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const uint64_t* row = keys + static_cast<size_t>(t) * nparts;
+  const uint64_t* row = keys + static_cast<size_t>(t) * ld;  // the first nparts keys of the row are written
   uint64_t best = 0;
   for (int p = threadIdx.x; p < nparts; p += 128) {
     const uint64_t v = row[p];
@@ -1624,7 +1661,7 @@ extern "C" MV_API mv_status lm_head_argmax_noalloc(const uint16_t* h, int32_t T,
   MV_TRY(lm_gemm_impl(h, T, H, w_lm, V, parts, lm_parts(V), err, sched, st, false, &used));
   e = run_kernel(KIND_LM_FINALIZE, st, [&] {
     return mv::launch_pdl(noalloc_finalize_kernel, dim3(T), dim3(128), 0, st, static_cast<const uint64_t*>(parts),
-                          lm_parts(V), static_cast<int>(T), argmax, static_cast<const int*>(err));
+                          used, lm_parts(V), static_cast<int>(T), argmax, static_cast<const int*>(err));
   });
   return e == cudaSuccess ? MV_OK : cuda_fail(e, "no-alloc argmax finalize launch");
 }

@@ -1,7 +1,9 @@
 // Grouped tensor-core GEMM on CTA pairs (tcgen05 cta_group::2) for the large
 // token groups of a prefill-sized MoE layer (8 pages x 1,156 visual tokens:
 // about 870 rows per routed expert; jina-ocr-v1 model card, architecture
-// paragraph: 64 routed + 2 shared SwiGLU experts).
+// paragraph: 64 routed + 2 shared SwiGLU experts), and for the LM head of 256
+// or more rows (129,280-token vocabulary, same paragraph), where each
+// vocabulary tile serves several token tiles and the tensor core bounds it.
 //
 // Why pairs.  With one CTA per tile (128 tokens x 256 weight rows) every
 // 64-wide k-block writes 48 KB into shared memory and the MMAs read the same
@@ -21,7 +23,8 @@
 //   warp 1      TMEM allocation (cta_group::2, both CTAs); MMA issue (even
 //               CTA only): M = 256 (128 rows per CTA), N = 256 (128 per CTA)
 //   warps 2..5  epilogue on this CTA's 128 token rows x 256 columns (gate|up
-//               -> SwiGLU, or two halves of W_down -> fp32 rows)
+//               -> SwiGLU, or two halves of W_down -> fp32 rows, or 256 LM-head
+//               rows -> one argmax key per token)
 // Units (group, M tile, 256-token tile) are assigned statically: cluster c
 // takes c, c + clusters, c + 2 clusters, ...  A down unit waits (bounded
 // acquire-poll) until every epilogue warp of both CTAs of every unit of its
@@ -441,6 +444,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                                    __uint_as_float(d[4 * q + 2]), __uint_as_float(d[4 * q + 3]));
           }
         }
+      } else if (S.epi == EPI_ARGMAX_ROWS) {
+        // LM head: this thread's token row holds the logits of vocabulary rows
+        // m0 .. m0 + 255 (this CTA's 128 and the other CTA's 128).  Per group
+        // of 32 rows: the first row's logit, then any strictly larger one (so
+        // the lowest index among equal maxima), packed with its index into a
+        // key (larger logit first, then lower index); rows past the vocabulary
+        // count as -inf.  The largest of the 8 keys is the unit's; tokens
+        // reduce their keys over all units afterwards.
+        uint64_t best_key = 0;
+        for (int c0 = 0; c0 < 256; c0 += 32) {
+          uint32_t d[32];
+          tmem_ld32(tl + c0, d);
+          tmem_ld_wait();
+          const int v0 = ui.m0 + c0;
+          float best = v0 < S.M ? __uint_as_float(d[0]) : -__int_as_float(0x7f800000);
+          int bi = 0;
+#pragma unroll
+          for (int j = 1; j < 32; ++j) {
+            const float x = (v0 + j < S.M) ? __uint_as_float(d[j]) : -__int_as_float(0x7f800000);
+            if (x > best) {
+              best = x;
+              bi = j;
+            }
+          }
+          const uint64_t key = argmax_key(best, static_cast<uint32_t>(S.key_row_base + v0 + bi));
+          best_key = key > best_key ? key : best_key;
+        }
+        if (tvalid) static_cast<uint64_t*>(S.out)[orow + S.key_part_base + ui.m0 / 256] = best_key;
       } else if (lane == 0) {
         atomicOr(p.err, kErrInternal);  // a set this kernel is not built for
       }

@@ -7,12 +7,14 @@
 namespace mv {
 
 enum { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_ARGMAX = 2, EPI_SWIGLU_ROWS = 3, EPI_STORE_ROWS = 4, EPI_TOPK = 5,
-       EPI_STORE_BF16 = 6 };  // EPI_STORE_BF16: bf16(res + acc), res nullable (swap-AB tiles)
+       EPI_STORE_BF16 = 6,    // bf16(res + acc), res nullable (swap-AB tiles)
+       EPI_ARGMAX_ROWS = 7 }; // CTA pairs, tokens on M: one argmax key per (token, 256 vocabulary rows)
 // Operand modes.  The first four put weights on the MMA's M side (swap-AB);
 // the tokens-on-M modes load the same tiles but multiply 128 token rows by 256
 // weight rows (gate|up tiles, or two halves of W_down) into one accumulator.
 enum { MODE_SINGLE = 0, MODE_GATEUP = 1, MODE_KPAIR = 2, MODE_MPAIR = 3, MODE_TGATEUP = 4, MODE_TPAIR = 5,
-       MODE_TROUTE = 6 };  // MODE_TROUTE: 128 token rows x the M (<= 256) router rows, one accumulator
+       MODE_TROUTE = 6,  // 128 token rows x the M (<= 256) router rows, one accumulator
+       MODE_TLM = 7 };   // CTA pairs: 256 token rows x 256 LM-head rows (128 of each per CTA)
 enum { GEMM_MOE_DECODE = 0, GEMM_MOE_PREFILL = 1, GEMM_LM = 2, GEMM_LM_WIDE = 3 };
 
 // B-operand TMA box height (rows) of each tile configuration; the host builds

@@ -216,6 +216,30 @@ def test_lm_head_ragged_vocab_and_rows():
     np.testing.assert_array_equal(am[ok], ref[ok])
 
 
+@pytest.mark.parametrize("T", [256, 300, 513])
+def test_lm_head_pairs_ragged_vocab_and_rows(T):
+    """From 256 rows the LM head runs on CTA pairs (256 tokens x 256
+    vocabulary rows per unit): a vocabulary that is not a multiple of 256, a
+    ragged last token tile, a reduction of 3 k-blocks (one stage half empty),
+    and vocabulary rows 7 and 900 made equal to rows 3 and 500 so that exact
+    ties occur and must go to the lower index."""
+    rng = np.random.default_rng(50 + T)
+    H, V = 192, 1000
+    h = wl.f32_to_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    wlm = wl.f32_to_bf16_bits(rng.standard_normal((V, H)).astype(np.float32) * 0.05)
+    wlm[7] = wlm[3]
+    wlm[900] = wlm[500]
+    h[:40] = wl.f32_to_bf16_bits(wl.bf16_bits_to_f32(wlm[3]) * 4.0)   # rows 3 and 7 lead, tied
+    ref, _, gap = oracle.lm_head_argmax(h, wlm)
+    am = to_np(bd.lm_head_argmax(bd.bf16_to_device(h), bd.bf16_to_device(wlm)))
+    ok = gap >= LM_GAP
+    assert ok.mean() > 0.5
+    np.testing.assert_array_equal(am[ok], ref[ok])
+    tied = gap == 0
+    np.testing.assert_array_equal(am[tied], ref[tied])
+    assert np.all(ref[:40] == 3) and np.all(am[:40] == 3)
+
+
 def test_greedy_accept_exhaustive():
     rng = np.random.default_rng(6)
     for K in (0, 1, 3, 7):
