@@ -717,12 +717,14 @@ mv_status lm_gemm_impl(const uint16_t* h, int T, int H, const uint16_t* w_lm, in
 constexpr int kAttnHeadDim = 128;
 constexpr int kAttnMaxHeads = 256;
 
-// Positions per split of one (sequence, head): a fixed 512, so the split
+// Positions per split of one (sequence, head): a fixed 1,024, so the split
 // boundaries (and with them the fp32 summation order of every row) depend on
 // nothing but the position: a sequence gives the same bits whatever B, K or
 // max_ctx the call has (batch invariance).  At 128 rows and 4,096 cached
-// positions that is 9 splits per pair, 2,880 CTAs: several waves of the GPU.
-constexpr int kAttnSplit = 512;
+// positions that is 5 splits per pair, 1,600 CTAs: several waves of the GPU
+// (512-position splits measured 7 % slower: twice the per-CTA set-up and
+// merge for the same bytes).
+constexpr int kAttnSplit = 1024;
 struct AttnPlan {
   int split_len, n_split, nq;
 };

@@ -18,9 +18,11 @@
 //     memory with the 128-byte swizzle (bank-conflict-free row reads);
 //   * CTA (split, head, sequence) streams its split of the positions through
 //     a ring of STAGES tiles with an online softmax in fp32;
-//   * QK: two threads per position (one per 64-dim half), the queries in
-//     shared memory; PV: a thread owns 4 dims of the output for a quarter of
-//     the positions; partial outputs are summed in a fixed order;
+//   * QK on the tensor core: the tile's K rows are the A operand of an
+//     M = 128 MMA, the queries (padded to 16 rows) the B operand, the scores
+//     land in TMEM and warps 0-1 read them (one position per thread); PV on
+//     the CUDA cores: a thread owns 4 dims of the output for a quarter of the
+//     positions; partial outputs are summed in a fixed order;
 //   * splits of one (sequence, head) are merged by the last CTA to finish
 //     (an atomic count per pair), in split order: deterministic.
 // Every wait is bounded; a CTA that gives up drains its copies, sets the

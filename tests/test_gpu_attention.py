@@ -72,7 +72,7 @@ def test_decode_attention_conc32_rows_over_thousands_of_positions():
     max_ctx = 4096
     rng = np.random.default_rng(1)
     ctx = rng.integers(0, max_ctx + 1, size=B)
-    ctx[:6] = [0, 1, 508, 509, 4096, 4092]   # n_keys = 4, 5, 512 (one whole split), 513, 4100, 4096
+    ctx[:8] = [0, 1, 508, 509, 1020, 1021, 4096, 4092]   # n_keys = 4, 5, 512, 513, 1024 (one whole split), 1025, 4100, 4096
     L_max = max_ctx + K + 1
     q, kc, vc, ctx = make_case(2, B, K, nh, ctx, L_max)
     got, _ = run_gpu(q, kc, vc, ctx, K, max_ctx)
