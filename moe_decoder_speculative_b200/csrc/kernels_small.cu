@@ -963,15 +963,13 @@ cudaError_t launch_permute_sorted(const int32_t* idx, int T, int E, int k, int32
 }
 
 // ---------------------------------------------------------------------------
-// Combine: m = sum_j w_j * y_j (slot order) + y_shared, out = bf16(res + m).
-// Each product and sum is rounded separately (no fused multiply-add), in the
-// order written.  One thread owns 8 consecutive hidden features of a row.
-// ---------------------------------------------------------------------------
 // Combine: out[r] = bf16(res[r] + (sum_j w[r][j] * y[pos(r, j)] + y_sh[r])), the
-// products and sums singly rounded, in slot order with the shared expert last.
-// One warp per row: lanes 0..k-1 load the row's routing once and broadcast it,
-// then each lane combines 8-column chunks lane, lane + 32, ...; all the loads
-// of a chunk (k expert rows, the shared row, the residual) issue together.
+// products and sums singly rounded (no fused multiply-add), in slot order with
+// the shared expert last.  A warp task is one 256-element slice of a row:
+// lanes 0..k-1 load the row's routing and broadcast it, then lane l combines
+// the 8 consecutive features of chunk 32 * slice + l; all the loads of a chunk
+// (k expert rows, the shared row, the residual) issue together.
+// ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y_perm,
                                                       const float* __restrict__ y_sh,
                                                       const int32_t* __restrict__ inv,
@@ -985,7 +983,13 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   const int hv = H / 8;
   const int lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
-  for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < T; r += nwarps) {  // uniform per warp
+  // A warp task is one 32-chunk slice (256 elements) of one row, so that a
+  // decode batch of a hundred rows still spreads over every launched warp.
+  const int nslice = (hv + 31) / 32;
+  const long long ntask = static_cast<long long>(T) * nslice;
+  for (long long q = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; q < ntask; q += nwarps) {  // uniform per warp
+    const int r = static_cast<int>(q / nslice);
+    const int slice = static_cast<int>(q - static_cast<long long>(r) * nslice);
     const int pl = (lane < k) ? inv[static_cast<size_t>(r) * k + lane] : -1;
     const float wl = (lane < k) ? w[static_cast<size_t>(r) * k + lane] : 0.f;
     int pos[8];
@@ -1000,8 +1004,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     bool bad = false;
 #pragma unroll
     for (int j = 0; j < 8; ++j) bad |= (j < k) && !okj[j];
-    if (lane == 0 && err && bad) atomicOr(err, kErrInternal);  // an entry routed to no valid expert
-    for (int c = lane; c < hv; c += 32) {
+    if (lane == 0 && slice == 0 && err && bad) atomicOr(err, kErrInternal);  // an entry routed to no valid expert
+    const int c = slice * 32 + lane;
+    if (c < hv) {
       float4 ya[8], yb[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -1059,7 +1064,8 @@ cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t
                            const float* w, const uint16_t* res, uint16_t* out, int T, int H,
                            int k, int n_pos, int* err, const L2Prefetch& pf, cudaStream_t s, bool y_by_entry) {
   if (T <= 0) return cudaSuccess;
-  const long long blocks = (static_cast<long long>(T) + 7) / 8;  // 8 rows (warps) per CTA
+  const long long tasks = static_cast<long long>(T) * ((H / 8 + 31) / 32);  // (row, 256-element slice)
+  const long long blocks = (tasks + 7) / 8;  // 8 tasks (warps) per CTA
   int grid = static_cast<int>(blocks < 148LL * 8 ? blocks : 148LL * 8);
   if (grid < prefetch_ctas(pf)) grid = prefetch_ctas(pf);  // the grid-stride loop leaves the extra CTAs idle
   return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, s, y_perm, y_sh, inv, w, res, out, T, H, k, n_pos, err,
