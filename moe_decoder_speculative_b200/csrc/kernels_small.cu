@@ -1073,27 +1073,35 @@ cudaError_t launch_combine(const float* y_perm, const float* y_sh, const int32_t
 }
 
 // ---------------------------------------------------------------------------
-// LM-head argmax finalisation: the GEMM epilogue leaves, per token, one packed
-// (order-preserving logit, inverted index) key per 32-row vocabulary block,
-// token-major ([T][nparts]); the largest key is the argmax with ties to the
-// lower index.  `nthr` threads (a multiple of 32) reduce one token's keys with
-// coalesced, unrolled loads.
+// LM-head argmax finalisation: the GEMM epilogue leaves, per token, packed
+// (order-preserving logit, inverted index) keys, token-major ([T][nparts]):
+// one per (256-row vocabulary tile, lane quarter) of the single-CTA tiles, or
+// one per 256-row tile on CTA pairs; the largest key is the argmax with ties
+// to the lower index.  `nthr` threads (a multiple of 32) reduce one token's
+// keys with coalesced, unrolled loads.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint64_t umax64(uint64_t a, uint64_t b) { return a > b ? a : b; }
 
 __device__ __forceinline__ uint64_t row_max_key(const uint64_t* row, int nparts, int t0, int nthr,
                                                 uint64_t* red, int lane, int wid) {
-  uint64_t b[8];
+  // sixteen independent loads in flight per thread: 256 threads cover the
+  // 2,264 keys of a 129,280-row vocabulary in one round trip
+  constexpr int kInFlight = 16;
+  uint64_t b[kInFlight];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) b[i] = 0;
-  for (int p0 = t0; p0 < nparts; p0 += 8 * nthr) {  // eight independent loads in flight per thread
+  for (int i = 0; i < kInFlight; ++i) b[i] = 0;
+  for (int p0 = t0; p0 < nparts; p0 += kInFlight * nthr) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kInFlight; ++i) {
       const int p = p0 + i * nthr;
       if (p < nparts) b[i] = umax64(b[i], row[p]);
     }
   }
-  uint64_t best = umax64(umax64(umax64(b[0], b[1]), umax64(b[2], b[3])), umax64(umax64(b[4], b[5]), umax64(b[6], b[7])));
+#pragma unroll
+  for (int w = kInFlight / 2; w > 0; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) b[i] = umax64(b[i], b[i + w]);
+  uint64_t best = b[0];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) best = umax64(best, __shfl_xor_sync(0xffffffffu, best, o));
   if (lane == 0) red[wid] = best;
