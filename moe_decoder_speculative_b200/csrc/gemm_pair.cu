@@ -48,6 +48,7 @@ constexpr int kPairStageBytes = 2 * kKB * kHalfTile;  // A: kKB k-blocks x 128 r
 constexpr int kPairStages = 6 / kKB;           // 192 KB of stages
 constexpr int kPairTok = 256;                  // token rows per unit (128 per CTA)
 constexpr int kAccCols = 256;                  // one accumulator: 256 columns; two of them
+constexpr int kPairTBufBytes = 4 * 32 * 33 * 4;  // fp32 32 x 33 transpose buffer per epilogue warp
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -388,6 +389,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   } else {
     // ========================= epilogue (warps 2..5, both CTAs) ==============
     const int wq = warp & 3;
+    float* tbuf = reinterpret_cast<float*>(smem + kPairStages * kPairStageBytes);
     const uint32_t tempty0 = map_to_rank(&tempty_bar[0], 0);
     for (int it = 0; it < my_units; ++it) {
       const PairUnit ui = decode(cluster + it * nclusters);
@@ -431,18 +433,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           }
         }
       } else if (S.epi == EPI_STORE_ROWS) {
+        // fp32 rows, written line by line: the warp's 32 rows x 32 columns
+        // pass through a padded buffer (row writes and column reads both
+        // bank-conflict-free), then each store instruction writes one row's
+        // 32 columns, a whole 128-byte line, instead of 16 bytes of 32 rows.
         float* out = static_cast<float*>(S.out);
+        float* tb = tbuf + wq * (32 * 33);
+        const int row_base = ui.b_row0 + 128 * static_cast<int>(rank) + wq * 32;
+        const int rows_here = min(32, nvalid - wq * 32);  // valid rows of this warp (may be <= 0)
         for (int c0 = 0; c0 < 256; c0 += 32) {
           uint32_t d[32];
           tmem_ld32(tl + c0, d);
           tmem_ld_wait();
-          if (tvalid && ui.m0 + c0 < S.M) {
-            float4* dst = reinterpret_cast<float4*>(out + orow + ui.m0 + c0);
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              dst[q] = make_float4(__uint_as_float(d[4 * q]), __uint_as_float(d[4 * q + 1]),
-                                   __uint_as_float(d[4 * q + 2]), __uint_as_float(d[4 * q + 3]));
-          }
+          for (int j = 0; j < 32; ++j) tb[lane * 33 + j] = __uint_as_float(d[j]);
+          __syncwarp();
+          const int col = ui.m0 + c0 + lane;
+          if (col < S.M)
+            for (int r = 0; r < rows_here; ++r)
+              out[static_cast<size_t>(row_base + r) * S.ld_out + col] = tb[r * 33 + lane];
+          __syncwarp();
         }
       } else if (S.epi == EPI_ARGMAX_ROWS) {
         // LM head: this thread's token row holds the logits of vocabulary rows
@@ -502,7 +512,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-static size_t pair_smem() { return static_cast<size_t>(kPairStages) * kPairStageBytes + 1024; }
+// The stage ring, the epilogue warps' 32 x 33 transpose buffers, alignment.
+static size_t pair_smem() { return static_cast<size_t>(kPairStages) * kPairStageBytes + kPairTBufBytes + 1024; }
 
 static cudaError_t pair_configure(int dev) {
   static thread_local int configured_dev = -1;
