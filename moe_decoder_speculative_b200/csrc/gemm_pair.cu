@@ -271,7 +271,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   if (warp == 0) {
     // ========================= TMA producer ==================================
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
+      // Weights stream once per token tile: kept in L2 (evict-last) when
+      // three or more token tiles of the group read the same weight tile, so
+      // the later readers hit; streamed through (evict-first) otherwise.
+      const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
       const uint32_t full0 = map_to_rank(&full_bar[0], 0);  // the even CTA's barriers
       int stage = 0;
@@ -299,6 +302,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           asm volatile("fence.proxy.async.global;" ::: "memory");
         }
         const int nstage = unit_stages(S);
+        const uint64_t pol_w = g_nt[ui.g] >= 3 ? pol_x : pol_stream;
         const bool gu = (S.mode == MODE_TGATEUP);
         // this CTA's weight rows: gate (even) / up (odd) of the 128-feature
         // tile, or the even / odd 128-row half of a 256-row W_down tile
