@@ -288,9 +288,14 @@ class VerifyPlan:
         self.c_layers = arr
         self.ws = workspace(verify_step_workspace_size(B, K, shape, self.V), device)
         T = B * (K + 1)
-        self.accepted = torch.empty(B, dtype=torch.int32, device=device)
-        self.next_token = torch.empty(B, dtype=torch.int32, device=device)
-        self.emitted = torch.empty((B, K + 1), dtype=torch.int32, device=device)
+        # the per-sequence results side by side in one block (`results`), so
+        # that a caller reads them back with one copy; each part starts on a
+        # 16-byte boundary, as the C interface requires
+        Bp = (B + 3) // 4 * 4
+        self.results = torch.empty(2 * Bp + B * (K + 1), dtype=torch.int32, device=device)
+        self.accepted = self.results[:B]
+        self.next_token = self.results[Bp:Bp + B]
+        self.emitted = self.results[2 * Bp:].view(B, K + 1)
         self.argmax = torch.empty(T, dtype=torch.int32, device=device)
 
     def __call__(self, hidden, drafts, stream=None):
@@ -343,9 +348,14 @@ class SpeculativePlan:
         n = int(lib().speculative_step_workspace_size(B, K, ctypes.byref(shape), draft.I_d, self.V))
         self.ws = workspace(n, device)
         T = B * (K + 1)
-        self.accepted = torch.empty(B, dtype=torch.int32, device=device)
-        self.next_token = torch.empty(B, dtype=torch.int32, device=device)
-        self.emitted = torch.empty((B, K + 1), dtype=torch.int32, device=device)
+        # the per-sequence results side by side in one block (`results`), so
+        # that a caller reads them back with one copy; each part starts on a
+        # 16-byte boundary, as the C interface requires
+        Bp = (B + 3) // 4 * 4
+        self.results = torch.empty(2 * Bp + B * (K + 1), dtype=torch.int32, device=device)
+        self.accepted = self.results[:B]
+        self.next_token = self.results[Bp:Bp + B]
+        self.emitted = self.results[2 * Bp:].view(B, K + 1)
         self.argmax = torch.empty(T, dtype=torch.int32, device=device)
         self.next_drafts = torch.empty((B, max(1, K)), dtype=torch.int32, device=device)
 
