@@ -10,7 +10,8 @@
 //
 // A decode step has K+1 queries per (sequence, head) against thousands of
 // cached positions: 4 flops per byte of cache, far below the tensor cores'
-// ridge, so this is a streaming kernel on the CUDA cores, bound by HBM.
+// ridge, so this is a streaming kernel bound by HBM; the MMAs only keep the
+// per-tile instruction count (and so the latency chain) short.
 // Layout and work split:
 //   * cache [B][heads][L_max][128] bf16 (head-major), so a tile of 64
 //     positions of one (sequence, head) is 16 KB of contiguous rows; one TMA
@@ -20,9 +21,12 @@
 //     a ring of STAGES tiles with an online softmax in fp32;
 //   * QK on the tensor core: the tile's K rows are the A operand of an
 //     M = 128 MMA, the queries (padded to 16 rows) the B operand, the scores
-//     land in TMEM and warps 0-1 read them (one position per thread); PV on
-//     the CUDA cores: a thread owns 4 dims of the output for a quarter of the
-//     positions; partial outputs are summed in a fixed order;
+//     land in TMEM and warps 0-1 read them (one position per thread);
+//   * PV on the tensor cores too, as warp-level MMAs (mma.sync m16n8k16, fp32
+//     accumulators in registers): V^T tiles straight from the swizzled stage
+//     (ldmatrix.trans), the softmax weights as two bf16 parts (high and the
+//     rounding remainder, summing to the fp32 weight within 2^-18 of it), so
+//     the products keep fp32 accuracy; warp w owns output dims [32w, 32w+32);
 //   * splits of one (sequence, head) are merged by the last CTA to finish
 //     (an atomic count per pair), in split order: deterministic.
 // Every wait is bounded; a CTA that gives up drains its copies, sets the
@@ -46,12 +50,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// bf16 element `col` (0..127) of row `row` of a swizzled [half][64 rows][64]
-// tile: 16-byte chunk index XOR (row % 8) within each 128-byte row.
-__device__ __forceinline__ const uint8_t* tile_chunk(const uint8_t* tile, int row, int half, int chunk) {
-  return tile + half * (kTile * 128) + row * 128 + ((chunk ^ (row & 7)) << 4);
-}
-
 }  // namespace
 
 template <int NQ, int STAGES>
@@ -60,7 +58,9 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // the queries as the MMA's B operand: bf16 [2 k-blocks][16 rows][64], 128-byte swizzle
   uint8_t* q_mma = smem + STAGES * 2 * kTileBytes;
-  float* p_s = reinterpret_cast<float*>(q_mma + 2 * kQRows * 128);  // [kTile][NQ]
+  // the tile's softmax weights as bf16 high and low parts, [8 queries][64 positions] each
+  uint16_t* p_hi = reinterpret_cast<uint16_t*>(q_mma + 2 * kQRows * 128);
+  uint16_t* p_lo = p_hi + 8 * kTile;
   __shared__ __align__(8) uint64_t full_bar[STAGES];
   __shared__ __align__(8) uint64_t s_bar;  // the tile's scores are in TMEM
   __shared__ __align__(8) uint64_t done_bar;  // every MMA of this CTA has completed (before TMEM is freed)
@@ -134,20 +134,25 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the MMA reads the queries through the async proxy
   __syncthreads();
 
-  const int g = tid & 31, kg = tid >> 5;  // PV: dims [4g, 4g+4), positions kg, kg+4, ...
+  // PV on the tensor cores (mma.sync m16n8k16, fp32 accumulators): warp w
+  // owns output dims [32w, 32w + 32) as two 16-dim tiles; thread (gq, tq) of
+  // a tile holds dims gq, gq + 8 for queries 2 tq, 2 tq + 1.
+  const int gq = lane >> 2, tq = lane & 3;
   const float scale = p.scale;
   // QK on the tensor core: S[128 x 16] = K_tile[128 x 128] . Q[16 x 128]^T with
   // the tile's 64 positions in rows 0-63 (rows 64-127 read the next 8 KB of
   // the stage and are ignored), fp32 in TMEM lanes = positions.
   const uint32_t idesc = idesc_bf16_f32(128, kQRows);
-  float m[NQ], l_part[NQ], o[4][NQ];
+  float m[NQ], l_part[NQ], o[2][4];
 #pragma unroll
   for (int j = 0; j < NQ; ++j) {
     m[j] = -__int_as_float(0x7f800000);
     l_part[j] = 0.f;
-#pragma unroll
-    for (int d = 0; d < 4; ++d) o[d][j] = 0.f;
   }
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) o[t][q] = 0.f;
 
   bool ok = true;
   for (int t = 0; t < ntiles; ++t) {
@@ -205,42 +210,73 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
       if (warp < 2) {
         const float pj = (none || s[j] == -__int_as_float(0x7f800000)) ? 0.f : expf(s[j] - mn);
         l_part[j] = l_part[j] * alpha[j] + pj;
-        p_s[key * NQ + j] = pj;
+        // bf16 high and low parts: p_hi + p_lo = pj to 2^-18 of it
+        const uint16_t hi = f32_to_bf16_bits(pj);
+        p_hi[j * kTile + key] = hi;
+        p_lo[j * kTile + key] = f32_to_bf16_bits(pj - bf16_bits_to_f32(hi));
       }
       m[j] = mn;
     }
+    if (nk < kTile) {  // the rows past the split (never visible) may hold anything: zero them for the MMAs
+      uint8_t* vz = const_cast<uint8_t*>(vt);
+      for (int i = tid; i < (kTile - nk) * 16; i += kAttnThreads) {
+        const int r = nk + (i >> 4), c = i & 15;  // row r, 16-byte chunk c of the two 64-dim halves
+        *reinterpret_cast<uint4*>(vz + (c >> 3) * (kTile * 128) + r * 128 + (c & 7) * 16) = make_uint4(0, 0, 0, 0);
+      }
+    }
     __syncthreads();
 
-    // ---- o += p . v over this tile's valid positions ----
+    // ---- o = o * alpha + P V^T on the tensor cores ----
+    {
+      float a_lo = 1.f, a_hi = 1.f;  // alpha of queries 2 tq, 2 tq + 1
 #pragma unroll
-    for (int d = 0; d < 4; ++d)
-#pragma unroll
-      for (int j = 0; j < NQ; ++j) o[d][j] *= alpha[j];
-  const int vhalf = g >> 4, vchunk = (g & 15) >> 1, vsub = (g & 1) * 8;
-    for (int kk = kg; kk < nk; kk += 4) {
-      const uint2 vv = *reinterpret_cast<const uint2*>(tile_chunk(vt, kk, vhalf, vchunk) + vsub);
-      const float vf[4] = {__uint_as_float(vv.x << 16), __uint_as_float(vv.x & 0xFFFF0000u),
-                           __uint_as_float(vv.y << 16), __uint_as_float(vv.y & 0xFFFF0000u)};
-      float pk[NQ];
-      if constexpr (NQ >= 4) {
-#pragma unroll
-        for (int j = 0; j < NQ; j += 4) {
-          const float4 p4 = *reinterpret_cast<const float4*>(p_s + kk * NQ + j);
-          pk[j] = p4.x;
-          pk[j + 1] = p4.y;
-          pk[j + 2] = p4.z;
-          pk[j + 3] = p4.w;
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < NQ; ++j) pk[j] = p_s[kk * NQ + j];
+      for (int j = 0; j < NQ; ++j) {
+        if (j == 2 * tq) a_lo = alpha[j];
+        if (j == 2 * tq + 1) a_hi = alpha[j];
       }
 #pragma unroll
-      for (int d = 0; d < 4; ++d)
+      for (int t = 0; t < 2; ++t) {
+        o[t][0] *= a_lo;
+        o[t][1] *= a_hi;
+        o[t][2] *= a_lo;
+        o[t][3] *= a_hi;
+      }
+      const uint32_t vbase = smem_u32(vt);
+      const int li = lane >> 3;  // the 8 x 8 matrix this lane addresses: dims + 8 (li & 1), positions + 8 (li >> 1)
 #pragma unroll
-        for (int j = 0; j < NQ; ++j) o[d][j] = fmaf(pk[j], vf[d], o[d][j]);
+      for (int ks = 0; ks < kTile / 16; ++ks) {
+        uint32_t bh0 = 0, bh1 = 0, bl0 = 0, bl1 = 0;  // P^T: positions 16 ks + 2 tq (+1) and +8, query gq
+        if (gq < NQ) {
+          const int pp = gq * kTile + 16 * ks + 2 * tq;
+          bh0 = *reinterpret_cast<const uint32_t*>(p_hi + pp);
+          bh1 = *reinterpret_cast<const uint32_t*>(p_hi + pp + 8);
+          bl0 = *reinterpret_cast<const uint32_t*>(p_lo + pp);
+          bl1 = *reinterpret_cast<const uint32_t*>(p_lo + pp + 8);
+        }
+        const int pos = 16 * ks + 8 * (li >> 1) + (lane & 7);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int dim = warp * 32 + t * 16 + 8 * (li & 1);
+          const uint32_t addr = vbase + static_cast<uint32_t>((dim >> 6) * (kTile * 128) + pos * 128) +
+                                static_cast<uint32_t>((((dim & 63) >> 3) ^ (pos & 7)) << 4);
+          uint32_t a0, a1, a2, a3;  // V^T: dims x positions
+          asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
+                       : "r"(addr));
+          asm volatile(
+              "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+              "{%0, %1, %2, %3};"
+              : "+f"(o[t][0]), "+f"(o[t][1]), "+f"(o[t][2]), "+f"(o[t][3])
+              : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(bh0), "r"(bh1));
+          asm volatile(
+              "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+              "{%0, %1, %2, %3};"
+              : "+f"(o[t][0]), "+f"(o[t][1]), "+f"(o[t][2]), "+f"(o[t][3])
+              : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(bl0), "r"(bl1));
+        }
+      }
     }
-    __syncthreads();  // every thread is done with this stage and with p_s
+    __syncthreads();  // every thread is done with this stage and with the weights
     if (tid == 0 && issued < ntiles) {
       fence_proxy_async_smem();  // order the reads of this stage before the copy that refills it
       issue(issued);
@@ -271,8 +307,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
     return;
   }
 
-  // ---- reduce l over positions and o over the four position groups (fixed order) ----
-  float* o_red = reinterpret_cast<float*>(smem);  // [4][NQ][128]; the ring is idle now
+  // ---- l over positions (fixed order); each thread's outputs are already whole ----
 #pragma unroll
   for (int j = 0; j < NQ; ++j) {
     float v = l_part[j];
@@ -284,24 +319,22 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
   if (lane == 0)
 #pragma unroll
     for (int j = 0; j < NQ; ++j) red_s[warp][j] = l_part[j];
-#pragma unroll
-  for (int d = 0; d < 4; ++d)
-#pragma unroll
-    for (int j = 0; j < NQ; ++j) o_red[(kg * NQ + j) * kHd + 4 * g + d] = o[d][j];
   __syncthreads();
-  const int dim = tid;  // one output dim per thread
-  float lsum[NQ], osum[NQ];
+  float lsum[NQ];
 #pragma unroll
-  for (int j = 0; j < NQ; ++j) {
-    lsum[j] = ((red_s[0][j] + red_s[1][j]) + red_s[2][j]) + red_s[3][j];
-    osum[j] = ((o_red[(0 * NQ + j) * kHd + dim] + o_red[(1 * NQ + j) * kHd + dim]) + o_red[(2 * NQ + j) * kHd + dim]) +
-              o_red[(3 * NQ + j) * kHd + dim];
-  }
+  for (int j = 0; j < NQ; ++j) lsum[j] = ((red_s[0][j] + red_s[1][j]) + red_s[2][j]) + red_s[3][j];
   const size_t ld_out = static_cast<size_t>(p.n_heads) * kHd;
   if (n_split_b == 1) {
 #pragma unroll
-    for (int j = 0; j < NQ; ++j)
-      if (j < nq) p.out[(static_cast<size_t>(b) * nq + j) * ld_out + h * kHd + dim] = f32_to_bf16_bits(osum[j] / lsum[j]);
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int dim = warp * 32 + t * 16 + gq + (q >= 2 ? 8 : 0), j = 2 * tq + (q & 1);
+        if (j < nq) {
+          const float lj = ((red_s[0][j] + red_s[1][j]) + red_s[2][j]) + red_s[3][j];
+          p.out[(static_cast<size_t>(b) * nq + j) * ld_out + h * kHd + dim] = f32_to_bf16_bits(o[t][q] / lj);
+        }
+      }
     return;
   }
   // several splits: write this split's (m, l, o), the last CTA of the pair merges them
@@ -309,7 +342,12 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
   float* po = p.part_o + (pair * p.n_split + split) * NQ * kHd;
   float* pml = p.part_ml + (pair * p.n_split + split) * NQ * 2;
 #pragma unroll
-  for (int j = 0; j < NQ; ++j) po[j * kHd + dim] = osum[j];
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int dim = warp * 32 + t * 16 + gq + (q >= 2 ? 8 : 0), j = 2 * tq + (q & 1);
+      if (j < NQ) po[j * kHd + dim] = o[t][q];
+    }
 #pragma unroll
   for (int j = 0; j < NQ; ++j)
     if (tid == j) {  // (a loop, not m[tid]: register arrays take constant indices)
@@ -322,6 +360,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
   __syncthreads();
   if (!last_s) return;
   __threadfence();
+  const int dim = tid;  // the merge: one output dim per thread
   const float* po0 = p.part_o + pair * p.n_split * NQ * kHd;
   const float* pml0 = p.part_ml + pair * p.n_split * NQ * 2;
 #pragma unroll
@@ -341,10 +380,11 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
   if (tid == 0) p.counters[pair] = 0;  // ready for the next call on this workspace
 }
 
-// Dynamic shared memory of one CTA: the tile ring, the queries, the weights.
+// Dynamic shared memory of one CTA: the tile ring, the queries, the weights (bf16 high and low parts).
 static size_t attention_smem(int nq_t, int stages) {
+  (void)nq_t;
   return static_cast<size_t>(stages) * 2 * kTileBytes + static_cast<size_t>(2) * kQRows * 128 +
-         static_cast<size_t>(kTile) * nq_t * 4 + 1024;
+         static_cast<size_t>(2) * 8 * kTile * 2 + 1024;
 }
 
 template <int NQ, int STAGES>
