@@ -44,6 +44,7 @@ constexpr int kHd = 128;          // head dim
 constexpr int kTile = 64;         // cache positions per tile
 constexpr int kTileBytes = kTile * kHd * 2;  // 16 KB per K or V tile
 constexpr int kAttnThreads = 128;
+constexpr int kPRow = kTile + 8;  // bf16 elements per row of the softmax-weight buffers
 constexpr int kQRows = 16;        // the queries padded to the MMA's N (16)
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -58,9 +59,11 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // the queries as the MMA's B operand: bf16 [2 k-blocks][16 rows][64], 128-byte swizzle
   uint8_t* q_mma = smem + STAGES * 2 * kTileBytes;
-  // the tile's softmax weights as bf16 high and low parts, [8 queries][64 positions] each
+  // the tile's softmax weights as bf16 high and low parts, [8 queries][64
+  // positions] each, rows kPRow elements apart (16 bytes of padding: the PV
+  // fragment loads of the 8 queries then hit 8 different bank groups)
   uint16_t* p_hi = reinterpret_cast<uint16_t*>(q_mma + 2 * kQRows * 128);
-  uint16_t* p_lo = p_hi + 8 * kTile;
+  uint16_t* p_lo = p_hi + 8 * kPRow;
   __shared__ __align__(8) uint64_t full_bar[STAGES];
   __shared__ __align__(8) uint64_t s_bar;  // the tile's scores are in TMEM
   __shared__ __align__(8) uint64_t done_bar;  // every MMA of this CTA has completed (before TMEM is freed)
@@ -212,8 +215,8 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
         l_part[j] = l_part[j] * alpha[j] + pj;
         // bf16 high and low parts: p_hi + p_lo = pj to 2^-18 of it
         const uint16_t hi = f32_to_bf16_bits(pj);
-        p_hi[j * kTile + key] = hi;
-        p_lo[j * kTile + key] = f32_to_bf16_bits(pj - bf16_bits_to_f32(hi));
+        p_hi[j * kPRow + key] = hi;
+        p_lo[j * kPRow + key] = f32_to_bf16_bits(pj - bf16_bits_to_f32(hi));
       }
       m[j] = mn;
     }
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
       for (int ks = 0; ks < kTile / 16; ++ks) {
         uint32_t bh0 = 0, bh1 = 0, bl0 = 0, bl1 = 0;  // P^T: positions 16 ks + 2 tq (+1) and +8, query gq
         if (gq < NQ) {
-          const int pp = gq * kTile + 16 * ks + 2 * tq;
+          const int pp = gq * kPRow + 16 * ks + 2 * tq;
           bh0 = *reinterpret_cast<const uint32_t*>(p_hi + pp);
           bh1 = *reinterpret_cast<const uint32_t*>(p_hi + pp + 8);
           bl0 = *reinterpret_cast<const uint32_t*>(p_lo + pp);
@@ -384,7 +387,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attention_kernel(const __
 static size_t attention_smem(int nq_t, int stages) {
   (void)nq_t;
   return static_cast<size_t>(stages) * 2 * kTileBytes + static_cast<size_t>(2) * kQRows * 128 +
-         static_cast<size_t>(2) * 8 * kTile * 2 + 1024;
+         static_cast<size_t>(2) * 8 * kPRow * 2 + 1024;
 }
 
 template <int NQ, int STAGES>
