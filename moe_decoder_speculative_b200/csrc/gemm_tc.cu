@@ -556,13 +556,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
           }
         };
-        for (int c0 = 0; c0 < S.M; c0 += 32) {
-          uint32_t d[32];
-          tmem_ld32(tl + c0, d);
+        // Four logits per TMEM load in a rolled loop: a fully unrolled pass
+        // over 32 logits (each with its insertion network) did not fit the
+        // instruction cache and stalled on instruction fetch.
+#pragma unroll 1
+        for (int c0 = 0; c0 < S.M; c0 += 4) {
+          uint32_t d[4];
+          tmem_ld4(tl + c0, d);
           tmem_ld_wait();
           if (tvalid) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
+            for (int j = 0; j < 4; ++j) {
               const int e = c0 + j;
               if (e >= S.M) continue;
               float v = __uint_as_float(d[j]);
