@@ -49,11 +49,6 @@ __device__ __forceinline__ void prefetch_share(const L2Prefetch& pf) {
   }
 }
 
-// (value, index) pair comparison: larger value wins, equal values -> lower index.
-__device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
-  return v > bv || (v == bv && i < bi);
-}
-
 // Order key of a logit: larger logits give larger keys, -0 and +0 the same
 // key, and NaN the smallest key of all (below -inf), so that a NaN is only
 // ever selected when a row has fewer than k numbers.
