@@ -15,7 +15,7 @@ enum { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_ARGMAX = 2, EPI_SWIGLU_ROWS = 3, E
 enum { MODE_SINGLE = 0, MODE_GATEUP = 1, MODE_KPAIR = 2, MODE_MPAIR = 3, MODE_TGATEUP = 4, MODE_TPAIR = 5,
        MODE_TROUTE = 6,  // 128 token rows x the M (<= 256) router rows, one accumulator
        MODE_TLM = 7 };   // CTA pairs: 256 token rows x 256 LM-head rows (128 of each per CTA)
-enum { GEMM_MOE_DECODE = 0, GEMM_MOE_PREFILL = 1, GEMM_LM = 2, GEMM_LM_WIDE = 3 };
+enum { GEMM_MOE_DECODE = 0, GEMM_MOE_PREFILL = 1, GEMM_LM = 2, GEMM_LM_WIDE = 3, GEMM_MOE_DECODE_FEW = 4 };
 
 // B-operand TMA box height (rows) of each tile configuration; the host builds
 // the B tensor maps with it.  Whole 128-row token tiles in one box matter: on

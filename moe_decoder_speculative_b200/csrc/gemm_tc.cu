@@ -32,7 +32,8 @@
 // shared-memory ring.  A set may depend on an earlier one (the down projection
 // of expert e on the gate/up of expert e): its units wait, with a bounded
 // acquire-poll, until the epilogue warps of every unit of that group have
-// released their stores.  Claims are in list order and only running CTAs
+// released their stores (with few rows, the unit's first stages take their
+// weights before that wait).  Claims are in list order and only running CTAs
 // claim, so every unit waited on is already held by a running CTA: no
 // deadlock whatever the residency.
 //
@@ -78,7 +79,9 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 }  // namespace
 
-template <int BN, int STAGES, int NB, bool LM, int BBOX>
+// DEPW: a unit that must wait for the group it reads from issues its first
+// stages' weights before that wait (they do not depend on it).
+template <int BN, int STAGES, int NB, bool LM, int BBOX, bool DEPW>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams p) {
   constexpr int kBBox = BBOX;  // B rows per TMA box (the B tensor maps are built with this box height)
   static_assert(BBOX % 8 == 0 && BBOX <= BN, "BBOX");
@@ -351,26 +354,61 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         if (u < 0) break;
         const UnitInfo ui = decode(u);
         const GemmSet& S = p.set[ui.set];
+        const int nstage = unit_stages(S);
+        int pre_u = 0;  // DEPW: stages of this unit whose weights went out before its dependency wait
         if (S.dep_set >= 0) {  // wait until the group this unit reads from is complete
           const int gd = set_base[S.dep_set] + ui.gi;
           const int target = 4 * group_units(gd);
           const int* flag = p.sched + 1 + gd;
-          while (ld_acquire_gpu(flag) < target) {
-            __nanosleep(64);
-            if (*static_cast<volatile int*>(&abort_s) || globaltimer_ns() > deadline) {
-              if (!abort_s) {
-                abort_s = 1;
-                atomicOr(p.err, kErrTimeout);
+          if constexpr (DEPW) {
+            const int stage_u = stage;
+            if (ld_acquire_gpu(flag) < target) {
+              // HBM keeps streaming this unit's weights while the group finishes.
+              for (const int want = min(STAGES, nstage); pre_u < want; ++pre_u) {
+                if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_s, p.err, deadline)) {
+                  ok = false;
+                  break;
+                }
+                issue_stage(S, ui, pre_u, stage, true, false);
+                fills[stage]++;
+                if (++stage == STAGES) {
+                  stage = 0;
+                  phase ^= 1u;
+                }
               }
-              ok = false;
-              break;
+              while (ok && ld_acquire_gpu(flag) < target) {
+                __nanosleep(64);
+                if (*static_cast<volatile int*>(&abort_s) || globaltimer_ns() > deadline) {
+                  if (!abort_s) {
+                    abort_s = 1;
+                    atomicOr(p.err, kErrTimeout);
+                  }
+                  ok = false;
+                }
+              }
             }
+            fence_proxy_async_global();
+            // The token rows of those stages (also after an abort, so that every
+            // armed barrier completes and the drain below ends).
+            for (int ks = 0; ks < pre_u; ++ks) issue_stage(S, ui, ks, (stage_u + ks) % STAGES, false, true);
+            if (!ok) break;
+          } else {
+            while (ld_acquire_gpu(flag) < target) {
+              __nanosleep(64);
+              if (*static_cast<volatile int*>(&abort_s) || globaltimer_ns() > deadline) {
+                if (!abort_s) {
+                  abort_s = 1;
+                  atomicOr(p.err, kErrTimeout);
+                }
+                ok = false;
+                break;
+              }
+            }
+            if (!ok) break;
+            fence_proxy_async_global();
           }
-          if (!ok) break;
-          fence_proxy_async_global();
         }
-        const int nstage = unit_stages(S);
-        for (int ks = 0; ks < nstage; ++ks) {
+        for (int ks = pre_u; ks < nstage; ++ks) {
           const bool pre = (it == 0 && ks < npre);  // weights already issued before the wait
           if (!pre && !mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_s, p.err, deadline)) {
             ok = false;
@@ -804,14 +842,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 // ---------------------------------------------------------------------------
 // host-side launch
 // ---------------------------------------------------------------------------
-template <int BN, int STAGES, int NB, bool LM, int BBOX>
+template <int BN, int STAGES, int NB, bool LM, int BBOX, bool DEPW = false>
 static cudaError_t launch_gemm_impl(const GemmParams& p, int grid, cudaStream_t stream) {
   constexpr int STAGE_BYTES = ((!LM && BN == 32) ? 4 : 2) * kATileBytes + NB * BN * 128;  // as in the kernel
   constexpr int EXTRA = LM ? 4 * 32 * 33 * 4 : 0;  // argmax epilogue transpose buffers
   constexpr int SMEM = STAGES * STAGE_BYTES + EXTRA + 1024;
   // the kernel's static shared memory is 9,216 bytes (ptxas); the opt-in limit is 227 KB
   static_assert(SMEM + 9216 <= 227 * 1024, "shared memory (dynamic + static)");
-  auto kern = gemm_tc_kernel<BN, STAGES, NB, LM, BBOX>;
+  auto kern = gemm_tc_kernel<BN, STAGES, NB, LM, BBOX, DEPW>;
   static thread_local int configured_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -824,13 +862,15 @@ static cudaError_t launch_gemm_impl(const GemmParams& p, int grid, cudaStream_t 
 }
 
 // Tile configurations:
-//   GEMM_MOE_DECODE   BN = 32, two B k-block slots, 5 stages of 40 KB
+//   GEMM_MOE_DECODE   BN = 32, two k-blocks per stage (3D boxes), 3 stages of 72 KB
+//   GEMM_MOE_DECODE_FEW  the same, the down units' weights issued before their dependency wait
 //   GEMM_MOE_PREFILL  BN = 128, one B slot, 4 stages of 48 KB (tokens-on-M modes)
 //   GEMM_LM           BN = 128, one B slot, 4 stages of 48 KB (MODE_MPAIR), 16-row token boxes
 //   GEMM_LM_WIDE      the same with 128-row token boxes, for 128 or more tokens
 cudaError_t launch_gemm(int config, const GemmParams& p, int grid, cudaStream_t stream) {
   switch (config) {
     case GEMM_MOE_DECODE: return launch_gemm_impl<32, 3, 2, false, kDecodeBBox>(p, grid, stream);
+    case GEMM_MOE_DECODE_FEW: return launch_gemm_impl<32, 3, 2, false, kDecodeBBox, true>(p, grid, stream);
     case GEMM_MOE_PREFILL: return launch_gemm_impl<128, 4, 1, false, kPrefillBBox>(p, grid, stream);
     case GEMM_LM: return launch_gemm_impl<128, 4, 1, true, kLmBBox>(p, grid, stream);
     case GEMM_LM_WIDE: return launch_gemm_impl<128, 4, 1, true, kLmWideBBox>(p, grid, stream);
