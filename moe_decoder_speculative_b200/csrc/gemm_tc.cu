@@ -264,11 +264,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       fills[ks]++;
     }
   }
-
-  pdl_wait();  // the group sizes and the B operands come from the previous kernels
-
-  // ---- group table (every CTA builds the same one) -----------------------
-  if (tid == 0) {
+  // A decode CTA without an early unit takes its first dynamic claim before
+  // the wait (the counter was zeroed before the step's first kernel), so the
+  // claim's round trip overlaps the wait instead of following the group table.
+  int pre_claim = -1;
+  if (kSwapAB && warp == 0 && lane == 0 && !early && p.sched) pre_claim = atomicAdd(p.sched, 1);
+  if (tid == 0) {  // set offsets of the group table: kernel parameters only
     int b = 0;
     for (int s = 0; s < p.nsets; ++s) {
       set_base[s] = b;
@@ -277,6 +278,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     set_base[p.nsets] = b;
   }
   __syncthreads();
+
+  pdl_wait();  // the group sizes and the B operands come from the previous kernels
+
+  // ---- group table (every CTA builds the same one) -----------------------
   const int ng = set_base[p.nsets];
   for (int g = tid; g < ng; g += kThreads) {
     int s = 0;
@@ -346,6 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         int u;
         if (it == 0 && early)
           u = static_cast<int>(blockIdx.x);
+        else if (it == 0 && pre_claim >= 0)
+          u = nstatic + pre_claim;
         else
           u = p.sched ? nstatic + atomicAdd(p.sched, 1) : static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
         if (u >= total_units) u = -1;
