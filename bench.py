@@ -440,48 +440,56 @@ def run_ours(args):
         # ---- end to end through the public API with host buffers ----
         # Every step copies its inputs (hidden rows, drafts) from pinned host
         # memory and reads its results (accepted, next token, emitted) back,
-        # all inside the timed region.  The inputs are double-buffered: step
-        # i+1's copy runs on a copy stream while step i computes, and step i+1
-        # waits for it; the results come back in one copy of the plan's
-        # contiguous result block.
+        # all inside the timed region.  Two plans (same weights, their own
+        # workspaces and result blocks) and two input buffers alternate: after
+        # step i a copy stream reads step i's results back in one copy of its
+        # plan's contiguous result block and then brings in step i+2's inputs,
+        # while step i+1 computes; step i+2 waits for both copies.
         hid_h = torch.from_numpy(inp["hidden"].view(np.int16)).pin_memory()
         dr_h = torch.from_numpy(drafts_np).pin_memory()
         hid_d = [torch.empty_like(hid_h, device=dev) for _ in range(2)]
         dr_d = [torch.empty_like(dr_h, device=dev) for _ in range(2)]
+        plans = [plan, bd.VerifyPlan(shape, layers, w_lm, w.B, w.K, dev)]
         if args.graph:
-            e2e_graph = [bd.VerifyGraph(plan, hid_d[i].view(torch.bfloat16), dr_d[i]) for i in range(2)]
+            e2e_graph = [bd.VerifyGraph(plans[i], hid_d[i].view(torch.bfloat16), dr_d[i]) for i in range(2)]
             e2e_step = lambda i: e2e_graph[i]()
         else:
             e2e_graph = None
-            e2e_step = lambda i: plan(hid_d[i].view(torch.bfloat16), dr_d[i])
-        res_h = torch.empty_like(plan.results, device="cpu").pin_memory()
+            e2e_step = lambda i: plans[i](hid_d[i].view(torch.bfloat16), dr_d[i])
+        res_h = [torch.empty_like(plan.results, device="cpu").pin_memory() for _ in range(2)]
         copy_stream = torch.cuda.Stream(device=dev)
         in_ready = [torch.cuda.Event() for _ in range(2)]
         step_done = [torch.cuda.Event() for _ in range(2)]
 
-        def h2d(i):  # step i's inputs, once the step that last read that buffer (i - 2) is done
-            b = i % 2
+        def h2d(b):  # inputs into buffer b (the copy stream has waited for their last reader)
             with torch.cuda.stream(copy_stream):
-                if i >= 2:
-                    copy_stream.wait_event(step_done[b])
                 hid_d[b].copy_(hid_h, non_blocking=True)
                 dr_d[b].copy_(dr_h, non_blocking=True)
                 in_ready[b].record(copy_stream)
 
+        for b in range(2):  # untimed: the second plan's first steps
+            h2d(b)
+            stream.wait_event(in_ready[b])
+            e2e_step(b)
+        plans[1].sync_status()
         barrier()
         torch.cuda.synchronize()
         ev4, ev5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ev4.record(stream)
         copy_stream.wait_stream(stream)
-        h2d(0)
+        for b in range(min(2, args.steps)):
+            h2d(b)
         for i in range(args.steps):
             b = i % 2
             stream.wait_event(in_ready[b])
             e2e_step(b)
             step_done[b].record(stream)
-            if i + 1 < args.steps:
-                h2d(i + 1)
-            res_h.copy_(plan.results, non_blocking=True)
+            with torch.cuda.stream(copy_stream):
+                copy_stream.wait_event(step_done[b])
+                res_h[b].copy_(plans[b].results, non_blocking=True)
+            if i + 2 < args.steps:
+                h2d(b)
+        stream.wait_stream(copy_stream)
         ev5.record(stream)
         torch.cuda.synchronize()
         ms_e2e = ev4.elapsed_time(ev5)
@@ -540,7 +548,7 @@ def run_ours(args):
         "kernels": kernels,
         "instrumented_ms_per_step": ms_instr / K,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(hid_h.numel() * 2 + dr_h.numel() * 4),
-                "d2h_bytes_per_step": int(res_h.numel() * 4)},
+                "d2h_bytes_per_step": int(res_h[0].numel() * 4)},
         "gpu_launches": int(launches),
         "clocks": clk,
         "touched_experts": touched,
@@ -564,7 +572,7 @@ def run_ours(args):
                                          f"accept, one pass, {dt:.1f} s"}
     if rank == 0:
         print(json.dumps(out))
-    plan = graph = e2e_graph = step = e2e_step = None
+    plan = plans = graph = e2e_graph = step = e2e_step = None
     if world > 1:
         dist.destroy_process_group()
     return 0
