@@ -23,6 +23,34 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
   }
 }
 
+__device__ __forceinline__ uint64_t pack2f(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 unpack2f(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return make_float2(lo, hi);
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// The fp32 pair of one bf16x2 word: (element 2i, element 2i+1).
+__device__ __forceinline__ uint64_t bf16x2_pair(uint32_t w) {
+  return pack2f(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+// acc += x . w over 8 bf16 elements as two fp32 partial sums, element 2i
+// into the low half and 2i+1 into the high half (one packed FMA per pair).
+__device__ __forceinline__ uint64_t dot8_pairs(const uint4& x, const uint4& w, uint64_t acc) {
+  acc = ffma2(bf16x2_pair(x.x), bf16x2_pair(w.x), acc);
+  acc = ffma2(bf16x2_pair(x.y), bf16x2_pair(w.y), acc);
+  acc = ffma2(bf16x2_pair(x.z), bf16x2_pair(w.z), acc);
+  return ffma2(bf16x2_pair(x.w), bf16x2_pair(w.w), acc);
+}
+
 // This CTA's share of the L2 prefetch ranges: the concatenated ranges are cut
 // into gridDim.x equal slices (16-byte multiples), issued as 64 KB bulk
 // prefetches by one thread.  Fire and forget: nothing waits for them.
@@ -66,12 +94,13 @@ __device__ __forceinline__ uint32_t logit_key(float v) {
 // lower expert id first" (NaN last), and the element of rank j < k takes
 // slot j, so the slots are in descending logit order.  Eight consecutive
 // threads share one element, each comparing it with an eighth of the row,
-// and add their counts with shuffles.  Then warp r writes row r's slots: ids,
+// and add their counts with shuffles (topk_rank_block, ending with a block
+// barrier).  Then a warp writes each row's slots (topk_weights_rows): ids,
 // and the renormalised softmax weights exp(l_j - l_0) / sum_{i<k}
 // exp(l_i - l_0), the sum taken in slot order.  slot_s holds 8 entries per
-// row (k <= 8) and keeps the selected ids for the caller.
-__device__ void topk_rows_block(const float* ls, int E, int k, int nrows, int32_t* slot_s,
-                                int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+// row (k <= 8) and keeps the selected ids for the caller.  topk_rows_block
+// does both with every warp of the block.
+__device__ void topk_rank_block(const float* ls, int E, int k, int nrows, int32_t* slot_s) {
   const int tid = threadIdx.x, lane = tid & 31;
   const int chunk = (E + 7) >> 3;
   const int items = nrows * E * 8;
@@ -98,8 +127,17 @@ __device__ void topk_rows_block(const float* ls, int E, int k, int nrows, int32_
     if (it < items && sub == 0 && cnt < k) slot_s[(q / E) * 8 + cnt] = e;
   }
   __syncthreads();
-  // lane j computes slot j's exponential; the sum adds them in slot order
-  for (int r = tid >> 5; r < nrows; r += blockDim.x >> 5) {  // whole warps: the shuffles see every lane
+}
+
+// The slots' renormalised softmax weights, after topk_rank_block: warp
+// w0 + i handles rows i, i + nw, ... (lane j computes slot j's exponential;
+// the sum adds them in slot order); whole warps call it.
+__device__ void topk_weights_rows(const float* ls, int E, int k, int nrows, const int32_t* slot_s,
+                                  int32_t* __restrict__ idx_out, float* __restrict__ w_out, int w0, int nw) {
+  const int lane = threadIdx.x & 31;
+  const int wi = (static_cast<int>(threadIdx.x) >> 5) - w0;
+  if (wi < 0 || wi >= nw) return;  // warp-uniform
+  for (int r = wi; r < nrows; r += nw) {  // whole warps: the shuffles see every lane
     const float* lr = ls + r * E;
     const int32_t* sl = slot_s + r * 8;
     const int e = lane < k ? sl[lane] : 0;
@@ -115,6 +153,12 @@ __device__ void topk_rows_block(const float* ls, int E, int k, int nrows, int32_
   }
 }
 
+__device__ void topk_rows_block(const float* ls, int E, int k, int nrows, int32_t* slot_s,
+                                int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+  topk_rank_block(ls, E, k, nrows, slot_s);
+  topk_weights_rows(ls, E, k, nrows, slot_s, idx_out, w_out, 0, static_cast<int>(blockDim.x >> 5));
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -122,6 +166,10 @@ __device__ void topk_rows_block(const float* ls, int E, int k, int nrows, int32_
 // the lower expert id, slots in descending order), weights =
 // exp(l_j - l_max) / sum_selected exp(l - l_max), which equals the softmax
 // over all E restricted to the kept experts and renormalised.
+// Every CUDA-core router takes the dot products in the same order: lane L
+// of a warp sums its 16-byte vectors L, L+32, ... as two fp32 partial sums
+// (even and odd elements, one packed f32x2 FMA per element pair), adds the
+// two, and the warp adds the lanes by an xor-shuffle tree.
 // A CTA of 8 warps owns R rows: the rows sit in shared memory, warp w computes
 // experts w, w+8, ... for all R rows (each router weight row is read once per
 // CTA, 16-byte loads), then the block selects the top-k of its rows by rank.
@@ -157,16 +205,18 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const uint16_t* __rest
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[r] = 0.f;
     const uint4* we = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e) * H);
+    uint64_t acc2[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc2[r] = 0ull;
     for (int c = lane; c < hv; c += 32) {
-      float wf[8];
-      bf16x8_to_f32(__ldg(we + c), wf);
+      const uint4 wv = __ldg(we + c);
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        float xf[8];
-        bf16x8_to_f32(reinterpret_cast<const uint4*>(xs + static_cast<size_t>(r) * H)[c], xf);
+      for (int r = 0; r < R; ++r) acc2[r] = dot8_pairs(reinterpret_cast<const uint4*>(xs + static_cast<size_t>(r) * H)[c], wv, acc2[r]);
+    }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[r] = fmaf(xf[j], wf[j], acc[r]);
-      }
+    for (int r = 0; r < R; ++r) {
+      const float2 pr = unpack2f(acc2[r]);
+      acc[r] = pr.x + pr.y;
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -253,16 +303,19 @@ __global__ void __launch_bounds__(256, 1) router_smem_kernel(const uint16_t* __r
 #pragma unroll
       for (int r = 0; r < R; ++r) acc[r] = 0.f;
       const uint4* we = reinterpret_cast<const uint4*>(wsm + static_cast<size_t>(e) * H);
+      uint64_t acc2[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) acc2[r] = 0ull;
       for (int c = lane; c < hv; c += 32) {
-        float wf[8];
-        bf16x8_to_f32(we[c], wf);
+        const uint4 wv = we[c];
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          float xf[8];
-          bf16x8_to_f32(reinterpret_cast<const uint4*>(xs + static_cast<size_t>(r) * H)[c], xf);
+        for (int r = 0; r < R; ++r)
+          acc2[r] = dot8_pairs(reinterpret_cast<const uint4*>(xs + static_cast<size_t>(r) * H)[c], wv, acc2[r]);
+      }
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[r] = fmaf(xf[j], wf[j], acc[r]);
-        }
+      for (int r = 0; r < R; ++r) {
+        const float2 pr = unpack2f(acc2[r]);
+        acc[r] = pr.x + pr.y;
       }
 #pragma unroll
       for (int r = 0; r < R; ++r) {
@@ -531,7 +584,8 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
   }
 
   // (2) router logits: warp w owns experts w, w+16, w+32, w+48 (one batch of
-  //     loads for E <= 64); each x vector is converted once and reused.
+  //     loads for E <= 64); each x vector is converted once and reused, and
+  //     the products go through packed f32x2 FMAs (even and odd partial sums).
   constexpr int EB = 4;
   const int nwarps = blockDim.x >> 5;
   for (int e0 = warp; e0 < E; e0 += nwarps * EB) {
@@ -555,24 +609,42 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
     for (int b = 0; b < EB; ++b)
 #pragma unroll
       for (int r = 0; r < R; ++r) acc[b][r] = 0.f;
+    uint64_t acc2[EB][R];
+#pragma unroll
+    for (int b = 0; b < EB; ++b)
+#pragma unroll
+      for (int r = 0; r < R; ++r) acc2[b][r] = 0ull;
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
       const int c = lane + 32 * v;
       if (c < hv) {
-        float xf[R][8];
+        uint64_t xp[R][4];
 #pragma unroll
-        for (int r = 0; r < R; ++r) bf16x8_to_f32(reinterpret_cast<const uint4*>(hs + static_cast<size_t>(r) * H)[c], xf[r]);
+        for (int r = 0; r < R; ++r) {
+          const uint4 xv = reinterpret_cast<const uint4*>(hs + static_cast<size_t>(r) * H)[c];
+          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) xp[r][i] = bf16x2_pair(xw[i]);
+        }
 #pragma unroll
         for (int b = 0; b < EB; ++b) {
-          float wf[8];
-          bf16x8_to_f32(wv[b][v], wf);
+          const uint32_t ww[4] = {wv[b][v].x, wv[b][v].y, wv[b][v].z, wv[b][v].w};
 #pragma unroll
-          for (int r = 0; r < R; ++r)
+          for (int i = 0; i < 4; ++i) {
+            const uint64_t wp = bf16x2_pair(ww[i]);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[b][r] = fmaf(xf[r][j], wf[j], acc[b][r]);
+            for (int r = 0; r < R; ++r) acc2[b][r] = ffma2(xp[r][i], wp, acc2[b][r]);
+          }
         }
       }
     }
+#pragma unroll
+    for (int b = 0; b < EB; ++b)
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float2 pr = unpack2f(acc2[b][r]);
+        acc[b][r] = pr.x + pr.y;
+      }
 #pragma unroll
     for (int b = 0; b < EB; ++b) {
       const int e = e0 + nwarps * b;
@@ -587,14 +659,17 @@ __global__ void __launch_bounds__(512) combine_route_kernel(
   }
   __syncthreads();
 
-  // (3) top-k
-  topk_rows_block(ls, E, k, nrows, sel_s, idx + static_cast<size_t>(row0) * k, wout + static_cast<size_t>(row0) * k);
+  // (3) top-k: the ranks by the whole block, then the weights by warps
+  //     0..R-1 while the last warp claims the slab rows (4)
+  topk_rank_block(ls, E, k, nrows, sel_s);
+  topk_weights_rows(ls, E, k, nrows, sel_s, idx + static_cast<size_t>(row0) * k, wout + static_cast<size_t>(row0) * k,
+                    0, R);
   if (!slab_counts) return;  // uniform across the CTA
 
   // (4) slab placement of the routed rows
-  __syncthreads();
-  if (tid < nrows * k) {
-    const int r = tid / k, j = tid % k;
+  const int ct = tid - (static_cast<int>(blockDim.x) - 32);  // lane of the last warp
+  if (ct >= 0 && ct < nrows * k) {
+    const int r = ct / k, j = ct % k;
     const int e = sel_s[r * 8 + j];
     int p = -1;
     if (e >= 0 && e < E) {
