@@ -253,6 +253,21 @@ def oracle_step(oracle, w, inp, drafts, S):
     return int(np.sum(st["accepted"] + 1))
 
 
+def oracle_single_thread(oracle):
+    """Seconds of one oracle verify step on one host thread, for the tiny
+    workload and the model-shape batch-1 layer.  It leaves the oracle on one
+    thread, so it runs after every other oracle timing."""
+    res = {}
+    for wid in (0, 1):
+        w = wl.workload(wid)
+        inp = wl.make_inputs(w)
+        drafts = np.zeros((w.B, w.K), np.int32)
+        t0 = time.perf_counter()
+        oracle.verify_step(inp["hidden"], drafts, w.B, w.K, inp["layers"], w.k, inp["w_lm"], n_threads=1)
+        res[w.name] = round(time.perf_counter() - t0, 4)
+    return res
+
+
 def oracle_sample_size(oracle, w, inp, budget_s):
     """Sequences per oracle step so that one step takes about budget_s seconds."""
     t0 = time.perf_counter()
@@ -570,6 +585,7 @@ def run_ours(args):
                                "kind": "oracle",
                                "sample": f"{S} of {w.B} sequences ({S * (w.K + 1)} rows) x {w.L} layers + LM head + "
                                          f"accept, one pass, {dt:.1f} s"}
+        out["cpu_baseline"]["single_thread_s_per_step"] = oracle_single_thread(oracle)
     if rank == 0:
         print(json.dumps(out))
     plan = plans = graph = e2e_graph = step = e2e_step = None
