@@ -392,7 +392,7 @@ mv::L2Prefetch lm_first_wave(const uint16_t* w_lm, int V, int H, uint64_t budget
 }
 
 #ifndef MV_PREFETCH_BUDGET_MB
-#define MV_PREFETCH_BUDGET_MB 32  // measured best of 0 / 32 / 64 / 96 MB on the concurrency-32 step
+#define MV_PREFETCH_BUDGET_MB 24  // measured best of 0 / 8 / 16 / 20 / 24 / 32 / 40 / 48 / 64 / 96 MB on the concurrency-32 step
 #endif
 constexpr uint64_t kPrefetchBudget = static_cast<uint64_t>(MV_PREFETCH_BUDGET_MB) << 20;
 
