@@ -360,10 +360,24 @@ int gemm_grid(int64_t units) {
 // The weights the grouped MoE GEMM of a layer streams first, in claim order
 // (shared gate/up, then the routed gate/up of experts 0, 1, ...), up to
 // `budget` bytes: what a kernel running before it can pull into L2 while HBM
-// is otherwise idle.
-mv::L2Prefetch moe_first_wave(const mv_moe_shape& s, const mv_moe_weights& w, uint64_t budget) {
+// is otherwise idle.  A batch of T rows with T * k <= E touches only a few
+// experts, unknown before its routing, so there the shared expert (gate, up
+// and down) is all that is prefetched.
+mv::L2Prefetch moe_first_wave(const mv_moe_shape& s, const mv_moe_weights& w, uint64_t budget, int64_t T = 0) {
   mv::L2Prefetch pf{};
   const uint64_t sh = static_cast<uint64_t>(s.I_shared) * s.H * 2;
+  if (T > 0 && T * s.k <= s.E) {  // few rows: the shared expert only (which routed experts is unknown)
+    if (s.I_shared > 0 && budget >= 3 * sh) {
+      pf.ptr[0] = w.ws_gate;
+      pf.bytes[0] = sh;
+      pf.ptr[1] = w.ws_up;
+      pf.bytes[1] = sh;
+      pf.ptr[2] = w.ws_down;
+      pf.bytes[2] = sh;
+      pf.n = 3;
+    }
+    return pf;
+  }
   if (s.I_shared > 0 && budget >= 2 * sh) {
     pf.ptr[pf.n] = w.ws_gate;
     pf.bytes[pf.n++] = sh;
@@ -1037,7 +1051,7 @@ static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts,
       a.w = tw_buf;
       a.err = err;
       a.timeout_ns = timeout_ns();
-      a.pf = moe_first_wave(*shape, layers[0], kPrefetchBudget);
+      a.pf = moe_first_wave(*shape, layers[0], kPrefetchBudget, T);
       a.slab_counts = slab_counts(0);
       a.inv_out = slab_inv(0);
       a.ent_out = fw.ent;
@@ -1090,7 +1104,7 @@ static mv_status verify_step_impl(const uint16_t* hidden, const int32_t* drafts,
           a.w = tw_n;
           a.err = err;
           a.timeout_ns = timeout_ns();
-          a.pf = moe_first_wave(*shape, wn, kPrefetchBudget);
+          a.pf = moe_first_wave(*shape, wn, kPrefetchBudget, T);
           a.slab_counts = slab_counts(l + 1);
           a.inv_out = slab_inv(l + 1);
           a.ent_out = fw.ent;
